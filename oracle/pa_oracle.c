@@ -1,0 +1,344 @@
+/*
+ * pa_oracle.c -- plain, slow, fp64 CPU oracle for paged-KV attention.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package's smoke check and the
+ * benchmark's CPU-baseline leg load this library. The product (the CUDA
+ * library and its Python binding) never calls, links or imports it, and it
+ * shares no code, header or table with the CUDA kernels.
+ *
+ * What each function follows (cited by page title and section):
+ *
+ *  [KV]  page "字节跳动 AI Infra (2)", question "KV Cache原理与优化" (KV cache
+ *        principle), the per-step formulas: the new token's K_t/V_t are
+ *        appended to the cache, K_cache = concat(K_cache, K_t), and the step's
+ *        output is softmax(Q_t . K_cache^T / sqrt(d)) . V_cache, shape [1, d].
+ *  [PG]  same page, question "vLLM与PagedAttention的原理" (PagedAttention
+ *        principle): a pool of fixed-size physical blocks (16 tokens of K/V
+ *        each in the example), a per-request block table mapping logical block
+ *        i to a physical block id, and the kernel sketch that finds a block's
+ *        keys at k_cache + physical_block * block_size * head_dim.
+ *  [GQA] page "LLM推理优化", section 1.3 (KV cache optimisation strategies):
+ *        under GQA several query heads share one K/V head; under MQA all do.
+ *  [FD]  page "字节跳动 AI Infra (2)", question "推理加速的综合策略有哪些",
+ *        table of algorithm-level optimisations, row FlashDecoding: decode is
+ *        parallelised by splitting along the KV length.
+ *  [CP]  page "vLLM框架是怎么做推理加速的", section 3 (Chunked Prefill): a
+ *        prompt is cut into chunks (512 tokens by default) that attend over
+ *        the cache; page "LLM推理优化", section 2.3: prefill attention is
+ *        causal (flash_attn_func(..., causal=True)).
+ *
+ * Readings taken where the pages are silent (each also listed in the design
+ * notes):
+ *  - Cache layout [num_blocks][num_kv_heads][block_size][head_dim]; the page's
+ *    pointer formula is the num_kv_heads == 1 case of it.
+ *  - Query head h reads K/V head h / (H_q / H_kv) (contiguous groups).
+ *  - The scale is a parameter (the pages use 1/sqrt(d)).
+ *  - context_lens[b] counts the valid tokens of sequence b, including the one
+ *    just appended; table entries and slots past it are never read.
+ *  - A sequence with no tokens yields out = 0 and lse = -inf.
+ *  - Chunk queries are bottom-right aligned: query i of a chunk of C queries
+ *    over ctx tokens sits at position ctx - C + i and attends keys 0..that
+ *    position. The chunk's own K/V are already in the cache.
+ *  - Stored values (fp32, or bf16 bit patterns) are widened exactly to double;
+ *    everything after that is plain fp64 arithmetic.
+ *  - softmax is evaluated as exp(s - max s) / sum exp(s - max s), which is the
+ *    definition multiplied through by exp(-max s) / exp(-max s).
+ *
+ * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -fPIC -shared.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_F32 = 0, OR_BF16 = 1 };
+enum { OR_OK = 0, OR_BAD_SLOT = 1, OR_BAD_BLOCK = 2, OR_BAD_ARG = 3, OR_NO_MEM = 4 };
+
+/* A stored element, widened exactly to double. bf16 is the top half of an
+ * IEEE binary32, so shifting its 16 bits up gives the same number as a float. */
+static double stored(const void *base, int64_t i, int dtype)
+{
+    if (dtype == OR_F32) return (double)((const float *)base)[i];
+    uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* One sequence's view of the pool: where its block table row is and which
+ * K/V head is being read. */
+typedef struct {
+    const void *k_cache, *v_cache;
+    int dtype;
+    const int32_t *table_row; /* block_tables[b][0 .. max_blocks_per_seq) */
+    int max_blocks;
+    int H_kv, D, bs;
+    int64_t NB;
+    int kv_head;
+} paged_seq;
+
+/* [PG] element index of K/V[position j][dim 0] of this sequence and head:
+ * logical block j / bs is looked up in the table; the token sits at offset
+ * j % bs inside the physical block. Returns -1 for an id outside the pool. */
+static int64_t token_base(const paged_seq *s, int64_t j)
+{
+    int64_t logical_block = j / s->bs;
+    int64_t offset = j % s->bs;
+    if (logical_block >= s->max_blocks) return -1;
+    int64_t phys = s->table_row[logical_block];
+    if (phys < 0 || phys >= s->NB) return -1;
+    return ((phys * s->H_kv + s->kv_head) * s->bs + offset) * s->D;
+}
+
+/* [KV] one query vector q[0..D) against the sequence's keys at positions
+ * [j0, j1): scores s_j = scale * (q . K_j), weights softmax(s), output
+ * sum_j softmax(s)_j V_j, and lse = log sum_j exp(s_j).
+ * sbuf must hold j1 - j0 doubles. */
+static int attend(double *o, double *lse, const double *q, const paged_seq *s,
+                  int64_t j0, int64_t j1, double scale, double *sbuf)
+{
+    const int D = s->D;
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (j1 <= j0) {
+        *lse = -INFINITY;
+        return OR_OK;
+    }
+    double m = -INFINITY;
+    for (int64_t j = j0; j < j1; ++j) {
+        int64_t base = token_base(s, j);
+        if (base < 0) return OR_BAD_BLOCK;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += q[d] * stored(s->k_cache, base + d, s->dtype);
+        double sc = scale * dot;
+        sbuf[j - j0] = sc;
+        if (sc > m) m = sc;
+    }
+    double denom = 0.0;
+    for (int64_t j = j0; j < j1; ++j) {
+        double p = exp(sbuf[j - j0] - m);
+        sbuf[j - j0] = p;
+        denom += p;
+    }
+    for (int64_t j = j0; j < j1; ++j) {
+        int64_t base = token_base(s, j);
+        double w = sbuf[j - j0] / denom;
+        for (int d = 0; d < D; ++d) o[d] += w * stored(s->v_cache, base + d, s->dtype);
+    }
+    *lse = m + log(denom);
+    return OR_OK;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* [KV]+[PG] the append step in paged form. For each new token t with slot
+ * s = slot_mapping[t] >= 0, the token's K/V rows for every K/V head are copied
+ * into physical block s / bs at offset s % bs. Negative slots are padding and
+ * are skipped. A slot past the pool returns OR_BAD_SLOT before anything is
+ * written. Element type does not matter: the copy is of bytes. */
+int oracle_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                             const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
+                             int head_dim, int block_size, int64_t num_blocks, int elem_bytes)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || elem_bytes <= 0)
+        return OR_BAD_ARG;
+    for (int64_t t = 0; t < num_tokens; ++t)
+        if (slot_mapping[t] >= num_blocks * (int64_t)block_size) return OR_BAD_SLOT;
+    const size_t row = (size_t)head_dim * (size_t)elem_bytes;
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t block = slot / block_size, offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            size_t src = ((size_t)t * num_kv_heads + h) * row;
+            size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) * row;
+            memcpy((char *)k_cache + dst, (const char *)key + src, row);
+            memcpy((char *)v_cache + dst, (const char *)value + src, row);
+        }
+    }
+    return OR_OK;
+}
+
+/* Shared argument checks for the attention entry points. */
+static int check_heads(int H_q, int H_kv, int D, int bs, int MB, int64_t NB)
+{
+    if (H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0 || D <= 0 || bs <= 0 || MB < 0 || NB <= 0)
+        return OR_BAD_ARG;
+    return OR_OK;
+}
+
+/* [KV]+[PG]+[GQA] decode: for every sequence b and query head h (or only the
+ * pairs with select[b*H_q+h] != 0), attend q[b][h] over positions
+ * [0, context_lens[b]) gathered through block_tables[b], reading K/V head
+ * h / (H_q/H_kv). out: [B][H_q][D] doubles; lse: [B][H_q] (may be NULL). */
+int oracle_decode(double *out, double *lse, const void *q, const void *k_cache,
+                  const void *v_cache, int dtype, const int32_t *block_tables,
+                  const int32_t *context_lens, int B, int H_q, int H_kv, int D, int bs, int MB,
+                  int64_t NB, double scale, const uint8_t *select)
+{
+    int rc = check_heads(H_q, H_kv, D, bs, MB, NB);
+    if (rc) return rc;
+    for (int b = 0; b < B; ++b)
+        if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)MB * bs) return OR_BAD_ARG;
+    const int group = H_q / H_kv;
+    int err = OR_OK;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : err)
+    for (int64_t bh = 0; bh < (int64_t)B * H_q; ++bh) {
+        if (select && !select[bh]) continue;
+        int b = (int)(bh / H_q), h = (int)(bh % H_q);
+        paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)b * MB, MB,
+                       H_kv, D, bs, NB, h / group};
+        double *qv = malloc(sizeof(double) * D);
+        double *sbuf = malloc(sizeof(double) * (context_lens[b] > 0 ? context_lens[b] : 1));
+        if (!qv || !sbuf) {
+            free(qv); free(sbuf);
+            err = OR_NO_MEM > err ? OR_NO_MEM : err;
+            continue;
+        }
+        for (int d = 0; d < D; ++d) qv[d] = stored(q, bh * D + d, dtype);
+        double l;
+        int r = attend(out + bh * D, &l, qv, &s, 0, context_lens[b], scale, sbuf);
+        if (lse) lse[bh] = l;
+        if (r > err) err = r;
+        free(qv);
+        free(sbuf);
+    }
+    return err;
+}
+
+/* [FD] the same decode restricted to KV partitions: partition p of sequence b
+ * covers positions [p*partition_tokens, min((p+1)*partition_tokens, ctx_b)).
+ * o_parts: [B][H_q][S][D], lse_parts: [B][H_q][S]; partitions past the end of
+ * a sequence hold o = 0, lse = -inf. */
+int oracle_decode_partials(double *o_parts, double *lse_parts, const void *q, const void *k_cache,
+                           const void *v_cache, int dtype, const int32_t *block_tables,
+                           const int32_t *context_lens, int B, int H_q, int H_kv, int D, int bs,
+                           int MB, int64_t NB, double scale, int partition_tokens, int S)
+{
+    int rc = check_heads(H_q, H_kv, D, bs, MB, NB);
+    if (rc) return rc;
+    if (partition_tokens <= 0 || S <= 0) return OR_BAD_ARG;
+    for (int b = 0; b < B; ++b)
+        if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)MB * bs ||
+            (int64_t)context_lens[b] > (int64_t)S * partition_tokens)
+            return OR_BAD_ARG;
+    const int group = H_q / H_kv;
+    int err = OR_OK;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : err)
+    for (int64_t bh = 0; bh < (int64_t)B * H_q; ++bh) {
+        int b = (int)(bh / H_q), h = (int)(bh % H_q);
+        paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)b * MB, MB,
+                       H_kv, D, bs, NB, h / group};
+        double *qv = malloc(sizeof(double) * D);
+        double *sbuf = malloc(sizeof(double) * partition_tokens);
+        if (!qv || !sbuf) {
+            free(qv); free(sbuf);
+            err = OR_NO_MEM > err ? OR_NO_MEM : err;
+            continue;
+        }
+        for (int d = 0; d < D; ++d) qv[d] = stored(q, bh * D + d, dtype);
+        for (int p = 0; p < S; ++p) {
+            int64_t j0 = (int64_t)p * partition_tokens;
+            int64_t j1 = j0 + partition_tokens;
+            if (j1 > context_lens[b]) j1 = context_lens[b];
+            int r = attend(o_parts + (bh * S + p) * D, lse_parts + bh * S + p, qv, &s, j0, j1,
+                           scale, sbuf);
+            if (r > err) err = r;
+        }
+        free(qv);
+        free(sbuf);
+    }
+    return err;
+}
+
+/* [FD] merge of partial results by log-sum-exp. With L = log sum_s exp(lse_s),
+ * out = sum_s exp(lse_s - L) o_s, which equals attention over the union of the
+ * partitions because each o_s is already normalised by its own exp(lse_s).
+ * Partitions with lse = -inf carry no weight; if all do, out = 0, lse = -inf.
+ * o_parts: [R][S][D], lse_parts: [R][S], out: [R][D], lse: [R]. */
+void oracle_lse_merge(double *out, double *lse, const double *o_parts, const double *lse_parts,
+                      int64_t R, int S, int D)
+{
+    for (int64_t r = 0; r < R; ++r) {
+        const double *ls = lse_parts + r * S;
+        double m = -INFINITY;
+        for (int p = 0; p < S; ++p)
+            if (ls[p] > m) m = ls[p];
+        for (int d = 0; d < D; ++d) out[r * D + d] = 0.0;
+        if (m == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double total = 0.0;
+        for (int p = 0; p < S; ++p) total += exp(ls[p] - m);
+        for (int p = 0; p < S; ++p) {
+            if (ls[p] == -INFINITY) continue;
+            double w = exp(ls[p] - m) / total;
+            for (int d = 0; d < D; ++d) out[r * D + d] += w * o_parts[(r * S + p) * D + d];
+        }
+        lse[r] = m + log(total);
+    }
+}
+
+/* [CP] chunked prefill. Chunk c owns query rows [qsl[c], qsl[c+1]) of q
+ * ([total_q][H_q][D]) and block_tables[c]; context_lens[c] is its total
+ * context (cached tokens plus the chunk's own C tokens, all in the cache).
+ * Query i attends positions [0, ctx - C + i] (causal, bottom-right aligned).
+ * out: [total_q][H_q][D]; lse: [total_q][H_q] (may be NULL); select as in
+ * oracle_decode over (row, head). */
+int oracle_prefill(double *out, double *lse, const void *q, const void *k_cache,
+                   const void *v_cache, int dtype, const int32_t *block_tables,
+                   const int32_t *context_lens, const int32_t *query_start_loc, int n_chunks,
+                   int H_q, int H_kv, int D, int bs, int MB, int64_t NB, double scale,
+                   const uint8_t *select)
+{
+    int rc = check_heads(H_q, H_kv, D, bs, MB, NB);
+    if (rc) return rc;
+    if (n_chunks < 0 || query_start_loc[0] != 0) return OR_BAD_ARG;
+    for (int c = 0; c < n_chunks; ++c) {
+        int64_t C = (int64_t)query_start_loc[c + 1] - query_start_loc[c];
+        if (C < 0 || context_lens[c] < C || (int64_t)context_lens[c] > (int64_t)MB * bs)
+            return OR_BAD_ARG;
+    }
+    const int64_t total_q = query_start_loc[n_chunks];
+    const int group = H_q / H_kv;
+    int err = OR_OK;
+#pragma omp parallel for schedule(dynamic, 4) reduction(max : err)
+    for (int64_t rh = 0; rh < total_q * H_q; ++rh) {
+        if (select && !select[rh]) continue;
+        int64_t row = rh / H_q;
+        int h = (int)(rh % H_q);
+        int c = 0;
+        while (query_start_loc[c + 1] <= row) ++c;
+        int64_t C = (int64_t)query_start_loc[c + 1] - query_start_loc[c];
+        int64_t i = row - query_start_loc[c];
+        int64_t pos = (int64_t)context_lens[c] - C + i; /* this query's position */
+        paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)c * MB, MB,
+                       H_kv, D, bs, NB, h / group};
+        double *qv = malloc(sizeof(double) * D);
+        double *sbuf = malloc(sizeof(double) * (pos + 1));
+        if (!qv || !sbuf) {
+            free(qv); free(sbuf);
+            err = OR_NO_MEM > err ? OR_NO_MEM : err;
+            continue;
+        }
+        for (int d = 0; d < D; ++d) qv[d] = stored(q, rh * D + d, dtype);
+        double l;
+        int r = attend(out + rh * D, &l, qv, &s, 0, pos + 1, scale, sbuf);
+        if (lse) lse[rh] = l;
+        if (r > err) err = r;
+        free(qv);
+        free(sbuf);
+    }
+    return err;
+}

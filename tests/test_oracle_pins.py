@@ -1,0 +1,424 @@
+"""Pins for the fp64 CPU oracle, against things other than the oracle itself:
+values the pages print, a library attention routine (torch's fp64
+scaled_dot_product_attention on contiguous K/V), closed forms, special cases
+and invariants that a dropped term, a wrong index or sign, or a transposed
+operand would break.
+
+Pages cited by title and section:
+* «字节跳动 AI Infra (2)», question «vLLM与PagedAttention的原理»: block pool,
+  block tables (A: 40 tokens -> [B2, B5, B7]; B: 20 tokens -> [B0, B4]),
+  beams sharing B1, B3 with a copy-on-write B6'.
+* same page, question «KV Cache原理与优化»: step-t formulas.
+* «LLM推理优化», section 1.2 (KV size example), 1.3 (GQA/MQA), 2.3 (causal),
+  3.2 (block counts).
+* «字节跳动 AI Infra (2)», FlashDecoding row: split along the KV length.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+F64 = torch.float64
+
+
+# ---------------------------------------------------------------------------
+# helpers (test-side, independent of the oracle's C code)
+# ---------------------------------------------------------------------------
+def place(seqs_k, seqs_v, tables, num_blocks, bs, dtype=torch.float32, fill=float("nan")):
+    """Write contiguous per-sequence K/V ([H_kv, ctx, D] each) into a fresh pool
+    following the given block tables; everything else holds ``fill``."""
+    H, _, D = seqs_k[0].shape
+    kc = torch.full((num_blocks, H, bs, D), fill, dtype=dtype)
+    vc = torch.full((num_blocks, H, bs, D), fill, dtype=dtype)
+    for k, v, row in zip(seqs_k, seqs_v, tables):
+        for j in range(k.shape[1]):
+            kc[row[j // bs], :, j % bs] = k[:, j].to(dtype)
+            vc[row[j // bs], :, j % bs] = v[:, j].to(dtype)
+    return kc, vc
+
+
+def pad_tables(rows, width, pad):
+    t = torch.full((len(rows), width), pad, dtype=torch.int32)
+    for i, r in enumerate(rows):
+        t[i, :len(r)] = torch.tensor(r, dtype=torch.int32)
+    return t
+
+
+def sdpa(q, k, v, scale, causal=False):
+    """torch's attention routine in fp64: q [H_q, Lq, D], k/v [H_kv, Lk, D]."""
+    return F.scaled_dot_product_attention(q[None].to(F64), k[None].to(F64), v[None].to(F64),
+                                          scale=scale, is_causal=causal,
+                                          enable_gqa=q.shape[0] != k.shape[0])[0]
+
+
+def random_paged(ctxs, H_q, H_kv, D, bs, seed, dtype=torch.float32, spare=3):
+    """Random contiguous K/V per sequence placed in a pool at random block ids."""
+    g = torch.Generator().manual_seed(seed)
+    need = [-(-c // bs) for c in ctxs]
+    NB = sum(need) + spare
+    perm = torch.randperm(NB, generator=g).tolist()
+    rows, at = [], 0
+    for n in need:
+        rows.append(perm[at:at + n])
+        at += n
+    pad = perm[-1]  # an unused id: every padded entry points at a NaN block
+    ks = [torch.randn(H_kv, c, D, generator=g).to(dtype) for c in ctxs]
+    vs = [torch.randn(H_kv, c, D, generator=g).to(dtype) for c in ctxs]
+    q = torch.randn(len(ctxs), H_q, D, generator=g).to(dtype)
+    kc, vc = place(ks, vs, rows, NB, bs, dtype)
+    MB = max(need + [1])
+    return q, ks, vs, kc, vc, pad_tables(rows, MB, pad), torch.tensor(ctxs, dtype=torch.int32)
+
+
+# ---------------------------------------------------------------------------
+# values the pages print
+# ---------------------------------------------------------------------------
+def test_kv_cache_size_example(golden):
+    ex = golden["kv_cache_size"]
+    n = oracle.kv_cache_bytes(ex["num_layers"], ex["num_heads"], ex["seq_len"], ex["head_dim"],
+                              ex["dtype_bytes"])
+    assert round(n / 1e9, 1) == ex["printed_gb"]
+    # the reading "GB = 10^9 bytes": the same count is exactly 10 GiB
+    assert n == 10 * 2 ** 30
+    # linear in every factor, and K and V both counted
+    assert oracle.kv_cache_bytes(1, 1, 1, 1, 1) == 2
+    assert oracle.kv_cache_bytes(80, 64, 8192, 128, 2) == 2 * n
+
+
+def test_block_counts_example(golden):
+    ex = golden["block_counts"]
+    counts = [oracle.blocks_needed(t, ex["block_size"]) for t, _ in ex["sequences"]]
+    assert counts == [c for _, c in ex["sequences"]]
+    assert sum(counts) == ex["printed_total"]
+    assert oracle.blocks_needed(0) == 0
+    assert oracle.blocks_needed(16) == 1 and oracle.blocks_needed(17) == 2
+
+
+def test_block_table_example_counts(golden):
+    ex = golden["block_tables"]
+    for req in ex["requests"].values():
+        assert oracle.blocks_needed(req["tokens"], ex["block_size"]) == len(req["table"])
+
+
+def test_block_table_example_gather(golden):
+    """Requests A and B of the diagram: with all keys equal the weights are
+    uniform, so the output is the mean of exactly the values the table
+    reaches. Each token's V carries its own position, so a wrong block or
+    offset changes the mean."""
+    ex = golden["block_tables"]
+    bs, NB, D = ex["block_size"], ex["pool"], 4
+    reqs = [ex["requests"]["A"], ex["requests"]["B"]]
+    ks = [torch.zeros(1, r["tokens"], D) for r in reqs]
+    vs = []
+    for i, r in enumerate(reqs):
+        pos = torch.arange(r["tokens"], dtype=torch.float32)
+        v = torch.stack([pos, pos * pos, torch.full_like(pos, i + 1.0), pos ** 3], dim=-1)
+        vs.append(v[None])
+    kc, vc = place(ks, vs, [r["table"] for r in reqs], NB, bs)
+    tables = pad_tables([r["table"] for r in reqs], 3, 3)  # B3 is not used by A or B
+    lens = torch.tensor([r["tokens"] for r in reqs], dtype=torch.int32)
+    q = torch.randn(2, 1, D)
+    out, lse = oracle.decode(q, kc, vc, tables, lens, 1.0)
+    for i, r in enumerate(reqs):
+        n = r["tokens"]
+        pos = np.arange(n, dtype=np.float64)
+        expect = [pos.mean(), (pos * pos).mean(), i + 1.0, (pos ** 3).mean()]
+        np.testing.assert_allclose(out[i, 0].numpy(), expect, rtol=1e-14, atol=1e-12)
+        assert lse[i, 0].item() == pytest.approx(math.log(n), abs=1e-14)
+
+
+def test_block_table_example_one_hot(golden):
+    """The diagram's request A: a query aligned with one key under a large
+    scale returns that key's value, for every position of the sequence."""
+    ex = golden["block_tables"]
+    bs, NB, D = ex["block_size"], ex["pool"], 8
+    A = ex["requests"]["A"]
+    g = torch.Generator().manual_seed(5)
+    k = torch.nn.functional.normalize(torch.randn(1, A["tokens"], D, generator=g), dim=-1)
+    v = torch.randn(1, A["tokens"], D, generator=g)
+    kc, vc = place([k], [v], [A["table"]], NB, bs)
+    tables = pad_tables([A["table"]], 3, 0)
+    for j in range(A["tokens"]):
+        q = k[0, j][None, None] * 1.0
+        out, _ = oracle.decode(q, kc, vc, tables, torch.tensor([A["tokens"]], dtype=torch.int32),
+                               1e4)
+        np.testing.assert_allclose(out[0, 0].numpy(), v[0, j].double().numpy(), atol=1e-9)
+
+
+def test_reshape_example_slots(golden):
+    """The new (last) token of request A lands in B7 at offset 7 (slot 119) and
+    of request B in B4 at offset 3 (slot 67); nothing else in the pool moves;
+    a negative slot is skipped."""
+    ex = golden["block_tables"]
+    bs, NB, H, D = ex["block_size"], ex["pool"], 2, 4
+    A, Bq = ex["requests"]["A"], ex["requests"]["B"]
+    slotA = A["table"][(A["tokens"] - 1) // bs] * bs + (A["tokens"] - 1) % bs
+    slotB = Bq["table"][(Bq["tokens"] - 1) // bs] * bs + (Bq["tokens"] - 1) % bs
+    assert (slotA, slotB) == (119, 67)
+    g = torch.Generator().manual_seed(1)
+    kc = torch.randn(NB, H, bs, D, generator=g)
+    vc = torch.randn(NB, H, bs, D, generator=g)
+    key = torch.randn(3, H, D, generator=g)
+    value = torch.randn(3, H, D, generator=g)
+    slots = torch.tensor([slotA, -1, slotB], dtype=torch.int64)
+    k2, v2 = kc.clone(), vc.clone()
+    oracle.reshape_and_cache(key, value, k2, v2, slots)
+    ek, ev = kc.clone(), vc.clone()
+    ek[7, :, 7], ev[7, :, 7] = key[0], value[0]
+    ek[4, :, 3], ev[4, :, 3] = key[2], value[2]
+    assert torch.equal(k2, ek) and torch.equal(v2, ev)
+
+
+def test_reshape_bytes_and_errors():
+    """bf16 rows are copied bit for bit; a slot past the pool is an error and
+    leaves the pool untouched."""
+    g = torch.Generator().manual_seed(2)
+    kc = torch.randn(4, 3, 16, 8, generator=g).to(torch.bfloat16)
+    vc = kc.clone()
+    key = torch.randn(2, 3, 8, generator=g).to(torch.bfloat16)
+    oracle.reshape_and_cache(key, key, kc, vc, torch.tensor([63, 0]))
+    assert torch.equal(kc[3, :, 15].view(torch.int16), key[0].view(torch.int16))
+    assert torch.equal(vc[0, :, 0].view(torch.int16), key[1].view(torch.int16))
+    before = kc.clone()
+    with pytest.raises(ValueError):
+        oracle.reshape_and_cache(key, key, kc, vc, torch.tensor([1, 64]))
+    assert torch.equal(before, kc)
+
+
+# ---------------------------------------------------------------------------
+# against a library routine
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("H_q,H_kv", [(4, 4), (4, 2), (8, 1)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_matches_sdpa(H_q, H_kv, dtype):
+    """Paged decode at random placements equals torch's attention on the same
+    K/V laid out contiguously (GQA by torch's own grouping, MQA with one kv
+    head). Ragged lengths span several blocks and partial last blocks."""
+    ctxs, D, bs = [1, 7, 16, 17, 40, 65], 8, 4
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=H_q * 10 + H_kv,
+                                                   dtype=dtype)
+    scale = 1 / math.sqrt(D)
+    out, lse = oracle.decode(q, kc, vc, tables, lens, scale)
+    for b, c in enumerate(ctxs):
+        ref = sdpa(q[b][:, None], ks[b], vs[b], scale)[:, 0]
+        torch.testing.assert_close(out[b], ref, rtol=1e-12, atol=1e-12)
+        # lse against the library's logsumexp of the scores
+        kk = ks[b].to(F64).repeat_interleave(H_q // H_kv, 0)
+        sc = torch.einsum("hd,hjd->hj", q[b].to(F64), kk) * scale
+        torch.testing.assert_close(lse[b], torch.logsumexp(sc, -1), rtol=1e-13, atol=1e-13)
+
+
+def test_decode_numpy_brute_force():
+    """A dense numpy evaluation on tiny inputs (explicit exponentials, no
+    max-shift) agrees with the oracle."""
+    ctxs, H_q, H_kv, D, bs = [3, 9], 2, 1, 4, 4
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=11)
+    out, _ = oracle.decode(q, kc, vc, tables, lens, 0.5)
+    for b in range(2):
+        K, V = ks[b][0].double().numpy(), vs[b][0].double().numpy()
+        for h in range(H_q):
+            e = np.exp(0.5 * (K @ q[b, h].double().numpy()))
+            np.testing.assert_allclose(out[b, h].numpy(), (e[:, None] * V).sum(0) / e.sum(),
+                                       rtol=1e-12)
+
+
+def test_gqa_head_mapping():
+    """With 4 q heads over 2 kv heads, heads 2 and 3 read kv head 1: a
+    constant V there gives that constant (up to the rounding of weights that
+    sum to one), and heads 0 and 1 do not."""
+    ctxs, D, bs = [20], 8, 16
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, 4, 2, D, bs, seed=3)
+    vs[0][1] = 0.375
+    kc, vc = place(ks, vs, [tables[0, :2].tolist()], kc.shape[0], bs)
+    out, _ = oracle.decode(q, kc, vc, tables, lens, 0.3)
+    torch.testing.assert_close(out[0, 2:], torch.full_like(out[0, 2:], 0.375), rtol=1e-15,
+                               atol=0)
+    assert torch.all((out[0, :2] - 0.375).abs() > 1e-3)
+
+
+# ---------------------------------------------------------------------------
+# special cases
+# ---------------------------------------------------------------------------
+def test_single_token_returns_its_value():
+    q, ks, vs, kc, vc, tables, lens = random_paged([1, 1], 2, 2, 8, 16, seed=4)
+    out, lse = oracle.decode(q, kc, vc, tables, lens, 0.7)
+    for b in range(2):
+        assert torch.equal(out[b], vs[b][:, 0].double())
+        sc = 0.7 * (q[b].double() * ks[b][:, 0].double()).sum(-1)
+        torch.testing.assert_close(lse[b], sc, rtol=0, atol=1e-15)
+
+
+def test_equal_keys_and_zero_scale_give_mean():
+    q, ks, vs, kc, vc, tables, lens = random_paged([33], 2, 2, 8, 16, seed=6)
+    out0, _ = oracle.decode(q, kc, vc, tables, lens, 0.0)
+    mean = vs[0].double().mean(1)
+    torch.testing.assert_close(out0[0], mean, rtol=1e-13, atol=1e-14)
+    ks[0][:] = ks[0][:, :1]
+    kc2, vc2 = place(ks, vs, [tables[0].tolist()], kc.shape[0], 16)
+    out1, lse1 = oracle.decode(q, kc2, vc2, tables, lens, 0.9)
+    torch.testing.assert_close(out1[0], mean, rtol=1e-13, atol=1e-14)
+    sc = 0.9 * (q[0].double() * ks[0][:, 0].double()).sum(-1)
+    torch.testing.assert_close(lse1[0], sc + math.log(33), rtol=1e-13, atol=1e-13)
+
+
+def test_empty_sequence():
+    q, ks, vs, kc, vc, tables, lens = random_paged([5], 2, 1, 4, 4, seed=8)
+    lens = torch.tensor([0], dtype=torch.int32)
+    out, lse = oracle.decode(q, kc, vc, tables, lens, 1.0)
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_bad_inputs_rejected():
+    q, ks, vs, kc, vc, tables, lens = random_paged([5], 2, 1, 4, 4, seed=9)
+    bad = tables.clone()
+    bad[0, 0] = kc.shape[0]
+    with pytest.raises(ValueError):
+        oracle.decode(q, kc, vc, bad, lens, 1.0)
+    with pytest.raises(ValueError):
+        oracle.decode(q, kc, vc, tables, torch.tensor([tables.shape[1] * 4 + 1],
+                                                      dtype=torch.int32), 1.0)
+
+
+# ---------------------------------------------------------------------------
+# invariants of paging
+# ---------------------------------------------------------------------------
+def test_block_permutation_invariance():
+    """Moving physical blocks (and remapping the tables) leaves the result
+    bit-identical: the gather reaches the same tokens in the same order."""
+    ctxs, H_q, H_kv, D, bs = [9, 30, 47], 4, 2, 16, 8
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=12,
+                                                   dtype=torch.bfloat16)
+    out, lse = oracle.decode(q, kc, vc, tables, lens, 0.25)
+    perm = torch.randperm(kc.shape[0], generator=torch.Generator().manual_seed(13))
+    kc2 = torch.empty_like(kc)
+    vc2 = torch.empty_like(vc)
+    kc2[perm], vc2[perm] = kc, vc  # block i moves to perm[i]
+    t2 = perm[tables.long()].to(torch.int32)
+    out2, lse2 = oracle.decode(q, kc2, vc2, t2, lens, 0.25)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def test_shared_prefix_equals_private_copies():
+    """Beams sharing prefix blocks (and a copied partial block, like B6') give
+    bit-identical results to beams with private copies of everything."""
+    bs, D, H = 16, 8, 2
+    g = torch.Generator().manual_seed(14)
+    prefix_k, prefix_v = torch.randn(H, 37, D, generator=g), torch.randn(H, 37, D, generator=g)
+    tails = [11, 25]
+    ks = [torch.cat([prefix_k, torch.randn(H, t, D, generator=g)], 1) for t in tails]
+    vs = [torch.cat([prefix_v, torch.randn(H, t, D, generator=g)], 1) for t in tails]
+    # shared: blocks 1 and 3 hold prefix positions 0..31 for both beams;
+    # positions 32..36 are in each beam's own block (6 and 8), copied
+    shared_rows = [[1, 3, 6, 2], [1, 3, 8, 9, 0]]
+    kc, vc = place(ks, vs, shared_rows, 12, bs)
+    private_rows = [[0, 2, 4, 5], [6, 7, 8, 9, 10]]
+    kp, vp = place(ks, vs, private_rows, 12, bs)
+    q = torch.randn(2, 4, D, generator=g)
+    lens = torch.tensor([37 + t for t in tails], dtype=torch.int32)
+    a = oracle.decode(q, kc, vc, pad_tables(shared_rows, 5, 11), lens, 0.3)
+    b = oracle.decode(q, kp, vp, pad_tables(private_rows, 5, 11), lens, 0.3)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------------------
+# KV split and log-sum-exp merge
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("part", [1, 3, 16, 64, 1000])
+def test_split_merge_equals_unsplit(part):
+    ctxs, H_q, H_kv, D, bs = [1, 16, 50, 130], 4, 2, 8, 16
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=15)
+    out, lse = oracle.decode(q, kc, vc, tables, lens, 0.4)
+    op, lp = oracle.decode_partials(q, kc, vc, tables, lens, 0.4, part)
+    assert op.shape[2] == -(-max(ctxs) // part)
+    mo, ml = oracle.lse_merge(op, lp)
+    torch.testing.assert_close(mo, out, rtol=1e-12, atol=1e-12)
+    torch.testing.assert_close(ml, lse, rtol=1e-12, atol=1e-12)
+
+
+def test_lse_merge_closed_forms():
+    """Two partials: the merged lse is log(e^a + e^b) and the output the
+    correspondingly weighted mean; -inf partials carry no weight."""
+    o = torch.tensor([[[1.0, 2.0], [3.0, -1.0], [9.0, 9.0]]], dtype=F64)
+    lse = torch.tensor([[math.log(1.0), math.log(3.0), float("-inf")]], dtype=F64)
+    mo, ml = oracle.lse_merge(o, lse)
+    torch.testing.assert_close(ml, torch.tensor([math.log(4.0)], dtype=F64))
+    torch.testing.assert_close(mo, torch.tensor([[2.5, -0.25]], dtype=F64))
+    mo, ml = oracle.lse_merge(o[:, :1], lse[:, :1])
+    assert torch.equal(mo, o[:, 0]) and ml.item() == 0.0
+    mo, ml = oracle.lse_merge(o[:, 2:], lse[:, 2:])
+    assert torch.all(mo == 0) and torch.isneginf(ml).all()
+
+
+# ---------------------------------------------------------------------------
+# chunked prefill
+# ---------------------------------------------------------------------------
+def test_prefill_no_cache_is_causal_attention():
+    """Chunks with nothing cached and identity tables equal torch's causal
+    attention over each chunk."""
+    Cs, H_q, H_kv, D, bs = [5, 16, 23], 4, 2, 8, 4
+    g = torch.Generator().manual_seed(16)
+    ks = [torch.randn(H_kv, c, D, generator=g) for c in Cs]
+    vs = [torch.randn(H_kv, c, D, generator=g) for c in Cs]
+    rows, at = [], 0
+    for c in Cs:
+        n = -(-c // bs)
+        rows.append(list(range(at, at + n)))
+        at += n
+    kc, vc = place(ks, vs, rows, at + 1, bs)
+    tables = pad_tables(rows, max(len(r) for r in rows), at)
+    qsl = torch.tensor([0] + list(np.cumsum(Cs)), dtype=torch.int32)
+    q = torch.randn(sum(Cs), H_q, D, generator=g)
+    out, _ = oracle.prefill(q, kc, vc, tables, torch.tensor(Cs, dtype=torch.int32), qsl, 0.35)
+    for c, C in enumerate(Cs):
+        qc = q[qsl[c]:qsl[c + 1]].transpose(0, 1)
+        ref = sdpa(qc, ks[c], vs[c], 0.35, causal=True).transpose(0, 1)
+        torch.testing.assert_close(out[qsl[c]:qsl[c + 1]], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_query_equals_decode_at_its_position():
+    """Query i of a chunk after ``cached`` tokens equals a decode over the
+    first cached+i+1 tokens (chunk length 1 is exactly decode)."""
+    ctxs, H_q, H_kv, D, bs = [37, 70], 4, 1, 8, 16
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=17)
+    Cs = [9, 1]
+    g = torch.Generator().manual_seed(18)
+    qp = torch.randn(sum(Cs), H_q, D, generator=g)
+    qsl = torch.tensor([0, Cs[0], Cs[0] + Cs[1]], dtype=torch.int32)
+    out, lse = oracle.prefill(qp, kc, vc, tables, lens, qsl, 0.3)
+    for c, C in enumerate(Cs):
+        for i in range(C):
+            row = int(qsl[c]) + i
+            pos = ctxs[c] - C + i
+            d, dl = oracle.decode(qp[row][None], kc, vc, tables[c:c + 1],
+                                  torch.tensor([pos + 1], dtype=torch.int32), 0.3)
+            assert torch.equal(out[row], d[0]) and torch.equal(lse[row], dl[0])
+
+
+def test_prefill_ignores_future_keys():
+    """Changing keys/values at positions after a query's own leaves that
+    query's output bit-identical (causality)."""
+    ctxs, H_q, H_kv, D, bs = [40], 2, 1, 8, 8
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=19)
+    qp = torch.randn(12, H_q, D, generator=torch.Generator().manual_seed(20))
+    qsl = torch.tensor([0, 12], dtype=torch.int32)
+    out, _ = oracle.prefill(qp, kc, vc, tables, lens, qsl, 0.3)
+    ks[0][:, 35:] += 3.0
+    vs[0][:, 35:] -= 2.0
+    kc2, vc2 = place(ks, vs, [tables[0].tolist()], kc.shape[0], bs)
+    out2, _ = oracle.prefill(qp, kc2, vc2, tables, lens, qsl, 0.3)
+    # query i sits at position 28 + i: rows 0..6 (positions 28..34) unchanged
+    assert torch.equal(out[:7], out2[:7])
+    assert not torch.equal(out[7:], out2[7:])
+
+
+def test_select_computes_only_selected():
+    q, ks, vs, kc, vc, tables, lens = random_paged([9, 30], 4, 2, 8, 8, seed=21)
+    full, _ = oracle.decode(q, kc, vc, tables, lens, 0.5)
+    sel = torch.zeros(2, 4, dtype=torch.bool)
+    sel[1, 3] = sel[0, 0] = True
+    part, _ = oracle.decode(q, kc, vc, tables, lens, 0.5, select=sel)
+    assert torch.equal(part[sel], full[sel]) and torch.all(part[~sel] == 0)
