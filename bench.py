@@ -1,0 +1,608 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+A step is one pass of the hot path over one batch of seeded synthetic input:
+reshape_and_cache of the step's new tokens, then paged decode attention
+(split-KV kernel and, when a sequence spans several partitions, the
+log-sum-exp merge); the mixed workload adds the chunked-prefill kernel. The
+default workload is the Llama-2-7B-shaped decode batch (64 sequences,
+lengths uniform in [128, 2048], 32/32 heads, head_dim 128, 16-token blocks,
+bf16). Its KV read per step (about 1.1 GB) is far larger than the 126 MB L2,
+so no L2 flush is needed between steps.
+
+One process per GPU; under torchrun each rank runs its own batch (different
+seed, same shape: weak scaling, no collective on the data path). Timing is
+CUDA events on the launching stream between barriers; the JSON line reports
+the slowest rank's time and the sum of all ranks' work.
+
+Printed (rank 0, one JSON line): metric/value/unit (KV-read GB/s of the
+decode attention, counted from the algorithmic bytes), tokens/s, the
+roofline of the dominant call against the measured HBM peak, the host
+oracle as a CPU baseline, an end-to-end figure through the public API with
+host buffers, the kernel launch count and the SM clocks seen while timing.
+``--impl reference`` times the fp64 CPU oracle instead, on bounded samples
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV-read GB/s (frac of HBM peak); tokens/s per batch"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# --------------------------------------------------------------------------
+# process / rank plumbing
+# --------------------------------------------------------------------------
+def rank_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, local, world
+
+
+def pin_device(local_rank: int, world: int):
+    """Under torchrun each rank sees only its own GPU (set before CUDA starts)."""
+    if world > 1:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        ids = vis.split(",") if vis else [str(i) for i in range(64)]
+        os.environ["CUDA_VISIBLE_DEVICES"] = ids[local_rank]
+
+
+def init_dist(world: int, backend: str, timeout_s: int = 300):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def aggregate(units: float, ms: float, world: int, device=None):
+    """Sum of every rank's work and the slowest rank's time (identical on all
+    ranks). Works with any process-group backend."""
+    import torch
+    if world <= 1:
+        return units, ms
+    import torch.distributed as dist
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(u.item()), float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# work accounting
+# --------------------------------------------------------------------------
+def decode_bytes(batch) -> float:
+    """Algorithmic bytes of one decode call: K and V of every valid token per
+    kv head, q and out, each CTA's table slice, and the lengths."""
+    import torch
+    if batch.q is None or batch.num_seqs == 0:
+        return 0.0
+    e = batch.k_cache.element_size()
+    ctx = batch.context_lens.to(torch.int64)
+    H_kv, D, bs = batch.num_kv_heads, batch.head_dim, batch.block_size
+    kv = int((2 * ctx * H_kv * D * e).sum())
+    qo = 2 * batch.num_seqs * batch.num_q_heads * D * e
+    tbl = int((4 * ((ctx + bs - 1) // bs) * H_kv).sum())
+    return float(kv + qo + tbl + 4 * batch.num_seqs)
+
+
+def reshape_bytes(batch) -> float:
+    """Algorithmic bytes of the cache scatter: read and write K and V rows of
+    every non-padding token, plus the slots."""
+    e = batch.k_cache.element_size()
+    T = int((batch.slot_mapping >= 0).sum())
+    return float(2 * 2 * T * batch.num_kv_heads * batch.head_dim * e + 8 * batch.slot_mapping.numel())
+
+
+def prefill_flops(batch) -> float:
+    """Algorithmic FLOPs of the chunked prefill: Q.K^T and P.V over each
+    query's causal range (4 D H_q per query-key pair)."""
+    if batch.prefill_q is None:
+        return 0.0
+    qsl = batch.query_start_loc.tolist()
+    ctx = batch.prefill_context_lens.tolist()
+    H_q, D = batch.num_q_heads, batch.head_dim
+    f = 0
+    for c in range(len(ctx)):
+        C = qsl[c + 1] - qsl[c]
+        cached = ctx[c] - C
+        f += 4 * D * H_q * (C * cached + C * (C + 1) // 2)
+    return float(f)
+
+
+def tokens_per_step(batch) -> int:
+    n = batch.num_seqs
+    if batch.prefill_q is not None:
+        n += batch.prefill_q.shape[0]
+    return n
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(
+            p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def source_digest(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(profile: str, kernel_files, units_scale: float = 1.0):
+    """DRAM bytes per launch recorded in a committed ncu summary, or None when
+    the summary is missing or the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", profile)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.lstrip().startswith(("source-sha256", "dram-bytes-per-launch")):
+            k, v = line.split(":", 1)
+            fields[k.strip().lstrip("-* ")] = v.strip().strip("`")
+    if fields.get("source-sha256") != source_digest(kernel_files):
+        return None
+    try:
+        return float(fields["dram-bytes-per-launch"]) * units_scale
+    except (KeyError, ValueError):
+        return None
+
+
+# --------------------------------------------------------------------------
+# clocks while timing (NVML reads only)
+# --------------------------------------------------------------------------
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            h = None
+            try:
+                p = torch.cuda.get_device_properties(0)
+                bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0]
+                h = pynvml.nvmlDeviceGetHandleByIndex(int(vis) if vis.isdigit() else 0)
+            self.h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _sample(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((sm, r))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if not self.ok:
+            return
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self._stop.set()
+        self._t.join()
+        try:
+            self._sample()
+        except Exception:
+            pass
+        sms = [s for s, _ in self.samples]
+        mask = 0
+        for _, r in self.samples:
+            mask |= int(r)
+        names = sorted(n for bit, n in REASONS.items() if mask & bit and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(sms)}
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def make_batch(name: str, seed: int):
+    from pagedattention_paged_kv_02_b200 import workloads as W
+    return W.WORKLOADS[name](seed=seed)
+
+
+class Runner:
+    """Holds a device batch and issues one step through the public binding."""
+
+    def __init__(self, batch, dev):
+        import torch
+        from pagedattention_paged_kv_02_b200 import pa
+        self.pa = pa
+        self.host = batch
+        self.d = batch.to(dev)
+        d = self.d
+        self.part = d.partition_size
+        self.max_ctx = batch.max_context_len  # host-side bound, computed once
+        self.ws = None
+        self.S = 0
+        if d.q is not None and d.num_seqs:
+            B, H_q, D = d.q.shape
+            n = pa.pa_decode_workspace_size(B, H_q, D, d.max_context_len, self.part)
+            self.ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+            P = pa.pa_decode_partition_tokens(d.max_context_len, self.part)
+            self.S = -(-d.max_context_len // P)
+            self.out = torch.empty_like(d.q)
+        if d.prefill_q is not None:
+            self.pout = torch.empty_like(d.prefill_q)
+            qsl = d.query_start_loc.cpu()
+            self.max_q = int((qsl[1:] - qsl[:-1]).max())
+
+    def launches_per_step(self) -> int:
+        n = 1  # reshape_and_cache
+        if self.d.q is not None and self.d.num_seqs:
+            n += 1 + (1 if self.S > 1 else 0)
+        if self.d.prefill_q is not None:
+            n += 1
+        return n
+
+    def step(self, ev=None, d=None, out=None):
+        """One pass; ``ev`` (start, end) events bracket the dominant call."""
+        pa = self.pa
+        d = d or self.d
+        pa.pa_reshape_and_cache(d.key, d.value, d.k_cache, d.v_cache, d.slot_mapping)
+        if d.prefill_q is not None:
+            if ev is not None and self.dominant == "prefill":
+                ev[0].record()
+            pa.pa_prefill_chunk(self.pout, d.prefill_q, d.k_cache, d.v_cache,
+                                d.prefill_block_tables, d.prefill_context_lens,
+                                d.query_start_loc, self.max_q, d.scale)
+            if ev is not None and self.dominant == "prefill":
+                ev[1].record()
+        if d.q is not None and d.num_seqs:
+            if ev is not None and self.dominant == "decode":
+                ev[0].record()
+            pa.pa_decode(out if out is not None else self.out, d.q, d.k_cache, d.v_cache,
+                         d.block_tables, d.context_lens, self.max_ctx, d.scale, self.part,
+                         self.ws)
+            if ev is not None and self.dominant == "decode":
+                ev[1].record()
+
+    @property
+    def dominant(self):
+        return "prefill" if self.d.prefill_q is not None else "decode"
+
+
+def run_ours(args, rank, world):
+    import torch
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    dist = init_dist(world, "nccl")
+    batch = make_batch(args.workload, seed=rank)
+    r = Runner(batch, dev)
+    hbm, bf16, bf16_sus, basis = load_peaks()
+
+    dbytes = decode_bytes(batch)
+    rbytes = reshape_bytes(batch)
+    pflops = prefill_flops(batch)
+
+    for _ in range(args.warmup):
+        r.step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record()
+    for i in range(K):
+        r.step(evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms_local = t0.elapsed_time(t1) / K
+    dom_ms = statistics.fmean(a.elapsed_time(b) for a, b in evs)
+
+    units = dbytes if r.dominant == "decode" else pflops
+    total_units, ms = aggregate(units, ms_local, world, dev)
+    tok_total, _ = aggregate(float(tokens_per_step(batch)), ms_local, world, dev)
+    dbytes_total, _ = aggregate(dbytes, ms_local, world, dev)
+
+    # end to end through the public API: per-step inputs from pinned host
+    # memory, the result read back every step
+    h = {}
+    names = ["key", "value", "slot_mapping"]
+    if batch.q is not None:
+        names += ["q", "block_tables", "context_lens"]
+    if batch.prefill_q is not None:
+        names += ["prefill_q", "prefill_block_tables", "prefill_context_lens", "query_start_loc"]
+    for n in names:
+        h[n] = getattr(batch, n).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    res = r.out if batch.q is not None else r.pout
+    out_h = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
+    d2h = out_h.numel() * out_h.element_size()
+    stage = {n: torch.empty_like(getattr(r.d, n)) for n in names}
+    import copy
+    dd = copy.copy(r.d)
+    for n in names:
+        setattr(dd, n, stage[n])
+
+    def e2e_step():
+        for n in names:
+            stage[n].copy_(h[n], non_blocking=True)
+        r.step(d=dd)
+        out_h.copy_(res, non_blocking=True)
+
+    for _ in range(max(3, args.warmup // 4)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms_local = e0.elapsed_time(e1) / K
+    _, e2e_ms = aggregate(0.0, e2e_ms_local, world, dev)
+
+    line = None
+    if rank == 0:
+        if r.dominant == "decode":
+            value = dbytes_total / (ms * 1e-3) / 1e9
+            unit = "GB/s"
+            achieved = dbytes / (dom_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                    "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                    "peak_basis": f"{basis} hbm_gbs",
+                    "kernel": "pa_decode (decode_split + decode_reduce)",
+                    "alg_bytes_per_launch": dbytes,
+                    "traffic": profiled_traffic(f"decode_{args.workload}.md",
+                                                DECODE_SOURCES)}
+        else:
+            value = dbytes_total / (ms * 1e-3) / 1e9
+            unit = "GB/s"
+            achieved = pflops / (dom_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_sus,
+                    "unit": "TFLOP/s", "frac": round(achieved / bf16_sus, 4),
+                    "peak_basis": f"{basis} bf16_tflops_sustained",
+                    "kernel": "pa_prefill_chunk", "alg_flops_per_launch": pflops,
+                    "traffic": profiled_traffic(f"prefill_{args.workload}.md",
+                                                PREFILL_SOURCES)}
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if batch.dtype.itemsize == 2 else "f32",
+            "data": "synthetic (seeded; one batch per rank)",
+            "config": workload_config(batch, args.workload, world, r),
+            "tokens_per_s": round(tok_total / (ms * 1e-3), 1),
+            "frac_of_hbm_peak": round(value / world / hbm, 4),
+            "frac_of_nominal_8tbs": round(value / world / 8000.0, 4),
+            "roofline": roof,
+            "e2e": {"value": round(dbytes_total / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 5)},
+            "gpu_launches": K * r.launches_per_step(),
+            "clocks": clk,
+        }
+        if r.dominant != "decode":
+            line["prefill_tflops"] = round(pflops * world / (ms * 1e-3) / 1e12, 1)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(batch, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+DECODE_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/decode.cuh",
+                  "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
+PREFILL_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/prefill.cuh",
+                   "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
+
+
+def workload_config(batch, name, world, r=None):
+    c = {"workload": batch.name, "name": name, "block_size": batch.block_size,
+         "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
+         "head_dim": batch.head_dim, "num_blocks": batch.num_blocks,
+         "parallelism": f"dp{world} (independent batches, no collective)",
+         "l2": "no flush: inputs larger than L2 (KV read per step >> 126 MB)"}
+    if batch.q is not None and batch.num_seqs:
+        lens = batch.context_lens
+        c.update({"num_seqs": batch.num_seqs, "context_len_mean": round(float(lens.float().mean()), 1),
+                  "context_len_max": int(lens.max()),
+                  "partition_tokens": None if r is None else
+                  r.pa.pa_decode_partition_tokens(batch.max_context_len, batch.partition_size)})
+    if batch.prefill_q is not None:
+        c.update({"prefill_chunks": batch.query_start_loc.numel() - 1,
+                  "prefill_tokens": batch.prefill_q.shape[0]})
+    return c
+
+
+# --------------------------------------------------------------------------
+# the fp64 host oracle as a baseline
+# --------------------------------------------------------------------------
+def _oracle_step(batch, k, v, select=None, pselect=None):
+    import oracle
+    oracle.reshape_and_cache(batch.key, batch.value, k, v, batch.slot_mapping)
+    if batch.prefill_q is not None:
+        oracle.prefill(batch.prefill_q, k, v, batch.prefill_block_tables,
+                       batch.prefill_context_lens, batch.query_start_loc, batch.scale,
+                       select=pselect)
+    if batch.q is not None and batch.num_seqs:
+        oracle.decode(batch.q, k, v, batch.block_tables, batch.context_lens, batch.scale,
+                      select=select)
+
+
+def _sample_masks(batch, frac: float, offset: int):
+    """Boolean masks selecting about ``frac`` of the (row, head) outputs,
+    rotated by ``offset`` so that successive samples cover different rows."""
+    import torch
+    sel = psel = None
+    if batch.q is not None and batch.num_seqs:
+        n = batch.num_seqs * batch.num_q_heads
+        k = max(1, int(round(frac * n)))
+        idx = (torch.arange(k) * max(1, n // k) + offset) % n
+        sel = torch.zeros(n, dtype=torch.bool)
+        sel[idx] = True
+    if batch.prefill_q is not None:
+        n = batch.prefill_q.shape[0] * batch.num_q_heads
+        k = max(1, int(round(frac * n)))
+        idx = (torch.arange(k) * max(1, n // k) + offset) % n
+        psel = torch.zeros(n, dtype=torch.bool)
+        psel[idx] = True
+    return sel, psel
+
+
+def cpu_baseline(batch, seconds: float):
+    """The oracle as it stands on this host's cores: whole-batch steps (or, for
+    workloads whose full step is too slow, evenly spaced samples of it)
+    repeated for about ``seconds``; value in the metric's unit."""
+    import oracle
+    k, v = batch.k_cache, batch.v_cache  # host pool; appending in place is idempotent
+    t = time.perf_counter()
+    sel, psel = _sample_masks(batch, 1.0 / 64, 0)
+    _oracle_step(batch, k, v, sel, psel)
+    probe = (time.perf_counter() - t) * 64
+    frac = 1.0 if probe < seconds / 2 else max(1e-4, seconds / 2 / probe)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        sel, psel = (None, None) if frac >= 1.0 else _sample_masks(batch, frac, reps * 7919)
+        _oracle_step(batch, k, v, sel, psel)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    work = decode_bytes(batch) * frac * reps
+    sample = ("whole batch" if frac >= 1.0 else f"{frac:.4%} of the batch's (row, head) outputs"
+              ) + f", {reps} step(s) in {dt:.1f} s"
+    return {"value": round(work / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": sample}
+
+
+def run_reference(args, rank, world):
+    """The oracle on the host cores, K timed steps of bounded samples."""
+    if rank != 0:
+        return
+    import oracle
+    batch = make_batch(args.workload, seed=0)
+    k, v = batch.k_cache, batch.v_cache
+    total = args.steps + args.warmup
+    t = time.perf_counter()
+    sel, psel = _sample_masks(batch, 1.0 / 64, 0)
+    _oracle_step(batch, k, v, sel, psel)
+    full = (time.perf_counter() - t) * 64
+    budget = max(0.02, args.reference_seconds / max(1, total))
+    frac = min(1.0, budget / full)
+    for i in range(args.warmup):
+        s, ps = _sample_masks(batch, frac, i * 104729)
+        _oracle_step(batch, k, v, s, ps)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        s, ps = _sample_masks(batch, frac, (i + args.warmup) * 104729)
+        _oracle_step(batch, k, v, s, ps)
+    dt = time.perf_counter() - t0
+    ms = dt / args.steps * 1e3
+    value = decode_bytes(batch) * frac / (ms * 1e-3) / 1e9
+    sample = f"{frac:.4%} of the batch's (row, head) outputs per step"
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+            "config": workload_config(batch, args.workload, world),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
+                             "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="llama7b_decode",
+                    choices=["tiny_fp32", "llama7b_decode", "gqa_decode", "long_context_decode",
+                             "mixed_prefill_decode"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, local, world = rank_env()
+    if world != args.gpus and world > 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    pin_device(local, world)
+    run_ours(args, rank, world)
+
+
+if __name__ == "__main__":
+    main()

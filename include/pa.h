@@ -1,0 +1,184 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged-KV attention on B200 (sm_100a).
+ *
+ * The operations, by the page and section that define them:
+ *
+ *  pa_reshape_and_cache
+ *      page "字节跳动 AI Infra (2)", question "KV Cache原理与优化": at step t
+ *      the new token's K_t and V_t are appended to the cache
+ *      (K_cache = concat(K_cache, K_t)). In paged form the append is a
+ *      scatter into a slot of a physical block (same page, question
+ *      "vLLM与PagedAttention的原理": a block of block_size tokens starts at
+ *      physical_block * block_size * head_dim).
+ *
+ *  pa_decode
+ *      same page, "KV Cache原理与优化": Attention_t = softmax(Q_t K^T / sqrt(d)) V
+ *      for the one new query of each sequence, with K/V reached through the
+ *      sequence's block table ("vLLM与PagedAttention的原理"); query heads
+ *      share K/V heads in groups (page "LLM推理优化", section 1.3, GQA/MQA);
+ *      long contexts are split along the KV length and the partial results
+ *      merged (page "字节跳动 AI Infra (2)", algorithm-level table, row
+ *      FlashDecoding), using online-softmax statistics (page "LLM推理优化",
+ *      section 2.1, FlashAttention's tiling and online softmax).
+ *
+ *  pa_prefill_chunk
+ *      page "vLLM框架是怎么做推理加速的", section 3 (Chunked Prefill): a
+ *      prompt is processed in chunks (512 tokens by default) that attend
+ *      over the paged cache; attention within the prompt is causal (page
+ *      "LLM推理优化", section 2.3, causal=True).
+ *
+ * Data layout (all device memory, row-major, owned by the caller):
+ *   k_cache, v_cache   [num_blocks][num_kv_heads][block_size][head_dim]
+ *                      One (block, kv head) page of block_size*head_dim
+ *                      elements is contiguous. With num_kv_heads == 1 this is
+ *                      exactly the pages' pointer formula.
+ *   block_tables       int32 [rows][max_blocks_per_seq]; entry i of row r is
+ *                      the physical block holding tokens [i*bs, (i+1)*bs) of
+ *                      sequence (or chunk) r. Entries past the valid tokens
+ *                      are never read.
+ *   context_lens       int32 [rows]; valid tokens of the row, including any
+ *                      token(s) appended in this step.
+ *   slot_mapping       int64 [num_tokens]; slot = physical_block*bs + offset.
+ *                      Negative slots are padding and are skipped.
+ *   q / out (decode)   [num_seqs][num_q_heads][head_dim]
+ *   q / out (prefill)  [total_q][num_q_heads][head_dim], chunk c owning rows
+ *                      [query_start_loc[c], query_start_loc[c+1]).
+ *   key / value        [num_tokens][num_kv_heads][head_dim]
+ *   Query head h reads K/V head h / (num_q_heads / num_kv_heads).
+ *   q, out, key, value and the caches all have element type `dtype`;
+ *   accumulation is fp32; bf16 outputs are rounded to nearest even.
+ *
+ * Conventions:
+ *   - Every call is asynchronous on `stream`, never allocates device memory,
+ *     and never synchronises, except where a function says otherwise.
+ *   - Argument checks run on the host before any launch. A failed check
+ *     returns an error code, launches nothing and writes nothing.
+ *   - Supported: head_dim in {64, 128}; block_size in {16, 32, 64};
+ *     num_q_heads % num_kv_heads == 0. Anything else returns
+ *     PA_ERR_UNSUPPORTED. Cache, q, out, key and value pointers must be
+ *     16-byte aligned, table and length pointers 4-byte aligned.
+ *   - Device data the host cannot see (block ids, lengths, slots) is checked
+ *     on the device: an out-of-range block id or slot is skipped, never
+ *     dereferenced, and recorded in a sticky device error word that
+ *     pa_device_error() reads. Device-side waits are bounded; a wait that
+ *     runs out records PA_ERR_TIMEOUT there and the kernel returns.
+ *   - A launch failure returns PA_ERR_CUDA (cudaGetLastError is consumed).
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1, /* null pointer, negative size, misalignment, bad dtype */
+    PA_ERR_UNSUPPORTED = 2, /* shape outside the supported set */
+    PA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+    PA_ERR_BAD_TABLE = 4,   /* a block id, slot or length outside its range */
+    PA_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out */
+    PA_ERR_CUDA = 6         /* a CUDA runtime call or launch failed */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Scatter new tokens' K/V rows into their cache slots:
+ *   for t with s = slot_mapping[t] >= 0 and every kv head h:
+ *     k_cache[s / block_size][h][s % block_size][:] = key[t][h][:]
+ *     v_cache[s / block_size][h][s % block_size][:] = value[t][h][:]
+ * Rows are copied bit for bit. A slot >= num_blocks*block_size is skipped
+ * and recorded as PA_ERR_BAD_TABLE in the device error word. Slots must be
+ * distinct (two tokens writing one slot race). num_tokens == 0 is a no-op. */
+PA_API pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                               const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               cudaStream_t stream);
+
+/* Bytes of workspace pa_decode needs for these sizes and partition_size
+ * (same meaning as in pa_decode). 0 when every sequence fits one partition. */
+PA_API size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                int partition_size);
+
+/* Token count of one KV partition that pa_decode uses for these arguments
+ * (resolves partition_size == 0 and < 0), or -1 for invalid arguments. */
+PA_API int pa_decode_partition_tokens(int max_context_len, int partition_size);
+
+/* Paged decode attention, one query per sequence:
+ *   out[b][h] = sum_j softmax_j(scale * q[b][h] . K_j) V_j
+ * over positions j < context_lens[b] of sequence b, K_j/V_j read from head
+ * h / (num_q_heads/num_kv_heads) of physical block block_tables[b][j / bs]
+ * at offset j % bs.
+ *   max_context_len   host-side upper bound of context_lens (lengths above
+ *                     it, or above max_blocks_per_seq*block_size, are clamped
+ *                     and recorded as PA_ERR_BAD_TABLE).
+ *   partition_size    KV tokens per split (multiple of 16, <= 16384);
+ *                     0 = choose automatically; < 0 = never split. Sequences
+ *                     longer than one partition are computed as partial
+ *                     results merged by log-sum-exp.
+ *   workspace         device scratch of >= pa_decode_workspace_size(...)
+ *                     bytes (may be NULL when that is 0), 256-byte aligned;
+ *                     contents on entry are ignored.
+ * A sequence with context_len 0 yields out = 0. */
+PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                    int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
+                    cudaStream_t stream);
+
+/* Chunked prefill: chunk c has C_c = query_start_loc[c+1] - query_start_loc[c]
+ * queries and context_lens[c] tokens in the cache (its own C_c tokens
+ * included, already written by pa_reshape_and_cache). Query i of the chunk
+ * sits at position p = context_lens[c] - C_c + i and attends positions 0..p:
+ *   out[r][h] = sum_{j<=p} softmax_j(scale * q[r][h] . K_j) V_j,  r = qsl[c]+i.
+ *   max_query_len     host-side upper bound of every C_c.
+ * bf16 only (tensor-core path); fp32 returns PA_ERR_UNSUPPORTED. */
+PA_API pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *block_tables, const int32_t *context_lens,
+                           const int32_t *query_start_loc, int num_chunks, int max_query_len,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, int max_blocks_per_seq, float scale, pa_dtype dtype,
+                           cudaStream_t stream);
+
+/* Check block tables and lengths on the device: every entry a row's valid
+ * tokens reach must lie in [0, num_blocks), and 0 <= context_lens[r] <=
+ * max_blocks_per_seq*block_size. d_scratch is one caller-owned device int32.
+ * SYNCHRONOUS: waits for `stream`, stores the number of bad rows in
+ * *bad_rows (may be NULL) and returns PA_ERR_BAD_TABLE if any. */
+PA_API pa_status pa_check_tables(const int32_t *block_tables, const int32_t *context_lens, int rows,
+                          int max_blocks_per_seq, int block_size, int num_blocks,
+                          int32_t *d_scratch, int *bad_rows, cudaStream_t stream);
+
+/* Read (and with clear != 0 reset) the sticky device error word of the
+ * current device: PA_OK, PA_ERR_BAD_TABLE or PA_ERR_TIMEOUT, the first one
+ * recorded. SYNCHRONOUS: waits for all prior work on the device. */
+PA_API pa_status pa_device_error(int *status, int clear);
+
+/* Failure-detection self test: launch one CTA that waits, with a bound of
+ * timeout_ns nanoseconds, on a barrier nothing will complete. The wait runs
+ * out, the kernel records PA_ERR_TIMEOUT in the device error word and
+ * returns; the GPU context stays usable. Asynchronous on `stream`. */
+PA_API pa_status pa_selftest_bounded_wait(long long timeout_ns, cudaStream_t stream);
+
+/* Static description of a status code. */
+PA_API const char *pa_status_string(pa_status status);
+
+/* ABI version, (major << 16) | minor. */
+PA_API int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,582 @@
+// decode.cuh -- paged decode attention: split-KV kernel and log-sum-exp merge.
+//
+// What is computed (page "字节跳动 AI Infra (2)", question "KV Cache原理与优化"):
+// for each sequence b and query head h, softmax(scale * q . K^T) V over the
+// sequence's context_lens[b] cached tokens. K/V are reached through the
+// block table (question "vLLM与PagedAttention的原理": logical block i of the
+// sequence lives in physical block block_tables[b][i]); query heads share K/V
+// heads in groups (page "LLM推理优化", section 1.3). Long contexts are split
+// along the KV length into partitions whose partial results are merged by
+// log-sum-exp (page "字节跳动 AI Infra (2)", FlashDecoding row), each
+// partition using a running max / running sum softmax (page "LLM推理优化",
+// section 2.1, online softmax).
+//
+// Work decomposition: one CTA per (KV partition, KV head [x query-head tile],
+// sequence). Every K/V byte fetched serves all query heads of the GQA group.
+// Inside the CTA each warp owns every NW-th 16-token chunk of the partition
+// and runs its own NS-deep pipeline: lane 0 issues TMA copies of the chunk's
+// K and V rows (contiguous inside a page) into a stage and the warp waits on
+// that stage's mbarrier, so up to NW*NS chunks per CTA are in flight. The
+// table slice of the partition is prefetched into shared memory first.
+//
+// bf16: Q K^T and P V run on warp-level tensor cores (m16n8k16, fp32
+// accumulate) with the GQA group as the M dimension (padded to 16); TMA
+// writes K/V tiles with 128-byte swizzle so ldmatrix reads are conflict-free.
+// fp32: plain FMA (tensor cores would round fp32 inputs to tf32).
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+constexpr int kChunk = 16;             // tokens per staged chunk
+constexpr int kMaxPartition = 16384;   // tokens per KV partition, upper bound
+constexpr int kHeadsBf16 = 16;         // query heads per CTA, tensor-core path
+constexpr int kHeadsF32 = 8;           // query heads per CTA, fp32 path
+
+struct DecodeArgs {
+    void *out;
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    float *part_o;    // [B][H_q][S_max][D] (split mode only)
+    float *part_lse;  // [B][H_q][S_max], base-2 log-sum-exp of scaled scores
+    int num_seqs, H_q, H_kv, group, bs, NB, MB, max_ctx, P, S_max, n_htiles;
+    float scale_log2;  // scale * log2(e): scores are kept in the base-2 domain
+    unsigned long long timeout_ns;
+};
+
+// Context length of sequence b as the kernels use it: clamped to what the
+// host bound and the table row allow (anything outside is recorded).
+__device__ __forceinline__ int clamped_ctx(const DecodeArgs &a, int b, bool report) {
+    int ctx = a.context_lens[b];
+    const int cap = min(a.max_ctx, a.MB * a.bs);
+    if (ctx < 0 || ctx > cap) {
+        if (report) flag_error(PA_ERR_BAD_TABLE);
+        ctx = ctx < 0 ? 0 : cap;
+    }
+    return ctx;
+}
+
+template <int NW, int NS, int STAGE_BYTES>
+struct DecodeSmem {
+    static constexpr int kStages = NW * NS * STAGE_BYTES;
+    static constexpr int kBars = kStages;  // NW*NS mbarriers (8 B each)
+    static constexpr int kTable = kBars + NW * NS * 8;
+};
+
+// Cross-warp merge of per-warp online-softmax states and the final write:
+// the output (one partition) or the partition's normalised partial and lse.
+template <int D, int NW, int HT, typename OutT>
+__device__ __forceinline__ void decode_epilogue(const DecodeArgs &a, const float *red_o,
+                                                const float *red_m, const float *red_l, int b,
+                                                int h0, int nh, int s, int n_splits) {
+    constexpr int OS = D + 4;  // padded row stride of red_o
+    for (int idx = threadIdx.x; idx < nh * (D / 2); idx += NW * 32) {
+        const int row = idx / (D / 2);
+        const int d = (idx - row * (D / 2)) * 2;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * HT + row]);
+        float L = 0.f, o0 = 0.f, o1 = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float f = exp2f(red_m[w * HT + row] - M);
+                L += f * red_l[w * HT + row];
+                o0 += f * red_o[(w * HT + row) * OS + d];
+                o1 += f * red_o[(w * HT + row) * OS + d + 1];
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const size_t bh = (size_t)b * a.H_q + h0 + row;
+        if (n_splits <= 1) {
+            if constexpr (sizeof(OutT) == 2) {
+                *reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(a.out) + bh * D +
+                                              d) = pack_bf16x2(o0 * inv, o1 * inv);
+            } else {
+                *reinterpret_cast<float2 *>(reinterpret_cast<float *>(a.out) + bh * D + d) =
+                    make_float2(o0 * inv, o1 * inv);
+            }
+        } else {
+            *reinterpret_cast<float2 *>(a.part_o + (bh * a.S_max + s) * D + d) =
+                make_float2(o0 * inv, o1 * inv);
+            if (d == 0) a.part_lse[bh * a.S_max + s] = L > 0.f ? M + log2f(L) : -INFINITY;
+        }
+    }
+}
+
+template <int D, typename OutT>
+__device__ __forceinline__ void write_zero_rows(const DecodeArgs &a, int b, int h0, int nh) {
+    for (int idx = threadIdx.x; idx < nh * D; idx += blockDim.x) {
+        const size_t e = ((size_t)b * a.H_q + h0) * D + idx;
+        reinterpret_cast<OutT *>(a.out)[e] = OutT(0.f);
+    }
+}
+
+// ------------------------------------------------------------------ bf16
+template <int D, int NW, int NS>
+__global__ void __launch_bounds__(NW * 32)
+    decode_split_bf16(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv) {
+    constexpr int HT = kHeadsBf16;
+    constexpr int KSTEPS = D / 16;
+    constexpr int DTILES = D / 8;
+    constexpr int HALF = kChunk * D * 2;    // bytes of one K (or V) chunk
+    constexpr int STAGE = 2 * HALF;
+    constexpr int SUBTILE = kChunk * 128;   // one 64-wide swizzled sub-tile
+    using L = DecodeSmem<NW, NS, STAGE>;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + L::kTable);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int s = blockIdx.x;
+    const int kvh = blockIdx.y / a.n_htiles, ht = blockIdx.y - kvh * a.n_htiles;
+    const int b = blockIdx.z;
+    const int h0 = kvh * a.group + ht * HT;
+    const int nh = min(HT, a.group - ht * HT);
+
+    const int ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+    const int n_splits = (ctx + a.P - 1) / a.P;
+    if (s >= (n_splits > 0 ? n_splits : 1)) return;
+    if (ctx == 0) {
+        write_zero_rows<D, __nv_bfloat16>(a, b, h0, nh);
+        return;
+    }
+    const int tok0 = s * a.P;
+    const int tok1 = min(tok0 + a.P, ctx);
+    const int n_chunks = (tok1 - tok0 + kChunk - 1) / kChunk;
+    const int lb0 = tok0 / a.bs;
+    const int n_tbl = (tok1 - 1) / a.bs - lb0 + 1;
+
+    // table slice of this partition -> shared memory (ids checked once here)
+    const int32_t *row = a.block_tables + (size_t)b * a.MB + lb0;
+    for (int i = threadIdx.x; i < n_tbl; i += NW * 32) {
+        int id = __ldg(row + i);
+        if (id < 0 || id >= a.NB) {
+            flag_error(PA_ERR_BAD_TABLE);
+            id = -1;
+        }
+        tbl[i] = id;
+    }
+    const uint32_t bar0 = sbase + L::kBars + warp * NS * 8;
+    if (lane == 0) {
+        for (int st = 0; st < NS; ++st) mbar_init(bar0 + st * 8, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int my_n = n_chunks > warp ? (n_chunks - warp + NW - 1) / NW : 0;
+    const uint32_t stage0 = sbase + warp * NS * STAGE;
+
+    auto issue = [&](int i) {  // lane 0: chunk i of this warp -> stage i % NS
+        const int st = i % NS;
+        const uint32_t bar = bar0 + st * 8;
+        const int t = tok0 + (warp + i * NW) * kChunk;
+        const int id = tbl[t / a.bs - lb0];
+        if (id < 0) {
+            mbar_arrive(bar);  // nothing to load; the chunk is skipped
+            return;
+        }
+        mbar_arrive_expect_tx(bar, STAGE);
+        const uint32_t kdst = stage0 + st * STAGE;
+        const int off = t % a.bs;
+#pragma unroll
+        for (int sub = 0; sub < D / 64; ++sub) {
+            tma_load_4d(kdst + sub * SUBTILE, &tmk, bar, sub * 64, off, kvh, id);
+            tma_load_4d(kdst + HALF + sub * SUBTILE, &tmv, bar, sub * 64, off, kvh, id);
+        }
+    };
+    if (lane == 0) {
+        for (int i = 0; i < NS && i < my_n; ++i) issue(i);
+    }
+
+    // Q fragments (rows = query heads of the tile, zero past nh)
+    const int g = lane >> 2, tig = lane & 3;
+    uint32_t qa[KSTEPS][4];
+    {
+        const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q) +
+                                  ((size_t)b * a.H_q + h0) * D;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int qr = g + 8 * (r & 1);
+                const int col = ks * 16 + 2 * tig + 8 * (r >> 1);
+                qa[ks][r] = qr < nh ? __ldg(reinterpret_cast<const uint32_t *>(qb + qr * D + col))
+                                    : 0u;
+            }
+    }
+
+    float o[DTILES][4];
+#pragma unroll
+    for (int i = 0; i < DTILES; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    int done = 0;
+    bool failed = false;
+
+    for (int i = 0; i < my_n; ++i) {
+        const int st = i % NS;
+        // the verdict is made warp-uniform: the tensor-core steps below need
+        // every lane
+        const bool ok = mbar_wait(bar0 + st * 8, (i / NS) & 1, a.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+            failed = true;
+            break;
+        }
+        done = i + 1;
+        const int t = tok0 + (warp + i * NW) * kChunk;
+        const int id = tbl[t / a.bs - lb0];
+        if (id >= 0) {
+            const int valid = min(kChunk, tok1 - t);
+            const uint32_t kb = stage0 + st * STAGE;
+            const uint32_t vb = kb + HALF;
+            if (valid < kChunk) {
+                // rows past the context may hold anything (NaN, Inf): zero
+                // the V rows so that P = 0 cannot turn them into NaN
+                const int nvec = (kChunk - valid) * (D / 8);
+                for (int e = lane; e < nvec; e += 32) {
+                    const int r = valid + e / (D / 8);
+                    const int u = e % (D / 8);
+                    const uint32_t addr = vb + (u / 8) * SUBTILE + r * 128 + (u % 8) * 16;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            // S = Q K^T over 16 tokens (two n-tiles of 8)
+            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            {
+                const int mi = lane >> 3;
+                const int r = (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const int col = ks * 16 + (mi & 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kb + (col / 64) * SUBTILE + sw128(r, (col % 64) / 8), b0, b1, b2, b3);
+                    mma_bf16_16816(sc[0], qa[ks], b0, b1);
+                    mma_bf16_16816(sc[1], qa[ks], b2, b3);
+                }
+            }
+            // online softmax in base 2; rows g (c0,c1) and g+8 (c2,c3)
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = nt * 8 + 2 * tig + (e & 1);
+                    sc[nt][e] = tok < valid ? sc[nt][e] * a.scale_log2 : -INFINITY;
+                }
+            mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+            mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
+            m0 = mn0;
+            m1 = mn1;
+            uint32_t pa[4];
+            pa[0] = pack_bf16x2(exp2f(sc[0][0] - mn0), exp2f(sc[0][1] - mn0));
+            pa[1] = pack_bf16x2(exp2f(sc[0][2] - mn1), exp2f(sc[0][3] - mn1));
+            pa[2] = pack_bf16x2(exp2f(sc[1][0] - mn0), exp2f(sc[1][1] - mn0));
+            pa[3] = pack_bf16x2(exp2f(sc[1][2] - mn1), exp2f(sc[1][3] - mn1));
+            // the denominator sums the same rounded weights the numerator uses
+            l0 = l0 * c0 + (bf16_lo(pa[0]) + bf16_hi(pa[0]) + bf16_lo(pa[2]) + bf16_hi(pa[2]));
+            l1 = l1 * c1 + (bf16_lo(pa[1]) + bf16_hi(pa[1]) + bf16_lo(pa[3]) + bf16_hi(pa[3]));
+#pragma unroll
+            for (int dt = 0; dt < DTILES; ++dt) {
+                o[dt][0] *= c0;
+                o[dt][1] *= c0;
+                o[dt][2] *= c1;
+                o[dt][3] *= c1;
+            }
+            // O += P V  (V^T fragments via transposed ldmatrix)
+            {
+                const int mi = lane >> 3;
+                const int r = (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+                for (int dp = 0; dp < DTILES / 2; ++dp) {
+                    const int col = (dp * 2 + (mi >> 1)) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vb + (col / 64) * SUBTILE + sw128(r, (col % 64) / 8), b0, b1, b2,
+                              b3);
+                    mma_bf16_16816(o[2 * dp], pa, b0, b1);
+                    mma_bf16_16816(o[2 * dp + 1], pa, b2, b3);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && i + NS < my_n) {
+            fence_proxy_async_smem();  // order this warp's reads before the refill
+            issue(i + NS);
+        }
+    }
+    if (failed) {
+        flag_error(PA_ERR_TIMEOUT);
+        // let copies already issued into this warp's stages land (bounded)
+        const int issued = min(my_n, done + NS);
+        for (int i = done; i < issued; ++i)
+            if (!mbar_wait(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns)) break;
+    }
+
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+
+    __syncthreads();  // every warp is done with its stages: reuse them
+    constexpr int OS = D + 4;
+    float *red_o = reinterpret_cast<float *>(smem);
+    float *red_m = reinterpret_cast<float *>(smem + NW * HT * OS * 4);
+    float *red_l = red_m + NW * HT;
+    if (tig == 0) {
+        red_m[warp * HT + g] = m0;
+        red_m[warp * HT + g + 8] = m1;
+        red_l[warp * HT + g] = l0;
+        red_l[warp * HT + g + 8] = l1;
+    }
+#pragma unroll
+    for (int dt = 0; dt < DTILES; ++dt) {
+        const int d = dt * 8 + 2 * tig;
+        *reinterpret_cast<float2 *>(red_o + (warp * HT + g) * OS + d) = make_float2(o[dt][0], o[dt][1]);
+        *reinterpret_cast<float2 *>(red_o + (warp * HT + g + 8) * OS + d) =
+            make_float2(o[dt][2], o[dt][3]);
+    }
+    __syncthreads();
+    decode_epilogue<D, NW, HT, __nv_bfloat16>(a, red_o, red_m, red_l, b, h0, nh, s, n_splits);
+}
+
+// ------------------------------------------------------------------ fp32
+template <int D, int NW, int NS>
+__global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constant__ DecodeArgs a) {
+    constexpr int HT = kHeadsF32;
+    constexpr int VEC = D / 32;          // dims per lane
+    constexpr int HALF = kChunk * D * 4;
+    constexpr int STAGE = 2 * HALF;
+    using L = DecodeSmem<NW, NS, STAGE>;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + L::kTable);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int s = blockIdx.x;
+    const int kvh = blockIdx.y / a.n_htiles, ht = blockIdx.y - kvh * a.n_htiles;
+    const int b = blockIdx.z;
+    const int h0 = kvh * a.group + ht * HT;
+    const int nh = min(HT, a.group - ht * HT);
+
+    const int ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+    const int n_splits = (ctx + a.P - 1) / a.P;
+    if (s >= (n_splits > 0 ? n_splits : 1)) return;
+    if (ctx == 0) {
+        write_zero_rows<D, float>(a, b, h0, nh);
+        return;
+    }
+    const int tok0 = s * a.P;
+    const int tok1 = min(tok0 + a.P, ctx);
+    const int n_chunks = (tok1 - tok0 + kChunk - 1) / kChunk;
+    const int lb0 = tok0 / a.bs;
+    const int n_tbl = (tok1 - 1) / a.bs - lb0 + 1;
+
+    const int32_t *row = a.block_tables + (size_t)b * a.MB + lb0;
+    for (int i = threadIdx.x; i < n_tbl; i += NW * 32) {
+        int id = __ldg(row + i);
+        if (id < 0 || id >= a.NB) {
+            flag_error(PA_ERR_BAD_TABLE);
+            id = -1;
+        }
+        tbl[i] = id;
+    }
+    const uint32_t bar0 = sbase + L::kBars + warp * NS * 8;
+    if (lane == 0) {
+        for (int st = 0; st < NS; ++st) mbar_init(bar0 + st * 8, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int my_n = n_chunks > warp ? (n_chunks - warp + NW - 1) / NW : 0;
+    const uint32_t stage0 = sbase + warp * NS * STAGE;
+    const float *kc = reinterpret_cast<const float *>(a.k_cache);
+    const float *vc = reinterpret_cast<const float *>(a.v_cache);
+
+    auto issue = [&](int i) {
+        const int st = i % NS;
+        const uint32_t bar = bar0 + st * 8;
+        const int t = tok0 + (warp + i * NW) * kChunk;
+        const int id = tbl[t / a.bs - lb0];
+        if (id < 0) {
+            mbar_arrive(bar);
+            return;
+        }
+        mbar_arrive_expect_tx(bar, STAGE);
+        const size_t page = (((size_t)id * a.H_kv + kvh) * a.bs + (t % a.bs)) * D;
+        bulk_load(stage0 + st * STAGE, kc + page, HALF, bar);
+        bulk_load(stage0 + st * STAGE + HALF, vc + page, HALF, bar);
+    };
+    if (lane == 0) {
+        for (int i = 0; i < NS && i < my_n; ++i) issue(i);
+    }
+
+    float qv[HT][VEC], acc[HT][VEC], mrow[HT], lrow[HT];
+    {
+        const float *qb = reinterpret_cast<const float *>(a.q) + ((size_t)b * a.H_q + h0) * D;
+#pragma unroll
+        for (int g = 0; g < HT; ++g) {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                qv[g][v] = g < nh ? __ldg(qb + g * D + lane * VEC + v) : 0.f;
+                acc[g][v] = 0.f;
+            }
+            mrow[g] = -INFINITY;
+            lrow[g] = 0.f;
+        }
+    }
+    int done = 0;
+    bool failed = false;
+    for (int i = 0; i < my_n; ++i) {
+        const int st = i % NS;
+        // the verdict is made warp-uniform: the tensor-core steps below need
+        // every lane
+        const bool ok = mbar_wait(bar0 + st * 8, (i / NS) & 1, a.timeout_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+            failed = true;
+            break;
+        }
+        done = i + 1;
+        const int t = tok0 + (warp + i * NW) * kChunk;
+        const int id = tbl[t / a.bs - lb0];
+        if (id >= 0) {
+            const int valid = min(kChunk, tok1 - t);
+            const float *ks = reinterpret_cast<const float *>(smem + warp * NS * STAGE + st * STAGE);
+            const float *vs = ks + kChunk * D;
+            for (int j = 0; j < valid; ++j) {  // tokens past the context are never touched
+                float kk[VEC], vv[VEC];
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    kk[v] = ks[j * D + lane * VEC + v];
+                    vv[v] = vs[j * D + lane * VEC + v];
+                }
+#pragma unroll
+                for (int g = 0; g < HT; ++g) {
+                    if (g < nh) {
+                        float dot = 0.f;
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) dot = fmaf(qv[g][v], kk[v], dot);
+                        const float sc = warp_sum(dot) * a.scale_log2;
+                        const float mn = fmaxf(mrow[g], sc);
+                        const float c = exp2f(mrow[g] - mn);
+                        const float p = exp2f(sc - mn);
+                        lrow[g] = lrow[g] * c + p;
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(acc[g][v], c, p * vv[v]);
+                        mrow[g] = mn;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && i + NS < my_n) {
+            fence_proxy_async_smem();  // order this warp's reads before the refill
+            issue(i + NS);
+        }
+    }
+    if (failed) {
+        flag_error(PA_ERR_TIMEOUT);
+        const int issued = min(my_n, done + NS);
+        for (int i = done; i < issued; ++i)
+            if (!mbar_wait(bar0 + (i % NS) * 8, (i / NS) & 1, a.timeout_ns)) break;
+    }
+
+    __syncthreads();
+    constexpr int OS = D + 4;
+    float *red_o = reinterpret_cast<float *>(smem);
+    float *red_m = reinterpret_cast<float *>(smem + NW * HT * OS * 4);
+    float *red_l = red_m + NW * HT;
+#pragma unroll
+    for (int g = 0; g < HT; ++g) {
+        if (lane == 0) {
+            red_m[warp * HT + g] = mrow[g];
+            red_l[warp * HT + g] = lrow[g];
+        }
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) red_o[(warp * HT + g) * OS + lane * VEC + v] = acc[g][v];
+    }
+    __syncthreads();
+    decode_epilogue<D, NW, HT, float>(a, red_o, red_m, red_l, b, h0, nh, s, n_splits);
+}
+
+// ------------------------------------------------------------- LSE merge
+// One CTA (4 warps) per (sequence, query head) with more than one
+// partition: out = sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M).
+template <int D, typename OutT>
+__global__ void __launch_bounds__(128) decode_reduce(const __grid_constant__ DecodeArgs a) {
+    constexpr int NWR = 4;
+    constexpr int VEC = D / 32;
+    const int bh = blockIdx.x;
+    const int b = bh / a.H_q;
+    const int ctx = clamped_ctx(a, b, false);
+    const int n = (ctx + a.P - 1) / a.P;
+    if (n <= 1) return;
+    const float *lse = a.part_lse + (size_t)bh * a.S_max;
+    const float *po = a.part_o + (size_t)bh * a.S_max * D;
+    __shared__ float red[NWR][D + 1];
+    __shared__ float wsum[NWR];
+    __shared__ float smax[NWR];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    float M = -INFINITY;
+    for (int s = threadIdx.x; s < n; s += 128) M = fmaxf(M, lse[s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) smax[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(smax[0], smax[1]), fmaxf(smax[2], smax[3]));
+
+    float acc[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+    float W = 0.f;
+    if (M != -INFINITY) {
+        for (int s = warp; s < n; s += NWR) {
+            const float w = exp2f(lse[s] - M);
+            W += w;
+            const float *src = po + (size_t)s * D + lane * VEC;
+            if constexpr (VEC == 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(src);
+                acc[0] = fmaf(w, x.x, acc[0]);
+                acc[1] = fmaf(w, x.y, acc[1]);
+                acc[2] = fmaf(w, x.z, acc[2]);
+                acc[3] = fmaf(w, x.w, acc[3]);
+            } else {
+                const float2 x = *reinterpret_cast<const float2 *>(src);
+                acc[0] = fmaf(w, x.x, acc[0]);
+                acc[1] = fmaf(w, x.y, acc[1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) red[warp][lane * VEC + v] = acc[v];
+    if (lane == 0) wsum[warp] = W;
+    __syncthreads();
+    if (threadIdx.x < D) {
+        const int d = threadIdx.x;
+        const float Wt = wsum[0] + wsum[1] + wsum[2] + wsum[3];
+        const float x = red[0][d] + red[1][d] + red[2][d] + red[3][d];
+        const float r = Wt > 0.f ? x / Wt : 0.f;
+        reinterpret_cast<OutT *>(a.out)[(size_t)bh * D + d] = OutT(r);
+    }
+}
+
+}  // namespace pa

@@ -1,0 +1,413 @@
+// pa_lib.cu -- the C ABI of libpa.so (declared in include/pa.h): host-side
+// argument checks, launch configuration, TMA descriptors, and the small
+// service kernels (table check, error word, bounded-wait self test).
+//
+// Everything is one translation unit so that every kernel records into the
+// same device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "pa.h"
+#include "pa_device.cuh"
+#include "reshape_and_cache.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+using namespace pa;
+
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+bool block_size_ok(int bs) { return bs == 16 || bs == 32 || bs == 64; }
+
+pa_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime so
+// that the library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// A 4-D view [num_blocks][H_kv][bs][D] of a bf16 cache with a box of
+// box_rows tokens x 64 dims (128 bytes) and 128-byte swizzle.
+bool encode_cache_map(CUtensorMap *m, const void *cache, int NB, int H_kv, int bs, int D,
+                      int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)bs, (cuuint64_t)H_kv, (cuuint64_t)NB};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)bs * D * 2,
+                             (cuuint64_t)H_kv * bs * D * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(cache), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// KV tokens per partition, or -1 if the request cannot be met.
+int partition_tokens(int max_ctx, int partition_size) {
+    if (max_ctx < 0) return -1;
+    if (partition_size > 0) {
+        if (partition_size % kChunk != 0 || partition_size > kMaxPartition) return -1;
+        return partition_size;
+    }
+    const int whole = ((max_ctx > 0 ? max_ctx : 1) + kChunk - 1) / kChunk * kChunk;
+    if (partition_size < 0) return whole <= kMaxPartition ? whole : -1;
+    return max_ctx <= 1024 ? whole : 512;  // automatic
+}
+
+size_t workspace_bytes(int B, int H_q, int D, int max_ctx, int P) {
+    const long long S = (max_ctx + P - 1) / P;
+    if (S <= 1) return 0;
+    const size_t o = (size_t)B * H_q * S * D * sizeof(float);
+    const size_t l = (size_t)B * H_q * S * sizeof(float);
+    return (o + 255) / 256 * 256 + (l + 255) / 256 * 256;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// ------------------------------------------------------------- decode
+// Launch shape of the split kernel: warps per CTA and pipeline stages per
+// warp. PA_DECODE_PIPE=<warps>x<stages> selects another built shape.
+struct Pipe {
+    int nw, ns;
+};
+
+Pipe decode_pipe() {
+    static Pipe p = [] {
+        Pipe r{4, 3};
+        if (const char *e = std::getenv("PA_DECODE_PIPE")) {
+            int w = 0, s = 0;
+            if (sscanf(e, "%dx%d", &w, &s) == 2) r = Pipe{w, s};
+        }
+        return r;
+    }();
+    return p;
+}
+
+template <int D, int NW, int NS>
+pa_status launch_decode_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
+                             dim3 grid, cudaStream_t st) {
+    constexpr int STAGE = 2 * kChunk * D * 2;
+    using L = DecodeSmem<NW, NS, STAGE>;
+    const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
+    auto k = decode_split_bf16<D, NW, NS>;
+    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
+    k<<<grid, NW * 32, smem, st>>>(a, mk, mv);
+    return launch_status();
+}
+
+template <int D, int NW, int NS>
+pa_status launch_decode_f32(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
+    constexpr int STAGE = 2 * kChunk * D * 4;
+    using L = DecodeSmem<NW, NS, STAGE>;
+    const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
+    auto k = decode_split_f32<D, NW, NS>;
+    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
+    k<<<grid, NW * 32, smem, st>>>(a);
+    return launch_status();
+}
+
+template <int D>
+pa_status dispatch_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
+                        dim3 grid, cudaStream_t st) {
+    const Pipe p = decode_pipe();
+    if (p.nw == 4 && p.ns == 2) return launch_decode_bf16<D, 4, 2>(a, mk, mv, grid, st);
+    if (p.nw == 4 && p.ns == 4) return launch_decode_bf16<D, 4, 4>(a, mk, mv, grid, st);
+    if (p.nw == 8 && p.ns == 2) return launch_decode_bf16<D, 8, 2>(a, mk, mv, grid, st);
+    return launch_decode_bf16<D, 4, 3>(a, mk, mv, grid, st);
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+int pa_version(void) { return (1 << 16) | 0; }
+
+const char *pa_status_string(pa_status s) {
+    switch (s) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARG: return "invalid argument";
+        case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case PA_ERR_WORKSPACE: return "workspace missing or too small";
+        case PA_ERR_BAD_TABLE: return "block id, slot or length out of range";
+        case PA_ERR_TIMEOUT: return "bounded device wait ran out";
+        case PA_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                               const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               cudaStream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (!head_dim_ok(head_dim) || !block_size_ok(block_size)) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(slot_mapping, 8))
+        return PA_ERR_INVALID_ARG;
+    const int elem = dtype == PA_BF16 ? 2 : 4;
+    ReshapeArgs a;
+    a.key = static_cast<const uint4 *>(key);
+    a.value = static_cast<const uint4 *>(value);
+    a.k_cache = static_cast<uint4 *>(k_cache);
+    a.v_cache = static_cast<uint4 *>(v_cache);
+    a.slot_mapping = slot_mapping;
+    a.vecs_per_row = head_dim * elem / 16;
+    a.vecs_per_token = num_kv_heads * a.vecs_per_row;
+    a.total_vecs = (long long)num_tokens * a.vecs_per_token;
+    a.num_kv_heads = num_kv_heads;
+    a.block_size = block_size;
+    a.num_slots = (long long)num_blocks * block_size;
+    const long long blocks = (a.total_vecs + 255) / 256;
+    if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    reshape_and_cache_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    return launch_status();
+}
+
+int pa_decode_partition_tokens(int max_context_len, int partition_size) {
+    return partition_tokens(max_context_len, partition_size);
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                int partition_size) {
+    const int P = partition_tokens(max_context_len, partition_size);
+    if (P <= 0 || num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+    return workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, P);
+}
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                    int partition_size, void *workspace, size_t workspace_bytes_given,
+                    pa_dtype dtype, cudaStream_t stream) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0 || !head_dim_ok(head_dim) || !block_size_ok(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PA_ERR_INVALID_ARG;
+    const int P = partition_tokens(max_context_len, partition_size);
+    if (P <= 0) return partition_size > 0 ? PA_ERR_INVALID_ARG : PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4))
+        return PA_ERR_INVALID_ARG;
+    const size_t need = workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, P);
+    if (need > 0 && (!workspace || workspace_bytes_given < need || !aligned(workspace, 256)))
+        return PA_ERR_WORKSPACE;
+    const int group = num_q_heads / num_kv_heads;
+    const int ht = dtype == PA_BF16 ? kHeadsBf16 : kHeadsF32;
+    const int n_htiles = (group + ht - 1) / ht;
+    const long long S = (max_context_len + P - 1) / P;
+    const long long gy = (long long)num_kv_heads * n_htiles;
+    if (gy > 65535 || num_seqs > 65535 || S > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+
+    DecodeArgs a;
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    const long long S1 = S > 0 ? S : 1;
+    a.part_o = need ? static_cast<float *>(workspace) : nullptr;
+    a.part_lse = need ? reinterpret_cast<float *>(
+                            static_cast<char *>(workspace) +
+                            ((size_t)num_seqs * num_q_heads * S1 * head_dim * 4 + 255) / 256 * 256)
+                      : nullptr;
+    a.num_seqs = num_seqs;
+    a.H_q = num_q_heads;
+    a.H_kv = num_kv_heads;
+    a.group = group;
+    a.bs = block_size;
+    a.NB = num_blocks;
+    a.MB = max_blocks_per_seq;
+    a.max_ctx = max_context_len;
+    a.P = P;
+    a.S_max = (int)S1;
+    a.n_htiles = n_htiles;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.timeout_ns = kWaitTimeoutNs;
+
+    const dim3 grid((unsigned)S1, (unsigned)gy, (unsigned)num_seqs);
+    pa_status st;
+    if (dtype == PA_BF16) {
+        CUtensorMap mk, mv;
+        if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, block_size, head_dim,
+                              kChunk) ||
+            !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, block_size, head_dim, kChunk))
+            return PA_ERR_CUDA;
+        st = head_dim == 128 ? dispatch_bf16<128>(a, mk, mv, grid, stream)
+                             : dispatch_bf16<64>(a, mk, mv, grid, stream);
+        if (st != PA_OK) return st;
+        if (S1 > 1) {
+            if (head_dim == 128)
+                decode_reduce<128, __nv_bfloat16><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
+            else
+                decode_reduce<64, __nv_bfloat16><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
+            st = launch_status();
+        }
+    } else {
+        st = head_dim == 128 ? launch_decode_f32<128, 4, 2>(a, grid, stream)
+                             : launch_decode_f32<64, 4, 2>(a, grid, stream);
+        if (st != PA_OK) return st;
+        if (S1 > 1) {
+            if (head_dim == 128)
+                decode_reduce<128, float><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
+            else
+                decode_reduce<64, float><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
+            st = launch_status();
+        }
+    }
+    return st;
+}
+
+pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *block_tables, const int32_t *context_lens,
+                           const int32_t *query_start_loc, int num_chunks, int max_query_len,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, int max_blocks_per_seq, float scale, pa_dtype dtype,
+                           cudaStream_t stream) {
+    if (num_chunks < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (dtype != PA_BF16 || num_q_heads % num_kv_heads != 0 || head_dim != 128 ||
+        !block_size_ok(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if (num_chunks == 0 || max_query_len == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
+        return PA_ERR_INVALID_ARG;
+    return launch_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                          num_chunks, max_query_len, num_q_heads, num_kv_heads, head_dim,
+                          block_size, num_blocks, max_blocks_per_seq, scale, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------- service kernels
+namespace {
+
+__global__ void check_tables_kernel(const int32_t *tables, const int32_t *lens, int MB, int bs,
+                                    int NB, int32_t *bad) {
+    __shared__ int row_bad;
+    const int r = blockIdx.x;
+    if (threadIdx.x == 0) row_bad = 0;
+    __syncthreads();
+    const int len = lens[r];
+    if (len < 0 || (long long)len > (long long)MB * bs) {
+        if (threadIdx.x == 0) row_bad = 1;
+    } else {
+        const int n = (len + bs - 1) / bs;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const int id = tables[(size_t)r * MB + i];
+            if (id < 0 || id >= NB) row_bad = 1;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && row_bad) atomicAdd(bad, 1);
+}
+
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // nothing arrives on this barrier: the bounded wait must run out
+    if (!mbar_wait(b, 0, timeout_ns) && threadIdx.x == 0) flag_error(PA_ERR_TIMEOUT);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_check_tables(const int32_t *block_tables, const int32_t *context_lens, int rows,
+                          int max_blocks_per_seq, int block_size, int num_blocks,
+                          int32_t *d_scratch, int *bad_rows, cudaStream_t stream) {
+    if (rows < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (bad_rows) *bad_rows = 0;
+    if (rows == 0) return PA_OK;
+    if (!block_tables || !context_lens || !d_scratch) return PA_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(d_scratch, 0, sizeof(int32_t), stream) != cudaSuccess) return PA_ERR_CUDA;
+    check_tables_kernel<<<rows, 128, 0, stream>>>(block_tables, context_lens, max_blocks_per_seq,
+                                                  block_size, num_blocks, d_scratch);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, d_scratch, sizeof(int32_t), cudaMemcpyDeviceToHost, stream) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (bad_rows) *bad_rows = h;
+    return h ? PA_ERR_BAD_TABLE : PA_OK;
+}
+
+pa_status pa_device_error(int *status, int clear) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, pa::g_pa_error, sizeof(int)) != cudaSuccess) return PA_ERR_CUDA;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(pa::g_pa_error, &zero, sizeof(int)) != cudaSuccess)
+            return PA_ERR_CUDA;
+    }
+    if (status) *status = v;
+    return PA_OK;
+}
+
+pa_status pa_selftest_bounded_wait(long long timeout_ns, cudaStream_t stream) {
+    if (timeout_ns <= 0 || timeout_ns > 10000000000LL) return PA_ERR_INVALID_ARG;
+    selftest_wait_kernel<<<1, 32, 0, stream>>>((unsigned long long)timeout_ns);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,196 @@
+"""Thin ctypes binding of ``libpa.so`` (C ABI in ``include/pa.h``).
+
+Each function has the name of the C entry point it calls and only marshals
+arguments: torch tensors become device pointers and sizes, the current torch
+CUDA stream becomes the ``cudaStream_t``, and a non-OK status becomes
+:class:`PAError`. Every step of the computation runs in the library's CUDA
+kernels. The library must have been built (``python -m
+pagedattention_paged_kv_02_b200.build``); loading fails loudly otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE = 0, 1, 2, 3
+PA_ERR_BAD_TABLE, PA_ERR_TIMEOUT, PA_ERR_CUDA = 4, 5, 6
+PA_F32, PA_BF16 = 0, 1
+
+EXPORTS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_partition_tokens",
+           "pa_decode", "pa_prefill_chunk", "pa_check_tables", "pa_device_error",
+           "pa_selftest_bounded_wait", "pa_status_string", "pa_version")
+
+
+class PAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded on first use)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m pagedattention_paged_kv_02_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, F, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float,
+                            ctypes.c_size_t)
+        L.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P]
+        L.pa_decode_workspace_size.argtypes = [I, I, I, I, I]
+        L.pa_decode_workspace_size.restype = SZ
+        L.pa_decode_partition_tokens.argtypes = [I, I]
+        L.pa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, SZ, I, P]
+        L.pa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P]
+        L.pa_check_tables.argtypes = [P, P, I, I, I, I, P, ctypes.POINTER(I), P]
+        L.pa_device_error.argtypes = [ctypes.POINTER(I), I]
+        L.pa_selftest_bounded_wait.argtypes = [I64, P]
+        L.pa_status_string.argtypes = [I]
+        L.pa_status_string.restype = ctypes.c_char_p
+        for f in ("pa_reshape_and_cache", "pa_decode", "pa_prefill_chunk", "pa_check_tables",
+                  "pa_device_error", "pa_selftest_bounded_wait", "pa_decode_partition_tokens",
+                  "pa_version"):
+            getattr(L, f).restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().pa_status_string(int(status)).decode()
+
+
+def _call(fn: str, *args):
+    st = getattr(lib(), fn)(*args)
+    if st != PA_OK:
+        raise PAError(fn, st)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    if t.dtype == torch.float32:
+        return PA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensors expected")
+    if not t.is_contiguous():
+        raise ValueError("contiguous tensors expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_int(t: torch.Tensor, dtype, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# ---------------------------------------------------------------------------
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None) -> None:
+    """Scatter ``key``/``value`` [T, H_kv, D] into the caches [NB, H_kv, bs, D]
+    at ``slot_mapping`` (int64 [T])."""
+    _check_int(slot_mapping, torch.int64, "slot_mapping")
+    NB, H_kv, bs, D = k_cache.shape
+    T = slot_mapping.numel()
+    if key.shape != (T, H_kv, D) or value.shape != (T, H_kv, D):
+        raise ValueError("key/value must be [num_tokens, num_kv_heads, head_dim]")
+    if not (key.dtype == value.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("key, value and caches must share one dtype")
+    _call("pa_reshape_and_cache", _p(key), _p(value), _p(k_cache), _p(v_cache),
+          _p(slot_mapping), T, H_kv, D, bs, NB, _dt(k_cache), _stream(stream))
+
+
+def pa_decode_workspace_size(num_seqs: int, num_q_heads: int, head_dim: int,
+                             max_context_len: int, partition_size: int = 0) -> int:
+    return int(lib().pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                              partition_size))
+
+
+def pa_decode_partition_tokens(max_context_len: int, partition_size: int = 0) -> int:
+    return int(lib().pa_decode_partition_tokens(max_context_len, partition_size))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+              scale: float, partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> None:
+    """Paged decode attention into ``out`` [B, H_q, D]. ``workspace`` is a
+    device byte buffer of at least :func:`pa_decode_workspace_size` bytes
+    (may be None when that size is 0)."""
+    _check_int(block_tables, torch.int32, "block_tables")
+    _check_int(context_lens, torch.int32, "context_lens")
+    B, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
+        raise ValueError("out must match q; caches must share head_dim")
+    if not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("q and caches must share one dtype")
+    MB = block_tables.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _call("pa_decode", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
+          _p(context_lens), B, H_q, H_kv, D, bs, NB, MB, int(max_context_len), float(scale),
+          int(partition_size), _p(workspace), ws_bytes, _dt(q), _stream(stream))
+
+
+def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                     max_query_len: int, scale: float, stream=None) -> None:
+    """Chunked prefill into ``out`` [total_q, H_q, D]."""
+    for t, n in ((block_tables, "block_tables"), (context_lens, "context_lens"),
+                 (query_start_loc, "query_start_loc")):
+        _check_int(t, torch.int32, n)
+    total_q, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
+        raise ValueError("out must match q; caches must share head_dim")
+    n_chunks = query_start_loc.numel() - 1
+    MB = block_tables.shape[1]
+    _call("pa_prefill_chunk", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
+          _p(context_lens), _p(query_start_loc), n_chunks, int(max_query_len), H_q, H_kv, D, bs,
+          NB, MB, float(scale), _dt(q), _stream(stream))
+
+
+def pa_check_tables(block_tables, context_lens, block_size: int, num_blocks: int,
+                    scratch: Optional[torch.Tensor] = None, stream=None) -> int:
+    """Synchronous device check of tables/lengths; returns the number of bad
+    rows (0 when all are valid)."""
+    rows, MB = block_tables.shape
+    if scratch is None:
+        scratch = torch.empty(1, dtype=torch.int32, device=block_tables.device)
+    bad = ctypes.c_int(0)
+    st = lib().pa_check_tables(_p(block_tables), _p(context_lens), rows, MB, block_size,
+                               num_blocks, _p(scratch), ctypes.byref(bad), _stream(stream))
+    if st not in (PA_OK, PA_ERR_BAD_TABLE):
+        raise PAError("pa_check_tables", st)
+    return int(bad.value)
+
+
+def pa_device_error(clear: bool = False) -> int:
+    """The sticky device error word (synchronous)."""
+    v = ctypes.c_int(0)
+    _call("pa_device_error", ctypes.byref(v), 1 if clear else 0)
+    return int(v.value)
+
+
+def pa_selftest_bounded_wait(timeout_ns: int, stream=None) -> None:
+    _call("pa_selftest_bounded_wait", int(timeout_ns), _stream(stream))
+
+
+def pa_version() -> int:
+    return int(lib().pa_version())
