@@ -260,8 +260,10 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
-def make_batch(name: str, seed: int):
+def make_batch(name: str, seed: int, num_blocks=None):
     from pagedattention_paged_kv_02_b200 import workloads as W
+    if num_blocks:
+        return W.WORKLOADS[name](seed=seed, num_blocks=num_blocks)
     return W.WORKLOADS[name](seed=seed)
 
 
@@ -331,7 +333,7 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     dist = init_dist(world, "nccl")
-    batch = make_batch(args.workload, seed=rank)
+    batch = make_batch(args.workload, seed=rank, num_blocks=args.num_blocks)
     r = Runner(batch, dev)
     hbm, bf16, bf16_sus, basis = load_peaks()
 
@@ -547,7 +549,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     import oracle
-    batch = make_batch(args.workload, seed=0)
+    batch = make_batch(args.workload, seed=0, num_blocks=args.num_blocks)
     k, v = batch.k_cache, batch.v_cache
     total = args.steps + args.warmup
     t = time.perf_counter()
@@ -589,6 +591,8 @@ def main(argv=None):
                              "mixed_prefill_decode"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--num-blocks", type=int, default=None,
+                    help="physical pool size override (a smaller pool for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     args = ap.parse_args(argv)

@@ -281,37 +281,37 @@ def tiny_fp32(seed: int = 0) -> Batch:
                         scale=1.0 / 8.0, name="tiny_fp32_b4_d64")
 
 
-def llama7b_decode(seed: int = 0) -> Batch:
+def llama7b_decode(seed: int = 0, num_blocks: int = 16384) -> Batch:
     """Llama-2-7B-shaped decode: 64 sequences with lengths uniform in
     [128, 2048], 32/32 heads, head_dim 128, 16-token blocks, 16384-block pool,
     bf16, N(0,1)."""
     gen = torch.Generator().manual_seed(seed + 7919)
     lens = torch.randint(128, 2049, (64,), generator=gen).tolist()
-    return decode_batch(lens, 32, 32, 128, 16, 16384, torch.bfloat16, 1.0, seed,
+    return decode_batch(lens, 32, 32, 128, 16, num_blocks, torch.bfloat16, 1.0, seed,
                         max_blocks_per_seq=128, name="llama7b_decode_b64_h32_d128_bs16")
 
 
-def gqa_decode(seed: int = 0) -> Batch:
+def gqa_decode(seed: int = 0, num_blocks: int = 32768) -> Batch:
     """GQA decode: 128 sequences, lengths log-normal with median 1024 and
     sigma 0.75 (natural-log scale) clipped to [16, 4096], 64 q / 8 kv heads,
     head_dim 128, 16-token blocks, 32768-block pool, bf16, N(0,1)."""
     gen = torch.Generator().manual_seed(seed + 104729)
     z = torch.randn(128, generator=gen, dtype=torch.float64)
     lens = torch.exp(math.log(1024.0) + 0.75 * z).round().clamp(16, 4096).to(torch.int64).tolist()
-    return decode_batch(lens, 64, 8, 128, 16, 32768, torch.bfloat16, 1.0, seed,
+    return decode_batch(lens, 64, 8, 128, 16, num_blocks, torch.bfloat16, 1.0, seed,
                         max_blocks_per_seq=256, name="gqa_decode_b128_h64kv8_d128_bs16")
 
 
-def long_context_decode(seed: int = 0) -> Batch:
+def long_context_decode(seed: int = 0, num_blocks: int = 8192) -> Batch:
     """Long-context split-KV decode: 4 sequences of 32K/64K/96K/128K tokens,
     32 q / 8 kv heads, head_dim 128, 64-token blocks, 8192-block pool, bf16,
     N(0, 0.5), 512-token KV partitions."""
-    return decode_batch([32768, 65536, 98304, 131072], 32, 8, 128, 64, 8192, torch.bfloat16,
+    return decode_batch([32768, 65536, 98304, 131072], 32, 8, 128, 64, num_blocks, torch.bfloat16,
                         0.5, seed, max_blocks_per_seq=2048, partition_size=512,
                         name="long_ctx_decode_b4_h32kv8_d128_bs64_p512")
 
 
-def mixed_prefill_decode(seed: int = 0) -> Batch:
+def mixed_prefill_decode(seed: int = 0, num_blocks: int = 16384) -> Batch:
     """8 prefill chunks of 512 query tokens after round(i*4096/7) cached tokens
     (i = 0..7), plus 192 decode sequences in 24 groups of 8 beams sharing a
     1024-token prefix (64 shared blocks) with private tails uniform in
@@ -321,7 +321,7 @@ def mixed_prefill_decode(seed: int = 0) -> Batch:
     tails = torch.randint(64, 513, (192,), generator=gen).tolist()
     ctx = [1024 + t for t in tails]
     groups = [b // 8 for b in range(192)]
-    return mixed_batch(cached, 512, ctx, groups, 1024, 32, 8, 128, 16, 16384, torch.bfloat16,
+    return mixed_batch(cached, 512, ctx, groups, 1024, 32, 8, 128, 16, num_blocks, torch.bfloat16,
                        1.0, seed, name="mixed_prefill8x512_decode192_h32kv8_d128_bs16")
 
 
