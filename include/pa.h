@@ -137,6 +137,31 @@ PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const 
                     int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
                     cudaStream_t stream);
 
+/* pa_decode without a caller-provided workspace. The pages have no
+ * counterpart: this exists for callers that cannot allocate device memory at
+ * the call site (a plugin handed only its input and output buffers, or a
+ * latency-critical caller that may not run cudaMalloc, which can synchronise
+ * the device). Arguments and results are those of pa_decode minus the
+ * workspace; the partial results live in a 16 MiB device array built into
+ * the library, which every GPU that loads the library keeps until exit.
+ *   - A request whose workspace (pa_decode_workspace_size) exceeds 16 MiB is
+ *     refused with PA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the one array: two calls whose kernels overlap on the
+ *     GPU (different streams, no ordering between them) race and may return
+ *     wrong results. Calls ordered on one stream are safe; nothing needs to
+ *     be cleared between them.
+ *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call). */
+PA_API pa_status pa_decode_static_workspace(void *out, const void *q, const void *k_cache,
+                                            const void *v_cache, const int32_t *block_tables,
+                                            const int32_t *context_lens, int num_seqs,
+                                            int num_q_heads, int num_kv_heads, int head_dim,
+                                            int block_size, int num_blocks,
+                                            int max_blocks_per_seq, int max_context_len,
+                                            float scale, int partition_size, pa_dtype dtype,
+                                            cudaStream_t stream);
+
 /* Chunked prefill: chunk c has C_c = query_start_loc[c+1] - query_start_loc[c]
  * queries and context_lens[c] tokens in the cache (its own C_c tokens
  * included, already written by pa_reshape_and_cache). Query i of the chunk

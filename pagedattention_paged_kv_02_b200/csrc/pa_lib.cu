@@ -411,3 +411,61 @@ pa_status pa_selftest_bounded_wait(long long timeout_ns, cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- decode without allocation
+// pa_decode_static_workspace: pa_decode for callers that cannot allocate the
+// workspace themselves -- for example a plugin that is handed only its input
+// and output buffers by a host engine, or a caller on a latency-critical path
+// where cudaMalloc (which may synchronise the whole device) is not allowed.
+// Its scratch is a file-scope device array compiled into the library, so
+// every GPU that loads the library holds these 16 MiB until the process
+// exits. In host code the array's name is only a host-side stand-in; the
+// device address is looked up with cudaGetSymbolAddress the first time the
+// entry point runs on a device (with that device current) and cached.
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = size_t(16) << 20;  // 16 MiB per device
+
+__device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void *g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of g_static_workspace on the current device, looked up once
+// per device; nullptr if the lookup fails.
+void *static_workspace_address() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    if (!g_static_ws_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) return nullptr;
+        g_static_ws_ptr[dev] = p;
+    }
+    return g_static_ws_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_static_workspace(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+    int max_context_len, float scale, int partition_size, pa_dtype dtype, cudaStream_t stream) {
+    // refuse, before touching the device, any request whose partials would
+    // not fit in the fixed array
+    const int P = partition_tokens(max_context_len, partition_size);
+    if (P > 0 && num_seqs >= 0 && num_q_heads > 0 && head_dim > 0 &&
+        workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, P) >
+            kStaticWorkspaceBytes)
+        return PA_ERR_WORKSPACE;
+    void *ws = static_workspace_address();
+    if (!ws) return PA_ERR_CUDA;
+    // the decode kernels write every partial they later read within the same
+    // call, so the array needs no clearing between calls
+    return pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads,
+                     num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                     max_context_len, scale, partition_size, ws, kStaticWorkspaceBytes, dtype,
+                     stream);
+}

@@ -24,7 +24,8 @@ PA_F32, PA_BF16 = 0, 1
 
 EXPORTS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_partition_tokens",
            "pa_decode", "pa_prefill_chunk", "pa_check_tables", "pa_device_error",
-           "pa_selftest_bounded_wait", "pa_status_string", "pa_version")
+           "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
+           "pa_decode_static_workspace")
 
 
 class PAError(RuntimeError):
@@ -51,13 +52,16 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_workspace_size.restype = SZ
         L.pa_decode_partition_tokens.argtypes = [I, I]
         L.pa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, SZ, I, P]
+        L.pa_decode_static_workspace.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I,
+                                                 I, P]
         L.pa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P]
         L.pa_check_tables.argtypes = [P, P, I, I, I, I, P, ctypes.POINTER(I), P]
         L.pa_device_error.argtypes = [ctypes.POINTER(I), I]
         L.pa_selftest_bounded_wait.argtypes = [I64, P]
         L.pa_status_string.argtypes = [I]
         L.pa_status_string.restype = ctypes.c_char_p
-        for f in ("pa_reshape_and_cache", "pa_decode", "pa_prefill_chunk", "pa_check_tables",
+        for f in ("pa_reshape_and_cache", "pa_decode", "pa_decode_static_workspace",
+                  "pa_prefill_chunk", "pa_check_tables",
                   "pa_device_error", "pa_selftest_bounded_wait", "pa_decode_partition_tokens",
                   "pa_version"):
             getattr(L, f).restype = I
@@ -147,6 +151,26 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
     _call("pa_decode", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
           _p(context_lens), B, H_q, H_kv, D, bs, NB, MB, int(max_context_len), float(scale),
           int(partition_size), _p(workspace), ws_bytes, _dt(q), _stream(stream))
+
+
+def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_lens,
+                               max_context_len: int, scale: float, partition_size: int = 0,
+                               stream=None) -> None:
+    """pa_decode using the library's built-in 16 MiB scratch array instead of
+    a workspace, for callers that cannot allocate device memory where they
+    call decode. Calls that overlap on the GPU share that array and race."""
+    _check_int(block_tables, torch.int32, "block_tables")
+    _check_int(context_lens, torch.int32, "context_lens")
+    B, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
+        raise ValueError("out must match q; caches must share head_dim")
+    if not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("q and caches must share one dtype")
+    MB = block_tables.shape[1]
+    _call("pa_decode_static_workspace", _p(out), _p(q), _p(k_cache), _p(v_cache),
+          _p(block_tables), _p(context_lens), B, H_q, H_kv, D, bs, NB, MB, int(max_context_len),
+          float(scale), int(partition_size), _dt(q), _stream(stream))
 
 
 def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
