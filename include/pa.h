@@ -167,11 +167,16 @@ PA_API pa_status pa_decode_static_workspace(void *out, const void *q, const void
  * included, already written by pa_reshape_and_cache). Query i of the chunk
  * sits at position p = context_lens[c] - C_c + i and attends positions 0..p:
  *   out[r][h] = sum_{j<=p} softmax_j(scale * q[r][h] . K_j) V_j,  r = qsl[c]+i.
+ *   num_query_tokens  rows of q and out (query_start_loc[num_chunks]); a
+ *                     chunk reaching past it, or with context_lens[c] < C_c,
+ *                     is skipped and recorded as PA_ERR_BAD_TABLE.
  *   max_query_len     host-side upper bound of every C_c.
- * bf16 only (tensor-core path); fp32 returns PA_ERR_UNSUPPORTED. */
+ * bf16 with head_dim 128 only (the tcgen05 tensor-core path); anything else
+ * returns PA_ERR_UNSUPPORTED. */
 PA_API pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
                            const int32_t *block_tables, const int32_t *context_lens,
-                           const int32_t *query_start_loc, int num_chunks, int max_query_len,
+                           const int32_t *query_start_loc, int num_chunks, int num_query_tokens,
+                           int max_query_len,
                            int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                            int num_blocks, int max_blocks_per_seq, float scale, pa_dtype dtype,
                            cudaStream_t stream);

@@ -307,27 +307,66 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
 
 pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
                            const int32_t *block_tables, const int32_t *context_lens,
-                           const int32_t *query_start_loc, int num_chunks, int max_query_len,
-                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                           int num_blocks, int max_blocks_per_seq, float scale, pa_dtype dtype,
-                           cudaStream_t stream) {
-    if (num_chunks < 0 || max_query_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
-        head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+                           const int32_t *query_start_loc, int num_chunks, int num_query_tokens,
+                           int max_query_len, int num_q_heads, int num_kv_heads, int head_dim,
+                           int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                           pa_dtype dtype, cudaStream_t stream) {
+    if (num_chunks < 0 || num_query_tokens < 0 || max_query_len < 0 || num_q_heads <= 0 ||
+        num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0)
         return PA_ERR_INVALID_ARG;
     if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
     if (dtype != PA_BF16 || num_q_heads % num_kv_heads != 0 || head_dim != 128 ||
         !block_size_ok(block_size))
         return PA_ERR_UNSUPPORTED;
-    if (num_chunks == 0 || max_query_len == 0) return PA_OK;
+    if (num_chunks == 0 || max_query_len == 0 || num_query_tokens == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
         return PA_ERR_INVALID_ARG;
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
         return PA_ERR_INVALID_ARG;
-    return launch_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
-                          num_chunks, max_query_len, num_q_heads, num_kv_heads, head_dim,
-                          block_size, num_blocks, max_blocks_per_seq, scale, stream);
+    const long long qtiles = (max_query_len + kPfRows - 1) / kPfRows;
+    if (num_q_heads > 65535 || num_chunks > 65535 || qtiles > 0x7fffffffLL)
+        return PA_ERR_UNSUPPORTED;
+
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return PA_ERR_CUDA;
+    CUtensorMap mq, mk, mv;
+    {
+        cuuint64_t dims[3] = {128, (cuuint64_t)num_q_heads, (cuuint64_t)num_query_tokens};
+        cuuint64_t strides[2] = {128 * 2, (cuuint64_t)num_q_heads * 128 * 2};
+        cuuint32_t box[3] = {64, 1, kPfRows};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return PA_ERR_CUDA;
+    }
+    if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, block_size, 128, 16) ||
+        !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, block_size, 128, 16))
+        return PA_ERR_CUDA;
+
+    PrefillArgs a;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.qsl = query_start_loc;
+    a.n_chunks = num_chunks;
+    a.total_q = num_query_tokens;
+    a.H_q = num_q_heads;
+    a.H_kv = num_kv_heads;
+    a.group = num_q_heads / num_kv_heads;
+    a.bs = block_size;
+    a.NB = num_blocks;
+    a.MB = max_blocks_per_seq;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.timeout_ns = kWaitTimeoutNs;
+    const size_t smem = 1024 + kPfSmem;
+    if (set_smem(prefill_tc_kernel, smem) != cudaSuccess) return PA_ERR_CUDA;
+    const dim3 grid((unsigned)qtiles, (unsigned)num_q_heads, (unsigned)num_chunks);
+    prefill_tc_kernel<<<grid, kPfThreads, smem, stream>>>(a, mq, mk, mv);
+    return launch_status();
 }
 
 }  // extern "C"

@@ -1,14 +1,445 @@
-// prefill.cuh -- chunked prefill over the paged cache (tensor-core kernel).
+// prefill.cuh -- chunked prefill over the paged cache on 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// What is computed (page "vLLM框架是怎么做推理加速的", section 3, Chunked
+// Prefill): a chunk of C prompt tokens, whose K/V are already appended to the
+// cache, attends over everything cached before it plus itself, causally
+// (page "LLM推理优化", section 2.3, causal=True): query i of the chunk sits at
+// position cached + i and sees keys 0..cached+i. K/V pages are reached through
+// the chunk's block table (page "字节跳动 AI Infra (2)", question
+// "vLLM与PagedAttention的原理"), and the softmax is computed tile by tile with
+// a running max and sum (page "LLM推理优化", section 2.1).
+//
+// One CTA = 128 query rows of one query head of one chunk (the tcgen05 M
+// tile); keys are processed in tiles of 128. Six warps:
+//   warp 4 (one lane)  TMA: the Q tile once, then each key tile's K and V as
+//                      16-token page pieces (128-byte swizzle) gathered
+//                      through the block table; K and V each single-buffered
+//                      with their own full/free barriers, so K(j+1) streams in
+//                      while tile j's softmax and P.V run.
+//   warp 5 (one lane)  MMA: S = Q K^T (8 x 128x128x16, both operands K-major
+//                      in shared memory) into tensor memory columns [0,128);
+//                      then O += P V with P read from tensor memory and V
+//                      MN-major in shared memory, into columns [128,256).
+//   warps 0-3          softmax: thread r owns row r (tensor-memory lane r):
+//                      row max, exp2, the running sum, bf16 P written back
+//                      over the consumed S columns; O is rescaled in tensor
+//                      memory only when a row's max grows by more than 2^8
+//                      (the result is exact for any reference max as long as
+//                      O and the sum share it); the epilogue divides by the
+//                      sum and writes bf16 rows.
+// All waits are bounded; a wait that runs out records PA_ERR_TIMEOUT, makes
+// every role leave its loop, drains outstanding copies and tensor-core work,
+// and frees the tensor memory.
 #pragma once
 
 #include "pa_device.cuh"
 
 namespace pa {
 
-inline pa_status launch_prefill(void *, const void *, const void *, const void *, const int32_t *,
-                                const int32_t *, const int32_t *, int, int, int, int, int, int,
-                                int, int, float, cudaStream_t) {
-    return PA_ERR_UNSUPPORTED;
+constexpr int kPfRows = 128;      // query rows per CTA
+constexpr int kPfKeys = 128;      // keys per tile
+constexpr int kPfThreads = 192;   // 4 softmax warps + TMA warp + MMA warp
+constexpr int kPfTileBytes = kPfRows * 128 * 2;  // 128 x 128 bf16 = 32 KB
+constexpr int kPfSmem = 3 * kPfTileBytes + 256;  // Q, K, V, barriers
+
+struct PrefillArgs {
+    __nv_bfloat16 *out;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    const int32_t *qsl;
+    int n_chunks, total_q, H_q, H_kv, group, bs, NB, MB;
+    float scale_log2;
+    unsigned long long timeout_ns;
+};
+
+// ------------------------------------------------------------ tcgen05 PTX
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive on `bar` once every tcgen05 operation this thread issued so far has
+// completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+// D(tmem) (+)= A(smem desc) * B(smem desc)
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc)
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+#define PA_R32(r)                                                                                 \
+    "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),         \
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), \
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),           \
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),           \
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives
+// its lane's 32 columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : PA_R32(r)
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm100 format: start,
+// leading and stride byte offsets in 16-byte units, version 1 at bit 46,
+// layout type 2 = SWIZZLE_128B at bits 61-63).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator (bit 4), bf16 A and B
+// (bits 7, 10), B MN-major when b_mn (bit 16), N>>3 at bit 17, M>>4 at bit 24.
+__host__ __device__ constexpr uint32_t f16_idesc(int M, int N, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+struct PfBars {
+    uint64_t q_full, k_full, k_free, v_full, v_free, s_full, p_full, o_full, fin;
+    uint32_t tmem_base;
+    volatile int abort;
+};
+
+// Bounded wait shared by all roles: false when the CTA is aborting or the
+// bound ran out (which starts the abort). Warp-uniform when `uniform`.
+__device__ __forceinline__ bool pf_wait(PfBars *bars, uint64_t *bar, uint32_t parity,
+                                        unsigned long long timeout_ns, bool uniform) {
+    bool ok = bars->abort == 0 && mbar_wait(smem_u32(bar), parity, timeout_ns);
+    if (uniform) ok = __all_sync(0xffffffffu, ok);
+    if (!ok && bars->abort == 0) {
+        bars->abort = 1;
+        flag_error(PA_ERR_TIMEOUT);
+    }
+    return ok;
+}
+
+__global__ void __launch_bounds__(kPfThreads, 2)
+    prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
+                      const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sQ = smem_u32(smem);
+    const uint32_t sK = sQ + kPfTileBytes;
+    const uint32_t sV = sK + kPfTileBytes;
+    PfBars *bars = reinterpret_cast<PfBars *>(smem + 3 * kPfTileBytes);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qt = blockIdx.x, h = blockIdx.y;
+    const int c = a.n_chunks - 1 - (int)blockIdx.z;  // later (longer) chunks first
+    const int q0 = a.qsl[c];
+    const int C = a.qsl[c + 1] - q0;
+    if (qt * kPfRows >= C) return;
+    const int ctx = a.context_lens[c];
+    if (q0 < 0 || C < 0 || q0 + C > a.total_q || ctx < C || (long long)ctx > (long long)a.MB * a.bs) {
+        if (threadIdx.x == 0) flag_error(PA_ERR_BAD_TABLE);
+        return;
+    }
+    const int cached = ctx - C;
+    const int rows = min(kPfRows, C - qt * kPfRows);
+    const int p_max = cached + qt * kPfRows + rows - 1;  // last key any row needs
+    const int n_tiles = p_max / kPfKeys + 1;
+    const int kvh = h / a.group;
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars->q_full), 1);
+        mbar_init(smem_u32(&bars->k_full), 1);
+        mbar_init(smem_u32(&bars->k_free), 1);
+        mbar_init(smem_u32(&bars->v_full), 1);
+        mbar_init(smem_u32(&bars->v_free), 1);
+        mbar_init(smem_u32(&bars->s_full), 1);
+        mbar_init(smem_u32(&bars->p_full), 128);
+        mbar_init(smem_u32(&bars->o_full), 1);
+        mbar_init(smem_u32(&bars->fin), 1);
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(&bars->tmem_base), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tS = bars->tmem_base;  // columns [0,128): S; P (bf16 pairs) over [0,64)
+    const uint32_t tO = tS + 128;         // columns [128,256): O
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA
+        if (lane == 0) {
+            const int n_blk = (ctx + a.bs - 1) / a.bs;
+            const int32_t *row = a.block_tables + (size_t)c * a.MB;
+            auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j) {
+                int ids[8];
+                int n = 0;
+#pragma unroll
+                for (int s16 = 0; s16 < 8; ++s16) {
+                    const int key = j * kPfKeys + s16 * 16;
+                    int id = -1;
+                    if (key < ctx) {
+                        const int lb = key / a.bs;
+                        id = lb < n_blk ? __ldg(row + lb) : -1;
+                        if (id < 0 || id >= a.NB) {
+                            flag_error(PA_ERR_BAD_TABLE);
+                            id = -1;
+                        }
+                    }
+                    ids[s16] = id;
+                    n += id >= 0;
+                }
+                mbar_arrive_expect_tx(smem_u32(bar), n * 2 * 2048);
+#pragma unroll
+                for (int s16 = 0; s16 < 8; ++s16) {
+                    if (ids[s16] < 0) continue;
+                    const int off = (j * kPfKeys + s16 * 16) % a.bs;
+                    tma_load_4d(dst + s16 * 2048, map, smem_u32(bar), 0, off, kvh, ids[s16]);
+                    tma_load_4d(dst + 16384 + s16 * 2048, map, smem_u32(bar), 64, off, kvh,
+                                ids[s16]);
+                }
+            };
+            mbar_arrive_expect_tx(smem_u32(&bars->q_full), kPfTileBytes);
+            tma_load_3d(sQ, &tmq, smem_u32(&bars->q_full), 0, h, q0 + qt * kPfRows);
+            tma_load_3d(sQ + 16384, &tmq, smem_u32(&bars->q_full), 64, h, q0 + qt * kPfRows);
+            int k_issued = 0, v_issued = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                if (j > 0 && !pf_wait(bars, &bars->k_free, (j - 1) & 1, a.timeout_ns, false)) break;
+                issue(sK, &tmk, &bars->k_full, j);
+                k_issued = j + 1;
+                if (j > 0 && !pf_wait(bars, &bars->v_free, (j - 1) & 1, a.timeout_ns, false)) break;
+                issue(sV, &tmv, &bars->v_full, j);
+                v_issued = j + 1;
+            }
+            if (bars->abort) {  // let copies already in flight land
+                mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
+                if (k_issued) mbar_wait(smem_u32(&bars->k_full), (k_issued - 1) & 1, a.timeout_ns);
+                if (v_issued) mbar_wait(smem_u32(&bars->v_full), (v_issued - 1) & 1, a.timeout_ns);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0) {
+            constexpr uint32_t kIdQK = f16_idesc(128, 128, false);
+            constexpr uint32_t kIdPV = f16_idesc(128, 128, true);
+            bool ok = pf_wait(bars, &bars->q_full, 0, a.timeout_ns, false);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                if (!pf_wait(bars, &bars->k_full, j & 1, a.timeout_ns, false)) break;
+                if (j > 0 && !pf_wait(bars, &bars->o_full, (j - 1) & 1, a.timeout_ns, false)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    mma_ss(tS, sw128_desc(sQ + koff, 16, 1024), sw128_desc(sK + koff, 16, 1024),
+                           kIdQK, ks > 0);
+                }
+                tc_commit(smem_u32(&bars->s_full));
+                tc_commit(smem_u32(&bars->k_free));
+                if (!pf_wait(bars, &bars->p_full, j & 1, a.timeout_ns, false)) break;
+                if (!pf_wait(bars, &bars->v_full, j & 1, a.timeout_ns, false)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    mma_ts(tO, tS + ks * 8, sw128_desc(sV + ks * 2048, 16384, 1024), kIdPV,
+                           (j > 0 || ks > 0) ? 1u : 0u);
+                }
+                tc_commit(smem_u32(&bars->o_full));
+                tc_commit(smem_u32(&bars->v_free));
+            }
+            // every tensor-core operation issued above completes before teardown
+            tc_commit(smem_u32(&bars->fin));
+            mbar_wait(smem_u32(&bars->fin), 0, a.timeout_ns);
+        }
+    } else {
+        // -------------------------------------------------------- softmax
+        const int r = threadIdx.x;  // row of the tile == tensor-memory lane
+        const int i = qt * kPfRows + r;
+        const bool row_valid = i < C;
+        const int pos = cached + min(i, C - 1);  // keys <= pos are visible
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sl2 = a.scale_log2;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            if (!pf_wait(bars, &bars->s_full, j & 1, a.timeout_ns, true)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const int key0 = j * kPfKeys;
+            float mt = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tS + lane_off + cc * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int key = key0 + cc * 32 + e;
+                    if (key <= pos) mt = fmaxf(mt, __uint_as_float(v[e]) * sl2);
+                }
+            }
+            const float m_new = fmaxf(m, mt);
+            if (j == 0) {
+                m = m_new;
+            } else if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
+                // re-reference O and the sum to the new max (warp-uniform)
+                const float corr = exp2f(m - m_new);
+                l *= corr;
+                m = m_new;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t v[32];
+                    tmem_ld32(tO + lane_off + cc * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
+                    tmem_st32(tO + lane_off + cc * 32, v);
+                }
+            }
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tS + lane_off + cc * 32, v);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int k0 = key0 + cc * 32 + 2 * e;
+                    const float p0 = k0 <= pos ? exp2f(__uint_as_float(v[2 * e]) * sl2 - m) : 0.f;
+                    const float p1 =
+                        k0 + 1 <= pos ? exp2f(__uint_as_float(v[2 * e + 1]) * sl2 - m) : 0.f;
+                    pk[e] = pack_bf16x2(p0, p1);
+                    l += bf16_lo(pk[e]) + bf16_hi(pk[e]);  // the weights P.V uses
+                }
+                // P for these 32 keys goes to columns [16cc, 16cc+16), whose
+                // S values were consumed earlier in this loop
+                tmem_st16(tS + lane_off + cc * 16, pk);
+            }
+            tmem_st_wait();
+            if (j == n_tiles - 1 && key0 + kPfKeys > ctx) {
+                // V rows past the context hold stale or unloaded data: zero
+                // them so that P = 0 cannot meet a NaN there
+                if (!pf_wait(bars, &bars->v_full, j & 1, a.timeout_ns, true)) {
+                    ok = false;
+                    break;
+                }
+                const int vr = ctx - key0;
+                for (int e = r; e < (kPfKeys - vr) * 16; e += 128) {
+                    const int row = vr + e / 16, u = e % 16;
+                    const uint32_t addr = sV + (u / 8) * 16384 + row * 128 + (u % 8) * 16;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->p_full));
+        }
+        if (ok && pf_wait(bars, &bars->o_full, (n_tiles - 1) & 1, a.timeout_ns, true)) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + h) * 128;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tO + lane_off + cc * 32, v);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
+                                        __uint_as_float(v[2 * e + 1]) * inv);
+                if (row_valid) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tS, 256);
+    }
 }
 
 }  // namespace pa

@@ -54,7 +54,7 @@ def lib() -> ctypes.CDLL:
         L.pa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, SZ, I, P]
         L.pa_decode_static_workspace.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I,
                                                  I, P]
-        L.pa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P]
+        L.pa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P]
         L.pa_check_tables.argtypes = [P, P, I, I, I, I, P, ctypes.POINTER(I), P]
         L.pa_device_error.argtypes = [ctypes.POINTER(I), I]
         L.pa_selftest_bounded_wait.argtypes = [I64, P]
@@ -186,8 +186,8 @@ def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query
     n_chunks = query_start_loc.numel() - 1
     MB = block_tables.shape[1]
     _call("pa_prefill_chunk", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
-          _p(context_lens), _p(query_start_loc), n_chunks, int(max_query_len), H_q, H_kv, D, bs,
-          NB, MB, float(scale), _dt(q), _stream(stream))
+          _p(context_lens), _p(query_start_loc), n_chunks, total_q, int(max_query_len), H_q,
+          H_kv, D, bs, NB, MB, float(scale), _dt(q), _stream(stream))
 
 
 def pa_check_tables(block_tables, context_lens, block_size: int, num_blocks: int,

@@ -124,14 +124,20 @@ def test_reshape_host_checks(L):
 def test_prefill_host_checks(L):
     from pagedattention_paged_kv_02_b200 import pa
     f = L.pa_prefill_chunk
-    base = [FAKE] * 7 + [2, 512, 32, 8, 128, 16, 64, 64, 0.1, 1, None]
-    assert f(*base[:16], 0, None) == pa.PA_ERR_UNSUPPORTED  # fp32 has no tensor-core path
+    # out, q, k, v, tables, lens, qsl, chunks, tokens, max_q, Hq, Hkv, D, bs, NB, MB, scale,
+    # dtype, stream
+    base = [FAKE] * 7 + [2, 1024, 512, 32, 8, 128, 16, 64, 64, 0.1, 1, None]
+    assert len(base) == 19
+    assert f(*base[:17], 0, None) == pa.PA_ERR_UNSUPPORTED  # fp32 has no tensor-core path
     b = list(base)
-    b[11] = 64
+    b[12] = 64
     assert f(*b) == pa.PA_ERR_UNSUPPORTED
     b = list(base)
-    b[9], b[10] = 12, 8
+    b[10], b[11] = 12, 8
     assert f(*b) == pa.PA_ERR_UNSUPPORTED
+    b = list(base)
+    b[8] = -1
+    assert f(*b) == pa.PA_ERR_INVALID_ARG
     b = list(base)
     b[1] = None
     assert f(*b) == pa.PA_ERR_INVALID_ARG

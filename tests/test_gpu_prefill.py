@@ -1,0 +1,121 @@
+"""GPU parity of chunked prefill (tcgen05 tensor-core kernel) against the fp64
+oracle, through the C ABI: ragged chunks that start mid-tile, span several
+128-key tiles, end in partial blocks and partial tiles, with every block size
+and head grouping; chunk length 1 against decode; and the mixed workload
+(8 x 512-token chunks after 0..4096 cached tokens plus 192 shared-prefix
+decode sequences) at full size, sampled rows for prefill and every output for
+decode."""
+import pytest
+import torch
+
+import oracle
+from helpers import assert_close, bits, gpu_decode, oracle_after_append
+from pagedattention_paged_kv_02_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from pagedattention_paged_kv_02_b200 import build, pa as _pa
+    build.build()
+    torch.cuda.init()
+    return _pa
+
+
+@pytest.fixture(autouse=True)
+def clean_error_word(pa):
+    pa.pa_device_error(clear=True)
+    yield
+    torch.cuda.synchronize()
+
+
+def run_prefill(pa, batch):
+    d = batch.to(DEV)
+    pa.pa_reshape_and_cache(d.key, d.value, d.k_cache, d.v_cache, d.slot_mapping)
+    out = torch.full_like(d.prefill_q, float("nan"))
+    qsl = batch.query_start_loc
+    max_q = int((qsl[1:] - qsl[:-1]).max())
+    pa.pa_prefill_chunk(out, d.prefill_q, d.k_cache, d.v_cache, d.prefill_block_tables,
+                        d.prefill_context_lens, d.query_start_loc, max_q, batch.scale)
+    torch.cuda.synchronize()
+    return d, out
+
+
+def oracle_prefill(batch, k, v, select=None):
+    return oracle.prefill(batch.prefill_q, k, v, batch.prefill_block_tables,
+                          batch.prefill_context_lens, batch.query_start_loc, batch.scale,
+                          select=select)
+
+
+CASES = [
+    # (cached per chunk, chunk lengths), H_q, H_kv, bs
+    (([0, 0, 100, 37], [5, 128, 129, 300]), 8, 2, 16),
+    (([1000, 300, 0], [64, 1, 257]), 4, 4, 32),
+    (([250, 700], [200, 77]), 8, 1, 64),
+    (([16, 127, 128], [16, 1, 129]), 32, 8, 16),
+]
+
+
+def mixed_chunks(cached, lens, Hq, Hkv, bs, seed):
+    """Chunks of differing lengths: built one length at a time, then merged."""
+    nb = sum(-(-(c + n) // bs) for c, n in zip(cached, lens)) + 8
+    gen = torch.Generator().manual_seed(seed)
+    from pagedattention_paged_kv_02_b200.workloads import SeqSpec, build_pool, Batch, _randn
+    specs = [SeqSpec(c + n, n) for c, n in zip(cached, lens)]
+    k, v, tables, key, value, slots, poison = build_pool(specs, Hkv, 128, bs, nb,
+                                                         torch.bfloat16, 1.0, gen)
+    qsl = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32)
+    q = _randn(gen, (int(qsl[-1]), Hq, 128), 1.0, torch.bfloat16)
+    return Batch(name="chunks", k_cache=k, v_cache=v, key=key, value=value, slot_mapping=slots,
+                 scale=128 ** -0.5, block_size=bs, poison_block=poison, prefill_q=q,
+                 prefill_block_tables=tables,
+                 prefill_context_lens=torch.tensor([s.ctx for s in specs], dtype=torch.int32),
+                 query_start_loc=qsl)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"h{c[1]}kv{c[2]}-bs{c[3]}-{max(c[0][1])}q")
+def test_prefill_small(pa, case):
+    (cached, lens), Hq, Hkv, bs = case
+    batch = mixed_chunks(cached, lens, Hq, Hkv, bs, seed=sum(lens) + Hq)
+    d, out = run_prefill(pa, batch)
+    k, v = oracle_after_append(batch)
+    ref, _ = oracle_prefill(batch, k, v)
+    assert_close(out, ref, f"prefill {case}")
+    assert pa.pa_device_error() == 0
+
+
+def test_prefill_single_query_equals_decode(pa):
+    """A chunk of one query is a decode step over the same context."""
+    batch = mixed_chunks([500, 2000, 31], [1, 1, 1], 8, 2, 16, seed=77)
+    d, out = run_prefill(pa, batch)
+    dec = torch.empty_like(d.prefill_q)
+    pa.pa_decode(dec, d.prefill_q, d.k_cache, d.v_cache, d.prefill_block_tables,
+                 d.prefill_context_lens, int(batch.prefill_context_lens.max()), batch.scale,
+                 -1)  # one partition per sequence: no workspace needed
+    torch.cuda.synchronize()
+    assert_close(out, dec.double().cpu(), "prefill C=1 vs decode")
+
+
+def test_mixed_workload_full(pa):
+    """The mixed prefill + shared-prefix decode step at full size."""
+    batch = W.mixed_prefill_decode()
+    d, out = run_prefill(pa, batch)
+    k, v = oracle_after_append(batch)
+    assert torch.equal(bits(d.k_cache.cpu()), bits(k)), "cache scatter not bit-exact"
+    assert torch.equal(bits(d.v_cache.cpu()), bits(v)), "cache scatter not bit-exact"
+    # prefill: every 13th query row (all heads), covering every chunk and tile
+    rows = torch.zeros(out.shape[0], dtype=torch.bool)
+    rows[::13] = True
+    rows[511::512] = True  # last row of every chunk
+    sel = rows[:, None].expand(-1, batch.num_q_heads)
+    ref, _ = oracle_prefill(batch, k, v, select=sel)
+    assert_close(out[rows], ref[rows], "mixed prefill")
+    # decode part, every output
+    dec = gpu_decode(pa, d)
+    torch.cuda.synchronize()
+    dref, _ = oracle.decode(batch.q, k, v, batch.block_tables, batch.context_lens, batch.scale)
+    assert_close(dec, dref, "mixed decode")
+    assert pa.pa_device_error() == 0
