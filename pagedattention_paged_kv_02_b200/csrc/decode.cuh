@@ -60,10 +60,15 @@ __device__ __forceinline__ int clamped_ctx(const DecodeArgs &a, int b, bool repo
     return ctx;
 }
 
-template <int NW, int NS, int STAGE_BYTES>
+// Shared-memory plan of a split CTA: the stage ring (reused after the main
+// loop for the cross-warp merge, so it is sized for whichever is larger),
+// then NW*NS mbarriers, then the partition's block-table slice.
+template <int NW, int NS, int STAGE_BYTES, int HT, int D>
 struct DecodeSmem {
-    static constexpr int kStages = NW * NS * STAGE_BYTES;
-    static constexpr int kBars = kStages;  // NW*NS mbarriers (8 B each)
+    static constexpr int kRing = NW * NS * STAGE_BYTES;
+    static constexpr int kMerge = NW * HT * (D + 4) * 4 + 2 * NW * HT * 4;
+    static constexpr int kStages = ((kRing > kMerge ? kRing : kMerge) + 1023) / 1024 * 1024;
+    static constexpr int kBars = kStages;
     static constexpr int kTable = kBars + NW * NS * 8;
 };
 
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(NW * 32)
     constexpr int HALF = kChunk * D * 2;    // bytes of one K (or V) chunk
     constexpr int STAGE = 2 * HALF;
     constexpr int SUBTILE = kChunk * 128;   // one 64-wide swizzled sub-tile
-    using L = DecodeSmem<NW, NS, STAGE>;
+    using L = DecodeSmem<NW, NS, STAGE, HT, D>;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -362,7 +367,7 @@ __global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constan
     constexpr int VEC = D / 32;          // dims per lane
     constexpr int HALF = kChunk * D * 4;
     constexpr int STAGE = 2 * HALF;
-    using L = DecodeSmem<NW, NS, STAGE>;
+    using L = DecodeSmem<NW, NS, STAGE, HT, D>;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &

@@ -106,7 +106,7 @@ struct Pipe {
 
 Pipe decode_pipe() {
     static Pipe p = [] {
-        Pipe r{4, 3};
+        Pipe r{4, 2};
         if (const char *e = std::getenv("PA_DECODE_PIPE")) {
             int w = 0, s = 0;
             if (sscanf(e, "%dx%d", &w, &s) == 2) r = Pipe{w, s};
@@ -120,7 +120,7 @@ template <int D, int NW, int NS>
 pa_status launch_decode_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
                              dim3 grid, cudaStream_t st) {
     constexpr int STAGE = 2 * kChunk * D * 2;
-    using L = DecodeSmem<NW, NS, STAGE>;
+    using L = DecodeSmem<NW, NS, STAGE, kHeadsBf16, D>;
     const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
     auto k = decode_split_bf16<D, NW, NS>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
@@ -131,7 +131,7 @@ pa_status launch_decode_bf16(const DecodeArgs &a, const CUtensorMap &mk, const C
 template <int D, int NW, int NS>
 pa_status launch_decode_f32(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
     constexpr int STAGE = 2 * kChunk * D * 4;
-    using L = DecodeSmem<NW, NS, STAGE>;
+    using L = DecodeSmem<NW, NS, STAGE, kHeadsF32, D>;
     const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
     auto k = decode_split_f32<D, NW, NS>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
@@ -143,10 +143,12 @@ template <int D>
 pa_status dispatch_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
                         dim3 grid, cudaStream_t st) {
     const Pipe p = decode_pipe();
-    if (p.nw == 4 && p.ns == 2) return launch_decode_bf16<D, 4, 2>(a, mk, mv, grid, st);
-    if (p.nw == 4 && p.ns == 4) return launch_decode_bf16<D, 4, 4>(a, mk, mv, grid, st);
-    if (p.nw == 8 && p.ns == 2) return launch_decode_bf16<D, 8, 2>(a, mk, mv, grid, st);
-    return launch_decode_bf16<D, 4, 3>(a, mk, mv, grid, st);
+    if (p.nw == 2 && p.ns == 2) return launch_decode_bf16<D, 2, 2>(a, mk, mv, grid, st);
+    if (p.nw == 2 && p.ns == 3) return launch_decode_bf16<D, 2, 3>(a, mk, mv, grid, st);
+    if (p.nw == 2 && p.ns == 4) return launch_decode_bf16<D, 2, 4>(a, mk, mv, grid, st);
+    if (p.nw == 4 && p.ns == 1) return launch_decode_bf16<D, 4, 1>(a, mk, mv, grid, st);
+    if (p.nw == 4 && p.ns == 3) return launch_decode_bf16<D, 4, 3>(a, mk, mv, grid, st);
+    return launch_decode_bf16<D, 4, 2>(a, mk, mv, grid, st);
 }
 
 }  // namespace
@@ -326,7 +328,7 @@ pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const 
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
         return PA_ERR_INVALID_ARG;
-    const long long qtiles = (max_query_len + kPfRows - 1) / kPfRows;
+    const long long qtiles = (max_query_len + kPfRows * kPfQTiles - 1) / (kPfRows * kPfQTiles);
     if (num_q_heads > 65535 || num_chunks > 65535 || qtiles > 0x7fffffffLL)
         return PA_ERR_UNSUPPORTED;
 
@@ -364,6 +366,13 @@ pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const 
     a.timeout_ns = kWaitTimeoutNs;
     const size_t smem = 1024 + kPfSmem;
     if (set_smem(prefill_tc_kernel, smem) != cudaSuccess) return PA_ERR_CUDA;
+    {
+        // the kernel's register split must fit the registers it launches
+        // with, or the warpgroups that grow would wait forever
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, prefill_tc_kernel) != cudaSuccess) return PA_ERR_CUDA;
+        if ((long long)fa.numRegs * kPfThreads < kPfRegsNeeded) return PA_ERR_UNSUPPORTED;
+    }
     const dim3 grid((unsigned)qtiles, (unsigned)num_q_heads, (unsigned)num_chunks);
     prefill_tc_kernel<<<grid, kPfThreads, smem, stream>>>(a, mq, mk, mv);
     return launch_status();

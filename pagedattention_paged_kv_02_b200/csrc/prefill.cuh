@@ -37,11 +37,21 @@
 
 namespace pa {
 
-constexpr int kPfRows = 128;      // query rows per CTA
-constexpr int kPfKeys = 128;      // keys per tile
-constexpr int kPfThreads = 192;   // 4 softmax warps + TMA warp + MMA warp
+constexpr int kPfRows = 128;      // query rows per Q tile (the tcgen05 M)
+constexpr int kPfQTiles = 2;      // Q tiles per CTA, sharing every K/V tile
+constexpr int kPfKeys = 128;      // keys per K/V tile
+constexpr int kPfStages = 2;      // K and V ring depth
+constexpr int kPfThreads = 384;   // 2 softmax warpgroups + a control warpgroup
+// Register split (setmaxnreg): the control warpgroup (TMA warp, MMA warp and
+// two idle warps) gives registers to the two softmax warpgroups, which hold
+// a full 128-column score row per thread. The shares must sum to at most the
+// launch allocation (384 threads x registers per thread); the host checks
+// that against the compiled kernel before launching.
+constexpr int kPfCtlRegs = 56;
+constexpr int kPfSoftmaxRegs = 224;
+constexpr int kPfRegsNeeded = 128 * (2 * kPfSoftmaxRegs + kPfCtlRegs);
 constexpr int kPfTileBytes = kPfRows * 128 * 2;  // 128 x 128 bf16 = 32 KB
-constexpr int kPfSmem = 3 * kPfTileBytes + 256;  // Q, K, V, barriers
+constexpr int kPfSmem = (kPfQTiles + 2 * kPfStages) * kPfTileBytes + 512;
 
 struct PrefillArgs {
     __nv_bfloat16 *out;
@@ -168,7 +178,10 @@ __host__ __device__ constexpr uint32_t f16_idesc(int M, int N, bool b_mn) {
 }
 
 struct PfBars {
-    uint64_t q_full, k_full, k_free, v_full, v_free, s_full, p_full, o_full, fin;
+    uint64_t q_full;
+    uint64_t k_full[kPfStages], k_free[kPfStages], v_full[kPfStages], v_free[kPfStages];
+    uint64_t s_full[kPfQTiles], p_full[kPfQTiles], o_full[kPfQTiles];
+    uint64_t fin;
     uint32_t tmem_base;
     volatile int abort;
 };
@@ -186,63 +199,81 @@ __device__ __forceinline__ bool pf_wait(PfBars *bars, uint64_t *bar, uint32_t pa
     return ok;
 }
 
-__global__ void __launch_bounds__(kPfThreads, 2)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    const uint32_t sQ = smem_u32(smem);
-    const uint32_t sK = sQ + kPfTileBytes;
-    const uint32_t sV = sK + kPfTileBytes;
-    PfBars *bars = reinterpret_cast<PfBars *>(smem + 3 * kPfTileBytes);
+    const uint32_t sQ = smem_u32(smem);                         // Q tile x at sQ + x*32K
+    const uint32_t sK = sQ + kPfQTiles * kPfTileBytes;          // K stage st at sK + st*32K
+    const uint32_t sV = sK + kPfStages * kPfTileBytes;          // V stage st at sV + st*32K
+    PfBars *bars = reinterpret_cast<PfBars *>(smem + (kPfQTiles + 2 * kPfStages) * kPfTileBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, h = blockIdx.y;
+    const int tp = blockIdx.x, h = blockIdx.y;
     const int c = a.n_chunks - 1 - (int)blockIdx.z;  // later (longer) chunks first
     const int q0 = a.qsl[c];
     const int C = a.qsl[c + 1] - q0;
-    if (qt * kPfRows >= C) return;
+    const int row0 = tp * kPfRows * kPfQTiles;  // first query of this CTA within the chunk
+    if (row0 >= C) return;
     const int ctx = a.context_lens[c];
     if (q0 < 0 || C < 0 || q0 + C > a.total_q || ctx < C || (long long)ctx > (long long)a.MB * a.bs) {
         if (threadIdx.x == 0) flag_error(PA_ERR_BAD_TABLE);
         return;
     }
     const int cached = ctx - C;
-    const int rows = min(kPfRows, C - qt * kPfRows);
-    const int p_max = cached + qt * kPfRows + rows - 1;  // last key any row needs
-    const int n_tiles = p_max / kPfKeys + 1;
+    // rows and K/V tiles of each Q tile (a Q tile past the chunk has none)
+    const int rows0 = min(kPfRows, C - row0);
+    const int rows1 = max(0, min(kPfRows, C - row0 - kPfRows));
+    const int ntile0 = (cached + row0 + rows0 - 1) / kPfKeys + 1;
+    const int ntile1 = rows1 > 0 ? (cached + row0 + kPfRows + rows1 - 1) / kPfKeys + 1 : 0;
+    auto ntile = [&](int x) { return x == 0 ? ntile0 : ntile1; };
+    const int n_kv = max(ntile0, ntile1);
     const int kvh = h / a.group;
 
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
-        mbar_init(smem_u32(&bars->k_full), 1);
-        mbar_init(smem_u32(&bars->k_free), 1);
-        mbar_init(smem_u32(&bars->v_full), 1);
-        mbar_init(smem_u32(&bars->v_free), 1);
-        mbar_init(smem_u32(&bars->s_full), 1);
-        mbar_init(smem_u32(&bars->p_full), 128);
-        mbar_init(smem_u32(&bars->o_full), 1);
+        for (int st = 0; st < kPfStages; ++st) {
+            mbar_init(smem_u32(&bars->k_full[st]), 1);
+            mbar_init(smem_u32(&bars->k_free[st]), 1);
+            mbar_init(smem_u32(&bars->v_full[st]), 1);
+            mbar_init(smem_u32(&bars->v_free[st]), 1);
+        }
+        for (int x = 0; x < kPfQTiles; ++x) {
+            mbar_init(smem_u32(&bars->s_full[x]), 1);
+            mbar_init(smem_u32(&bars->p_full[x]), 128);
+            mbar_init(smem_u32(&bars->o_full[x]), 1);
+        }
         mbar_init(smem_u32(&bars->fin), 1);
         bars->abort = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
-        tmem_alloc(smem_u32(&bars->tmem_base), 256);
+    if (warp == 9) {
+        tmem_alloc(smem_u32(&bars->tmem_base), 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tS = bars->tmem_base;  // columns [0,128): S; P (bf16 pairs) over [0,64)
-    const uint32_t tO = tS + 128;         // columns [128,256): O
+    // tensor memory: S/P of Q tile x in columns [128x, 128x+128) (P, bf16
+    // pairs, over the first 64); O of Q tile x in [256+128x, 256+128x+128)
+    const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 4) {
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfCtlRegs));
+      if (warp == 8) {
         // ------------------------------------------------------------ TMA
         if (lane == 0) {
             const int n_blk = (ctx + a.bs - 1) / a.bs;
-            const int32_t *row = a.block_tables + (size_t)c * a.MB;
+            const int32_t *trow = a.block_tables + (size_t)c * a.MB;
             auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j) {
                 int ids[8];
                 int n = 0;
@@ -252,7 +283,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
                     int id = -1;
                     if (key < ctx) {
                         const int lb = key / a.bs;
-                        id = lb < n_blk ? __ldg(row + lb) : -1;
+                        id = lb < n_blk ? __ldg(trow + lb) : -1;
                         if (id < 0 || id >= a.NB) {
                             flag_error(PA_ERR_BAD_TABLE);
                             id = -1;
@@ -271,163 +302,226 @@ __global__ void __launch_bounds__(kPfThreads, 2)
                                 ids[s16]);
                 }
             };
-            mbar_arrive_expect_tx(smem_u32(&bars->q_full), kPfTileBytes);
-            tma_load_3d(sQ, &tmq, smem_u32(&bars->q_full), 0, h, q0 + qt * kPfRows);
-            tma_load_3d(sQ + 16384, &tmq, smem_u32(&bars->q_full), 64, h, q0 + qt * kPfRows);
+            const int nq = rows1 > 0 ? 2 : 1;
+            mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * kPfTileBytes);
+            for (int x = 0; x < nq; ++x) {
+                const int r0 = q0 + row0 + x * kPfRows;
+                tma_load_3d(sQ + x * kPfTileBytes, &tmq, smem_u32(&bars->q_full), 0, h, r0);
+                tma_load_3d(sQ + x * kPfTileBytes + 16384, &tmq, smem_u32(&bars->q_full), 64, h, r0);
+            }
             int k_issued = 0, v_issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                if (j > 0 && !pf_wait(bars, &bars->k_free, (j - 1) & 1, a.timeout_ns, false)) break;
-                issue(sK, &tmk, &bars->k_full, j);
+            for (int j = 0; j < n_kv; ++j) {
+                const int st = j % kPfStages;
+                const uint32_t use = j / kPfStages;
+                if (use > 0 && !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, false))
+                    break;
+                issue(sK + st * kPfTileBytes, &tmk, &bars->k_full[st], j);
                 k_issued = j + 1;
-                if (j > 0 && !pf_wait(bars, &bars->v_free, (j - 1) & 1, a.timeout_ns, false)) break;
-                issue(sV, &tmv, &bars->v_full, j);
+                if (use > 0 && !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, false))
+                    break;
+                issue(sV + st * kPfTileBytes, &tmv, &bars->v_full[st], j);
                 v_issued = j + 1;
             }
             if (bars->abort) {  // let copies already in flight land
                 mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
-                if (k_issued) mbar_wait(smem_u32(&bars->k_full), (k_issued - 1) & 1, a.timeout_ns);
-                if (v_issued) mbar_wait(smem_u32(&bars->v_full), (v_issued - 1) & 1, a.timeout_ns);
+                for (int j = max(0, k_issued - kPfStages); j < k_issued; ++j)
+                    mbar_wait(smem_u32(&bars->k_full[j % kPfStages]), (j / kPfStages) & 1,
+                              a.timeout_ns);
+                for (int j = max(0, v_issued - kPfStages); j < v_issued; ++j)
+                    mbar_wait(smem_u32(&bars->v_full[j % kPfStages]), (j / kPfStages) & 1,
+                              a.timeout_ns);
             }
         }
-    } else if (warp == 5) {
+      } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             constexpr uint32_t kIdQK = f16_idesc(128, 128, false);
             constexpr uint32_t kIdPV = f16_idesc(128, 128, true);
-            bool ok = pf_wait(bars, &bars->q_full, 0, a.timeout_ns, false);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                if (!pf_wait(bars, &bars->k_full, j & 1, a.timeout_ns, false)) break;
-                if (j > 0 && !pf_wait(bars, &bars->o_full, (j - 1) & 1, a.timeout_ns, false)) break;
+            auto issue_s = [&](int x, int j) -> bool {  // S_x = Q_x K_j^T
+                const int st = j % kPfStages;
+                if (!pf_wait(bars, &bars->k_full[st], (j / kPfStages) & 1, a.timeout_ns, false))
+                    return false;
                 tc_fence_after();
+                const uint32_t q = sQ + x * kPfTileBytes, k = sK + st * kPfTileBytes;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_ss(tS, sw128_desc(sQ + koff, 16, 1024), sw128_desc(sK + koff, 16, 1024),
-                           kIdQK, ks > 0);
+                    mma_ss(tmem + x * 128, sw128_desc(q + koff, 16, 1024),
+                           sw128_desc(k + koff, 16, 1024), kIdQK, ks > 0);
                 }
-                tc_commit(smem_u32(&bars->s_full));
-                tc_commit(smem_u32(&bars->k_free));
-                if (!pf_wait(bars, &bars->p_full, j & 1, a.timeout_ns, false)) break;
-                if (!pf_wait(bars, &bars->v_full, j & 1, a.timeout_ns, false)) break;
+                tc_commit(smem_u32(&bars->s_full[x]));
+                return true;
+            };
+            auto issue_pv = [&](int x, int j) -> bool {  // O_x += P_x V_j
+                const int st = j % kPfStages;
+                if (!pf_wait(bars, &bars->p_full[x], j & 1, a.timeout_ns, false)) return false;
+                if (!pf_wait(bars, &bars->v_full[st], (j / kPfStages) & 1, a.timeout_ns, false))
+                    return false;
                 tc_fence_after();
+                const uint32_t v = sV + st * kPfTileBytes;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    mma_ts(tO, tS + ks * 8, sw128_desc(sV + ks * 2048, 16384, 1024), kIdPV,
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ts(tmem + 256 + x * 128, tmem + x * 128 + ks * 8,
+                           sw128_desc(v + ks * 2048, 16384, 1024), kIdPV,
                            (j > 0 || ks > 0) ? 1u : 0u);
+                tc_commit(smem_u32(&bars->o_full[x]));
+                return true;
+            };
+            bool ok = pf_wait(bars, &bars->q_full, 0, a.timeout_ns, false);
+            // S for the first K tile of every Q tile, then per K/V tile j:
+            // P.V of each Q tile and, behind it in issue order (the tensor
+            // core runs one thread's operations in order, so S may reuse the
+            // P columns), S of the next tile
+            ok = ok && issue_s(0, 0);
+            if (ok && ntile1 > 0) ok = issue_s(1, 0);
+            if (ok) tc_commit(smem_u32(&bars->k_free[0]));
+            for (int j = 0; ok && j < n_kv; ++j) {
+#pragma unroll
+                for (int x = 0; x < kPfQTiles; ++x) {
+                    if (!ok || j >= ntile(x)) continue;
+                    ok = issue_pv(x, j);
+                    if (ok && j + 1 < ntile(x)) ok = issue_s(x, j + 1);
                 }
-                tc_commit(smem_u32(&bars->o_full));
-                tc_commit(smem_u32(&bars->v_free));
+                if (!ok) break;
+                if (j + 1 < n_kv) tc_commit(smem_u32(&bars->k_free[(j + 1) % kPfStages]));
+                tc_commit(smem_u32(&bars->v_free[j % kPfStages]));
             }
             // every tensor-core operation issued above completes before teardown
             tc_commit(smem_u32(&bars->fin));
             mbar_wait(smem_u32(&bars->fin), 0, a.timeout_ns);
         }
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPfSoftmaxRegs));
         // -------------------------------------------------------- softmax
-        const int r = threadIdx.x;  // row of the tile == tensor-memory lane
-        const int i = qt * kPfRows + r;
+        const int x = warp >> 2;                      // Q tile of this warpgroup
+        const int r = threadIdx.x & 127;              // row of the tile == lane
+        const int i = row0 + x * kPfRows + r;         // query index in the chunk
         const bool row_valid = i < C;
-        const int pos = cached + min(i, C - 1);  // keys <= pos are visible
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int pos = cached + min(i, C - 1);       // keys <= pos are visible
+        const int pos_first = cached + row0 + x * kPfRows;  // smallest pos of the tile
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + x * 128 + lane_off;
+        const uint32_t tO = tmem + 256 + x * 128 + lane_off;
         const float sl2 = a.scale_log2;
+        const int nt = ntile(x);
+        // the warpgroup that first consumes the last K/V tile clears its
+        // rows past the context
+        const bool zeroes_tail = nt == n_kv && (x == 0 || ntile0 < n_kv);
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
-            if (!pf_wait(bars, &bars->s_full, j & 1, a.timeout_ns, true)) {
+        for (int j = 0; j < nt; ++j) {
+            if (!pf_wait(bars, &bars->s_full[x], j & 1, a.timeout_ns, true)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            uint32_t sv[128];
+            tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+            tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+            tmem_ld_wait();
             const int key0 = j * kPfKeys;
-            float mt = -INFINITY;
+            const bool diag = key0 + kPfKeys - 1 > pos_first;  // some key masked for some row
+            if (diag) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(tS + lane_off + cc * 32, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int key = key0 + cc * 32 + e;
-                    if (key <= pos) mt = fmaxf(mt, __uint_as_float(v[e]) * sl2);
-                }
+                for (int e = 0; e < 128; ++e)
+                    if (key0 + e > pos) sv[e] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
             }
-            const float m_new = fmaxf(m, mt);
+            // the row's largest scaled score (raw max, or raw min for a
+            // negative scale)
+            float ext = __uint_as_float(sv[0]);
+            if (sl2 >= 0.f) {
+#pragma unroll
+                for (int e = 1; e < 128; ++e) ext = fmaxf(ext, __uint_as_float(sv[e]));
+            } else {
+#pragma unroll
+                for (int e = 1; e < 128; ++e) ext = fminf(ext, __uint_as_float(sv[e]));
+            }
+            const float m_tile = isinf(ext) ? -INFINITY : ext * sl2;
+            const float m_new = fmaxf(m, m_tile);
             if (j == 0) {
                 m = m_new;
             } else if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
-                // re-reference O and the sum to the new max (warp-uniform)
-                const float corr = exp2f(m - m_new);
+                // re-reference O and the sum to the new max
+                const float corr = ex2_approx(m - m_new);
                 l *= corr;
                 m = m_new;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     uint32_t v[32];
-                    tmem_ld32(tO + lane_off + cc * 32, v);
+                    tmem_ld32(tO + cc * 32, v);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
-                    tmem_st32(tO + lane_off + cc * 32, v);
+                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
+                    tmem_st32(tO + cc * 32, v);
                 }
             }
+            const float neg_m = -m;
+            uint32_t pk[64];
+            if (diag) {
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(tS + lane_off + cc * 32, v);
-                tmem_ld_wait();
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int k0 = key0 + cc * 32 + 2 * e;
-                    const float p0 = k0 <= pos ? exp2f(__uint_as_float(v[2 * e]) * sl2 - m) : 0.f;
-                    const float p1 =
-                        k0 + 1 <= pos ? exp2f(__uint_as_float(v[2 * e + 1]) * sl2 - m) : 0.f;
+                for (int e = 0; e < 64; ++e) {
+                    const float p0 = key0 + 2 * e <= pos
+                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m)) : 0.f;
+                    const float p1 = key0 + 2 * e + 1 <= pos
+                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m)) : 0.f;
+                    l += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
-                    l += bf16_lo(pk[e]) + bf16_hi(pk[e]);  // the weights P.V uses
                 }
-                // P for these 32 keys goes to columns [16cc, 16cc+16), whose
-                // S values were consumed earlier in this loop
-                tmem_st16(tS + lane_off + cc * 16, pk);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m));
+                    l += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
             }
+            tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_st_wait();
-            if (j == n_tiles - 1 && key0 + kPfKeys > ctx) {
+            if (zeroes_tail && j == nt - 1 && key0 + kPfKeys > ctx) {
                 // V rows past the context hold stale or unloaded data: zero
                 // them so that P = 0 cannot meet a NaN there
-                if (!pf_wait(bars, &bars->v_full, j & 1, a.timeout_ns, true)) {
+                const int st = j % kPfStages;
+                if (!pf_wait(bars, &bars->v_full[st], (j / kPfStages) & 1, a.timeout_ns, true)) {
                     ok = false;
                     break;
                 }
                 const int vr = ctx - key0;
+                const uint32_t vb = sV + st * kPfTileBytes;
                 for (int e = r; e < (kPfKeys - vr) * 16; e += 128) {
                     const int row = vr + e / 16, u = e % 16;
-                    const uint32_t addr = sV + (u / 8) * 16384 + row * 128 + (u % 8) * 16;
+                    const uint32_t addr = vb + (u / 8) * 16384 + row * 128 + (u % 8) * 16;
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
                                  : "memory");
                 }
                 fence_proxy_async_smem();
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(&bars->p_full));
+            mbar_arrive(smem_u32(&bars->p_full[x]));
         }
-        if (ok && pf_wait(bars, &bars->o_full, (n_tiles - 1) & 1, a.timeout_ns, true)) {
+        if (ok && nt > 0 && pf_wait(bars, &bars->o_full[x], (nt - 1) & 1, a.timeout_ns, true)) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + h) * 128;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 uint32_t v[32];
-                tmem_ld32(tO + lane_off + cc * 32, v);
+                tmem_ld32(tO + cc * 32, v);
                 tmem_ld_wait();
-                uint32_t pk[16];
+                uint32_t o[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
-                                        __uint_as_float(v[2 * e + 1]) * inv);
+                    o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
+                                       __uint_as_float(v[2 * e + 1]) * inv);
                 if (row_valid) {
                     uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
                 }
             }
         }
@@ -435,10 +529,10 @@ __global__ void __launch_bounds__(kPfThreads, 2)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tS, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
