@@ -51,7 +51,8 @@ constexpr int kPfCtlRegs = 56;
 constexpr int kPfSoftmaxRegs = 224;
 constexpr int kPfRegsNeeded = 128 * (2 * kPfSoftmaxRegs + kPfCtlRegs);
 constexpr int kPfTileBytes = kPfRows * 128 * 2;  // 128 x 128 bf16 = 32 KB
-constexpr int kPfSmem = (kPfQTiles + 2 * kPfStages) * kPfTileBytes + 512;
+constexpr int kPfTblMax = 4096;   // block-table entries staged in shared memory
+constexpr int kPfSmem = (kPfQTiles + 2 * kPfStages) * kPfTileBytes + 512 + kPfTblMax * 4;
 
 struct PrefillArgs {
     __nv_bfloat16 *out;
@@ -216,6 +217,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t sK = sQ + kPfQTiles * kPfTileBytes;          // K stage st at sK + st*32K
     const uint32_t sV = sK + kPfStages * kPfTileBytes;          // V stage st at sV + st*32K
     PfBars *bars = reinterpret_cast<PfBars *>(smem + (kPfQTiles + 2 * kPfStages) * kPfTileBytes);
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + (kPfQTiles + 2 * kPfStages) * kPfTileBytes +
+                                               512);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tp = blockIdx.x, h = blockIdx.y;
@@ -260,6 +263,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_alloc(smem_u32(&bars->tmem_base), 512);
         tmem_relinquish();
     }
+    // the chunk's block-table slice, checked once, into shared memory (the
+    // first kPfTblMax entries; a longer context reads the rest from global)
+    const int n_blk = (ctx + a.bs - 1) / a.bs;
+    const int32_t *trow = a.block_tables + (size_t)c * a.MB;
+    for (int e = threadIdx.x; e < min(n_blk, kPfTblMax); e += kPfThreads) {
+        int id = __ldg(trow + e);
+        if (id < 0 || id >= a.NB) {
+            flag_error(PA_ERR_BAD_TABLE);
+            id = -1;
+        }
+        tbl[e] = id;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -271,66 +286,63 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfCtlRegs));
       if (warp == 8) {
         // ------------------------------------------------------------ TMA
-        if (lane == 0) {
-            const int n_blk = (ctx + a.bs - 1) / a.bs;
-            const int32_t *trow = a.block_tables + (size_t)c * a.MB;
-            auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j) {
-                int ids[8];
-                int n = 0;
-#pragma unroll
-                for (int s16 = 0; s16 < 8; ++s16) {
-                    const int key = j * kPfKeys + s16 * 16;
-                    int id = -1;
-                    if (key < ctx) {
-                        const int lb = key / a.bs;
-                        id = lb < n_blk ? __ldg(trow + lb) : -1;
-                        if (id < 0 || id >= a.NB) {
-                            flag_error(PA_ERR_BAD_TABLE);
-                            id = -1;
-                        }
+        // One box per lane: a thread issuing tensor copies back to back is
+        // slow (each issue takes a while to be accepted), so the 16 boxes
+        // of a K or V tile (8 pieces of 16 tokens x 2 halves of 64 dims)
+        // go out from 16 lanes at once. Lane 0 arms the barrier first with
+        // the exact byte count of the pieces that exist.
+        const int s16 = lane >> 1, half = lane & 1;
+        auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j) {
+            const int key = j * kPfKeys + s16 * 16;
+            int id = -1;
+            if (lane < 16 && key < ctx) {
+                const int lb = key / a.bs;
+                if (lb < kPfTblMax) {
+                    id = tbl[lb];
+                } else {
+                    id = __ldg(trow + lb);
+                    if (id < 0 || id >= a.NB) {
+                        flag_error(PA_ERR_BAD_TABLE);
+                        id = -1;
                     }
-                    ids[s16] = id;
-                    n += id >= 0;
                 }
-                mbar_arrive_expect_tx(smem_u32(bar), n * 2 * 2048);
-#pragma unroll
-                for (int s16 = 0; s16 < 8; ++s16) {
-                    if (ids[s16] < 0) continue;
-                    const int off = (j * kPfKeys + s16 * 16) % a.bs;
-                    tma_load_4d(dst + s16 * 2048, map, smem_u32(bar), 0, off, kvh, ids[s16]);
-                    tma_load_4d(dst + 16384 + s16 * 2048, map, smem_u32(bar), 64, off, kvh,
-                                ids[s16]);
-                }
-            };
-            const int nq = rows1 > 0 ? 2 : 1;
-            mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * kPfTileBytes);
-            for (int x = 0; x < nq; ++x) {
-                const int r0 = q0 + row0 + x * kPfRows;
-                tma_load_3d(sQ + x * kPfTileBytes, &tmq, smem_u32(&bars->q_full), 0, h, r0);
-                tma_load_3d(sQ + x * kPfTileBytes + 16384, &tmq, smem_u32(&bars->q_full), 64, h, r0);
             }
-            int k_issued = 0, v_issued = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int st = j % kPfStages;
-                const uint32_t use = j / kPfStages;
-                if (use > 0 && !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, false))
-                    break;
-                issue(sK + st * kPfTileBytes, &tmk, &bars->k_full[st], j);
-                k_issued = j + 1;
-                if (use > 0 && !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, false))
-                    break;
-                issue(sV + st * kPfTileBytes, &tmv, &bars->v_full[st], j);
-                v_issued = j + 1;
-            }
-            if (bars->abort) {  // let copies already in flight land
-                mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
-                for (int j = max(0, k_issued - kPfStages); j < k_issued; ++j)
-                    mbar_wait(smem_u32(&bars->k_full[j % kPfStages]), (j / kPfStages) & 1,
-                              a.timeout_ns);
-                for (int j = max(0, v_issued - kPfStages); j < v_issued; ++j)
-                    mbar_wait(smem_u32(&bars->v_full[j % kPfStages]), (j / kPfStages) & 1,
-                              a.timeout_ns);
-            }
+            const int n = __popc(__ballot_sync(0xffffffffu, id >= 0));
+            if (lane == 0) mbar_arrive_expect_tx(smem_u32(bar), n * 2048);
+            __syncwarp();
+            if (id >= 0)
+                tma_load_4d(dst + half * 16384 + s16 * 2048, map, smem_u32(bar), half * 64,
+                            key % a.bs, kvh, id);
+        };
+        const int nq = rows1 > 0 ? 2 : 1;
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * kPfTileBytes);
+        __syncwarp();
+        if (lane < 2 * nq) {
+            const int x = lane >> 1, hf = lane & 1;
+            tma_load_3d(sQ + x * kPfTileBytes + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64,
+                        h, q0 + row0 + x * kPfRows);
+        }
+        int k_issued = 0, v_issued = 0;
+        for (int j = 0; j < n_kv; ++j) {
+            const int st = j % kPfStages;
+            const uint32_t use = j / kPfStages;
+            if (use > 0 && !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
+                break;
+            issue(sK + st * kPfTileBytes, &tmk, &bars->k_full[st], j);
+            k_issued = j + 1;
+            if (use > 0 && !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
+                break;
+            issue(sV + st * kPfTileBytes, &tmv, &bars->v_full[st], j);
+            v_issued = j + 1;
+        }
+        if (bars->abort && lane == 0) {  // let copies already in flight land
+            mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
+            for (int j = max(0, k_issued - kPfStages); j < k_issued; ++j)
+                mbar_wait(smem_u32(&bars->k_full[j % kPfStages]), (j / kPfStages) & 1,
+                          a.timeout_ns);
+            for (int j = max(0, v_issued - kPfStages); j < v_issued; ++j)
+                mbar_wait(smem_u32(&bars->v_full[j % kPfStages]), (j / kPfStages) & 1,
+                          a.timeout_ns);
         }
       } else if (warp == 9) {
         // ------------------------------------------------------------ MMA
@@ -431,13 +443,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
             // the row's largest scaled score (raw max, or raw min for a
             // negative scale)
-            float ext = __uint_as_float(sv[0]);
-            if (sl2 >= 0.f) {
+            float ext;
+            {
+                // eight independent running extrema, then a tree
+                float t[8];
 #pragma unroll
-                for (int e = 1; e < 128; ++e) ext = fmaxf(ext, __uint_as_float(sv[e]));
-            } else {
+                for (int u = 0; u < 8; ++u) t[u] = __uint_as_float(sv[u]);
+                if (sl2 >= 0.f) {
 #pragma unroll
-                for (int e = 1; e < 128; ++e) ext = fminf(ext, __uint_as_float(sv[e]));
+                    for (int e = 8; e < 128; ++e) t[e & 7] = fmaxf(t[e & 7], __uint_as_float(sv[e]));
+#pragma unroll
+                    for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                        for (int u = 0; u < w; ++u) t[u] = fmaxf(t[u], t[u + w]);
+                } else {
+#pragma unroll
+                    for (int e = 8; e < 128; ++e) t[e & 7] = fminf(t[e & 7], __uint_as_float(sv[e]));
+#pragma unroll
+                    for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                        for (int u = 0; u < w; ++u) t[u] = fminf(t[u], t[u + w]);
+                }
+                ext = t[0];
             }
             const float m_tile = isinf(ext) ? -INFINITY : ext * sl2;
             const float m_new = fmaxf(m, m_tile);
@@ -460,6 +487,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
             const float neg_m = -m;
             uint32_t pk[64];
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
             if (diag) {
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
@@ -467,7 +495,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                          ? ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m)) : 0.f;
                     const float p1 = key0 + 2 * e + 1 <= pos
                                          ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m)) : 0.f;
-                    l += p0 + p1;
+                    ls[e & 3] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
             } else {
@@ -475,10 +503,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 for (int e = 0; e < 64; ++e) {
                     const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m));
                     const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m));
-                    l += p0 + p1;
+                    ls[e & 3] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }
             }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
             tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_st_wait();

@@ -218,3 +218,66 @@ def pa_selftest_bounded_wait(timeout_ns: int, stream=None) -> None:
 
 def pa_version() -> int:
     return int(lib().pa_version())
+
+
+# ---------------------------------------------------------------------------
+# prepared calls: arguments marshalled once, for loops that issue the same
+# call every step (the tensors' storage must stay alive and unmoved)
+# ---------------------------------------------------------------------------
+class Prepared:
+    """One C-ABI call with its pointer and size arguments fixed. Calling it
+    launches on the given (or current) stream and raises on a non-OK status."""
+
+    def __init__(self, fn: str, args):
+        self.name = fn
+        self._fn = getattr(lib(), fn)
+        self._args = tuple(args)
+
+    def __call__(self, stream=None):
+        st = self._fn(*self._args, _stream(stream))
+        if st != PA_OK:
+            raise PAError(self.name, st)
+
+
+def prepare_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping) -> Prepared:
+    _check_int(slot_mapping, torch.int64, "slot_mapping")
+    NB, H_kv, bs, D = k_cache.shape
+    T = slot_mapping.numel()
+    if key.shape != (T, H_kv, D) or value.shape != (T, H_kv, D):
+        raise ValueError("key/value must be [num_tokens, num_kv_heads, head_dim]")
+    return Prepared("pa_reshape_and_cache", (_p(key), _p(value), _p(k_cache), _p(v_cache),
+                                             _p(slot_mapping), T, H_kv, D, bs, NB,
+                                             _dt(k_cache)))
+
+
+def prepare_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
+                   scale: float, partition_size: int = 0,
+                   workspace: Optional[torch.Tensor] = None) -> Prepared:
+    _check_int(block_tables, torch.int32, "block_tables")
+    _check_int(context_lens, torch.int32, "context_lens")
+    B, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
+        raise ValueError("out must match q; caches must share head_dim")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return Prepared("pa_decode", (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
+                                  _p(context_lens), B, H_q, H_kv, D, bs, NB,
+                                  block_tables.shape[1], int(max_context_len), float(scale),
+                                  int(partition_size), _p(workspace), ws_bytes, _dt(q)))
+
+
+def prepare_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                          max_query_len: int, scale: float) -> Prepared:
+    for t, n in ((block_tables, "block_tables"), (context_lens, "context_lens"),
+                 (query_start_loc, "query_start_loc")):
+        _check_int(t, torch.int32, n)
+    total_q, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
+        raise ValueError("out must match q; caches must share head_dim")
+    return Prepared("pa_prefill_chunk", (_p(out), _p(q), _p(k_cache), _p(v_cache),
+                                         _p(block_tables), _p(context_lens), _p(query_start_loc),
+                                         query_start_loc.numel() - 1, total_q, int(max_query_len),
+                                         H_q, H_kv, D, bs, NB, block_tables.shape[1],
+                                         float(scale), _dt(q)))
+
