@@ -342,6 +342,8 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     dist = init_dist(world, "nccl")
     batch = make_batch(args.workload, seed=rank, num_blocks=args.num_blocks)
+    if args.partition is not None:
+        batch.partition_size = args.partition
     r = Runner(batch, dev)
     hbm, bf16, bf16_sus, basis = load_peaks()
 
@@ -638,6 +640,8 @@ def main(argv=None):
                              "mixed_prefill_decode"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--partition", type=int, default=None,
+                    help="decode KV partition tokens (0 automatic, <0 no split)")
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="physical pool size override (a smaller pool for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

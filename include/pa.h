@@ -181,6 +181,35 @@ PA_API pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache,
                            int num_blocks, int max_blocks_per_seq, float scale, pa_dtype dtype,
                            cudaStream_t stream);
 
+/* Copy-on-write of whole blocks inside one pool: for each pair i of
+ * block_mapping (int64 [num_pairs][2], device-readable), block
+ * block_mapping[i][1] := block block_mapping[i][0], every kv head, K and V,
+ * bit for bit. This is how a beam gets its own copy of a shared, partially
+ * filled block before writing into it (page "字节跳动 AI Infra (2)", question
+ * "vLLM与PagedAttention的原理": B6' is a copy-on-write copy of B6).
+ * Destinations must be distinct and must not be sources of other pairs (the
+ * pairs run concurrently). An id outside [0, num_blocks) skips its pair and
+ * is recorded as PA_ERR_BAD_TABLE. */
+PA_API pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping,
+                                int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                                int num_blocks, pa_dtype dtype, cudaStream_t stream);
+
+/* Whole-block copies between two pools of the same block shape, e.g. the
+ * device pool and a pinned host pool holding swapped-out requests (page
+ * "字节跳动 AI Infra (2)", scheduler: KV caches are swapped to CPU memory when
+ * GPU memory runs short, and back). For each pair i: block mapping[i][1] of
+ * (dst_k, dst_v) := block mapping[i][0] of (src_k, src_v). Every pointer must
+ * be addressable by the GPU: device memory, or pinned host memory (page-
+ * locked with cudaHostAlloc / cudaHostRegister, addressed through unified
+ * virtual addressing); the copy then runs over the host link inside one
+ * kernel. Ids outside their pool skip the pair and are recorded as
+ * PA_ERR_BAD_TABLE. */
+PA_API pa_status pa_swap_blocks(const void *src_k, const void *src_v, int src_blocks,
+                                void *dst_k, void *dst_v, int dst_blocks,
+                                const int64_t *block_mapping, int num_pairs, int num_kv_heads,
+                                int head_dim, int block_size, pa_dtype dtype,
+                                cudaStream_t stream);
+
 /* Check block tables and lengths on the device: every entry a row's valid
  * tokens reach must lie in [0, num_blocks), and 0 <= context_lens[r] <=
  * max_blocks_per_seq*block_size. d_scratch is one caller-owned device int32.

@@ -74,8 +74,9 @@ def _load():
             lib.oracle_lse_merge.argtypes = [P, P, P, P, I64, I, I]
             lib.oracle_lse_merge.restype = None
             lib.oracle_prefill.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, I, I64, D, P]
+            lib.oracle_copy_blocks.argtypes = [P, P, I64, P, P, I64, P, I64, I64]
             for f in ("oracle_reshape_and_cache", "oracle_decode", "oracle_decode_partials",
-                      "oracle_prefill"):
+                      "oracle_prefill", "oracle_copy_blocks"):
                 getattr(lib, f).restype = I
             _lib = lib
     return _lib
@@ -238,3 +239,20 @@ def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, sc
                                 n_chunks, H_q, H_kv, D, bs, MB, NB, float(scale), _ptr(sel))
     _check(rc, "prefill")
     return out, lse
+
+
+def copy_blocks(src_k, src_v, dst_k, dst_v, mapping) -> None:
+    """Whole-block copies between pools (or within one): for each row (s, d)
+    of ``mapping`` (int64 [n, 2]), block d of dst := block s of src, K and
+    V. Copy-on-write and swap-out/in are both this operation."""
+    mapping = _cpu(mapping, torch.int64)
+    for t in (src_k, src_v, dst_k, dst_v):
+        if not t.is_contiguous() or t.device.type != "cpu":
+            raise ValueError("pools must be contiguous host tensors")
+    assert src_k.shape[1:] == dst_k.shape[1:] and src_k.dtype == dst_k.dtype
+    block_bytes = src_k[0].numel() * src_k.element_size()
+    rc = _load().oracle_copy_blocks(_ptr(src_k), _ptr(src_v), src_k.shape[0], _ptr(dst_k),
+                                    _ptr(dst_v), dst_k.shape[0], _ptr(mapping),
+                                    mapping.shape[0] if mapping.numel() else 0, block_bytes)
+    _check(rc, "copy_blocks")
+

@@ -342,3 +342,29 @@ int oracle_prefill(double *out, double *lse, const void *q, const void *k_cache,
     }
     return err;
 }
+
+/* Block copies of the paged pool, whole blocks (every K/V head) at a time:
+ * page "字节跳动 AI Infra (2)", question "vLLM与PagedAttention的原理": a beam
+ * that must write into a block it shares gets a copy of it first (B6' is a
+ * copy-on-write copy of B6); the scheduler moves a swapped-out request's
+ * blocks to CPU memory and back (same page, scheduler section: KV cache
+ * swapped to CPU when memory runs short).
+ * For each pair i: block mapping[2i+1] of (dst_k, dst_v) := block mapping[2i]
+ * of (src_k, src_v); a block is block_bytes contiguous bytes. A pair with an
+ * id outside its pool returns OR_BAD_BLOCK before anything is written. */
+int oracle_copy_blocks(const void *src_k, const void *src_v, int64_t src_blocks, void *dst_k,
+                       void *dst_v, int64_t dst_blocks, const int64_t *mapping, int64_t num_pairs,
+                       int64_t block_bytes)
+{
+    if (num_pairs < 0 || block_bytes <= 0 || src_blocks <= 0 || dst_blocks <= 0) return OR_BAD_ARG;
+    for (int64_t i = 0; i < num_pairs; ++i)
+        if (mapping[2 * i] < 0 || mapping[2 * i] >= src_blocks || mapping[2 * i + 1] < 0 ||
+            mapping[2 * i + 1] >= dst_blocks)
+            return OR_BAD_BLOCK;
+    for (int64_t i = 0; i < num_pairs; ++i) {
+        size_t s = (size_t)mapping[2 * i] * block_bytes, d = (size_t)mapping[2 * i + 1] * block_bytes;
+        memcpy((char *)dst_k + d, (const char *)src_k + s, block_bytes);
+        memcpy((char *)dst_v + d, (const char *)src_v + s, block_bytes);
+    }
+    return OR_OK;
+}

@@ -19,6 +19,7 @@
 #include "reshape_and_cache.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "blocks.cuh"
 
 namespace {
 
@@ -149,6 +150,32 @@ pa_status dispatch_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtens
     if (p.nw == 4 && p.ns == 1) return launch_decode_bf16<D, 4, 1>(a, mk, mv, grid, st);
     if (p.nw == 4 && p.ns == 3) return launch_decode_bf16<D, 4, 3>(a, mk, mv, grid, st);
     return launch_decode_bf16<D, 4, 2>(a, mk, mv, grid, st);
+}
+
+// PA_PREFILL_POLY=4 computes every 4th pair of softmax exponentials in full
+// prefill tiles on the FMA pipe instead of the special-function unit. Off by
+// default: on B200 the softmax is limited by instruction issue, not by the
+// special-function unit, and the extra instructions cost more than they save.
+int prefill_poly() {
+    static int v = [] {
+        const char *e = std::getenv("PA_PREFILL_POLY");
+        return (e && std::atoi(e) == 4) ? 4 : 0;
+    }();
+    return v;
+}
+
+template <int POLY>
+pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                            const CUtensorMap &mv, dim3 grid, size_t smem, cudaStream_t st) {
+    auto k = prefill_tc_kernel<POLY>;
+    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
+    // the kernel's register split must fit the registers it launches with,
+    // or the warpgroups that grow would wait forever
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return PA_ERR_CUDA;
+    if ((long long)fa.numRegs * kPfThreads < kPfRegsNeeded) return PA_ERR_UNSUPPORTED;
+    k<<<grid, kPfThreads, smem, st>>>(a, mq, mk, mv);
+    return launch_status();
 }
 
 }  // namespace
@@ -365,17 +392,63 @@ pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const 
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
     const size_t smem = 1024 + kPfSmem;
-    if (set_smem(prefill_tc_kernel, smem) != cudaSuccess) return PA_ERR_CUDA;
-    {
-        // the kernel's register split must fit the registers it launches
-        // with, or the warpgroups that grow would wait forever
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, prefill_tc_kernel) != cudaSuccess) return PA_ERR_CUDA;
-        if ((long long)fa.numRegs * kPfThreads < kPfRegsNeeded) return PA_ERR_UNSUPPORTED;
-    }
     const dim3 grid((unsigned)qtiles, (unsigned)num_q_heads, (unsigned)num_chunks);
-    prefill_tc_kernel<<<grid, kPfThreads, smem, stream>>>(a, mq, mk, mv);
+    if (prefill_poly() == 4) return launch_prefill_tc<4>(a, mq, mk, mv, grid, smem, stream);
+    return launch_prefill_tc<0>(a, mq, mk, mv, grid, smem, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+pa_status launch_copy_blocks(const void *src_k, const void *src_v, long long src_blocks,
+                             void *dst_k, void *dst_v, long long dst_blocks,
+                             const int64_t *mapping, int num_pairs, int num_kv_heads, int head_dim,
+                             int block_size, pa_dtype dtype, cudaStream_t stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        src_blocks <= 0 || dst_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (!head_dim_ok(head_dim) || !block_size_ok(block_size)) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!src_k || !src_v || !dst_k || !dst_v || !mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned(src_k, 16) || !aligned(src_v, 16) || !aligned(dst_k, 16) ||
+        !aligned(dst_v, 16) || !aligned(mapping, 8))
+        return PA_ERR_INVALID_ARG;
+    const long long bytes = (long long)num_kv_heads * block_size * head_dim *
+                            (dtype == PA_BF16 ? 2 : 4);
+    if (bytes / 16 > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    CopyArgs a;
+    a.src_k = static_cast<const uint4 *>(src_k);
+    a.src_v = static_cast<const uint4 *>(src_v);
+    a.dst_k = static_cast<uint4 *>(dst_k);
+    a.dst_v = static_cast<uint4 *>(dst_v);
+    a.mapping = mapping;
+    a.src_blocks = src_blocks;
+    a.dst_blocks = dst_blocks;
+    a.vecs_per_block = (int)(bytes / 16);
+    copy_blocks_kernel<<<num_pairs, 256, 0, stream>>>(a);
     return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, cudaStream_t stream) {
+    return launch_copy_blocks(k_cache, v_cache, num_blocks, k_cache, v_cache, num_blocks,
+                              block_mapping, num_pairs, num_kv_heads, head_dim, block_size, dtype,
+                              stream);
+}
+
+pa_status pa_swap_blocks(const void *src_k, const void *src_v, int src_blocks, void *dst_k,
+                         void *dst_v, int dst_blocks, const int64_t *block_mapping, int num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, pa_dtype dtype,
+                         cudaStream_t stream) {
+    return launch_copy_blocks(src_k, src_v, src_blocks, dst_k, dst_v, dst_blocks, block_mapping,
+                              num_pairs, num_kv_heads, head_dim, block_size, dtype, stream);
 }
 
 }  // extern "C"

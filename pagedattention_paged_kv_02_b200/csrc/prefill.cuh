@@ -206,6 +206,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, to take part of the softmax's exponentials off the
+// special-function unit. Cody-Waite style range reduction: x = n + f with
+// n = round(x) (adding 1.5*2^23 leaves n in the low mantissa bits) and
+// |f| <= 1/2; 2^f by a cubic 1 + c1 f + c2 f^2 + c3 f^3 whose coefficients
+// were fitted for minimum maximum relative error on [-1/2, 1/2] (1.02e-4,
+// about 2^-13, exact at f = 0: below the bf16 rounding of P); 2^n is added
+// to the exponent field. Inputs below -125 give 2^-125.
+__device__ __forceinline__ float ex2_poly(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float n = t - 12582912.f;
+    const float f = x - n;
+    const float p = fmaf(fmaf(fmaf(0.05500824f, f, 0.24220951f), f, 0.69328284f), f, 1.f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// POLY: every POLY-th pair of exponentials in a full (unmasked) tile is
+// computed with ex2_poly instead of the special-function unit (0 = none).
+template <int POLY>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
@@ -501,8 +520,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             } else {
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m));
+                    float p0, p1;
+                    if (POLY > 0 && e % POLY == POLY - 1) {
+                        p0 = ex2_poly(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m));
+                        p1 = ex2_poly(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m));
+                    } else {
+                        p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m));
+                        p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m));
+                    }
                     ls[e & 3] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
                 }

@@ -25,7 +25,7 @@ PA_F32, PA_BF16 = 0, 1
 EXPORTS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_partition_tokens",
            "pa_decode", "pa_prefill_chunk", "pa_check_tables", "pa_device_error",
            "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
-           "pa_decode_static_workspace")
+           "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks")
 
 
 class PAError(RuntimeError):
@@ -55,13 +55,15 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_static_workspace.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I,
                                                  I, P]
         L.pa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P]
+        L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P]
+        L.pa_swap_blocks.argtypes = [P, P, I, P, P, I, P, I, I, I, I, I, P]
         L.pa_check_tables.argtypes = [P, P, I, I, I, I, P, ctypes.POINTER(I), P]
         L.pa_device_error.argtypes = [ctypes.POINTER(I), I]
         L.pa_selftest_bounded_wait.argtypes = [I64, P]
         L.pa_status_string.argtypes = [I]
         L.pa_status_string.restype = ctypes.c_char_p
         for f in ("pa_reshape_and_cache", "pa_decode", "pa_decode_static_workspace",
-                  "pa_prefill_chunk", "pa_check_tables",
+                  "pa_prefill_chunk", "pa_check_tables", "pa_copy_blocks", "pa_swap_blocks",
                   "pa_device_error", "pa_selftest_bounded_wait", "pa_decode_partition_tokens",
                   "pa_version"):
             getattr(L, f).restype = I
@@ -188,6 +190,39 @@ def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query
     _call("pa_prefill_chunk", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
           _p(context_lens), _p(query_start_loc), n_chunks, total_q, int(max_query_len), H_q,
           H_kv, D, bs, NB, MB, float(scale), _dt(q), _stream(stream))
+
+
+def _addressable(t: torch.Tensor):
+    """Device tensors, or pinned host tensors the GPU reaches directly."""
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError("device or pinned host tensors expected")
+    if not t.is_contiguous():
+        raise ValueError("contiguous tensors expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:
+    """Copy-on-write: block ``block_mapping[i, 1]`` := block
+    ``block_mapping[i, 0]`` in the same pool (int64 [n, 2])."""
+    _check_int(block_mapping, torch.int64, "block_mapping")
+    NB, H_kv, bs, D = k_cache.shape
+    n = block_mapping.shape[0] if block_mapping.numel() else 0
+    _call("pa_copy_blocks", _p(k_cache), _p(v_cache), _addressable(block_mapping), n, H_kv, D,
+          bs, NB, _dt(k_cache), _stream(stream))
+
+
+def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, stream=None) -> None:
+    """Block ``block_mapping[i, 1]`` of the destination pool := block
+    ``block_mapping[i, 0]`` of the source pool; either pool may be pinned
+    host memory."""
+    _check_int(block_mapping, torch.int64, "block_mapping")
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype:
+        raise ValueError("pools must share block shape and dtype")
+    _, H_kv, bs, D = src_k.shape
+    n = block_mapping.shape[0] if block_mapping.numel() else 0
+    _call("pa_swap_blocks", _addressable(src_k), _addressable(src_v), src_k.shape[0],
+          _addressable(dst_k), _addressable(dst_v), dst_k.shape[0], _addressable(block_mapping),
+          n, H_kv, D, bs, _dt(src_k), _stream(stream))
 
 
 def pa_check_tables(block_tables, context_lens, block_size: int, num_blocks: int,

@@ -422,3 +422,59 @@ def test_select_computes_only_selected():
     sel[1, 3] = sel[0, 0] = True
     part, _ = oracle.decode(q, kc, vc, tables, lens, 0.5, select=sel)
     assert torch.equal(part[sel], full[sel]) and torch.all(part[~sel] == 0)
+
+
+# ---------------------------------------------------------------------------
+# whole-block copies (copy-on-write, swap)
+# ---------------------------------------------------------------------------
+def test_cow_copy_then_diverge(golden):
+    """The beam example: beams share B1, B3 and B6; before beam 2 appends,
+    B6 is copied to B6'. Afterwards beam 1 and beam 2 read the same prefix
+    and differ only in what each appended; the copy is bit-exact and nothing
+    else in the pool moves."""
+    ex = golden["block_tables"]
+    bs, H, D = ex["block_size"], 2, 8
+    g = torch.Generator().manual_seed(30)
+    NB = 9  # B0..B7 plus B6' at id 8
+    kc = torch.randn(NB, H, bs, D, generator=g)
+    vc = torch.randn(NB, H, bs, D, generator=g)
+    before_k, before_v = kc.clone(), vc.clone()
+    oracle.copy_blocks(kc, vc, kc, vc, torch.tensor([[6, 8]]))
+    assert torch.equal(kc[8], before_k[6]) and torch.equal(vc[8], before_v[6])
+    assert torch.equal(kc[:8], before_k[:8]) and torch.equal(vc[:8], before_v[:8])
+    # beam 2 appends at offset 5 of its copy; beam 1 at offset 5 of B6
+    shared = ex["beams"]["shared"]
+    b1 = shared + [6]
+    b2 = shared + [8]
+    key = torch.randn(2, H, D, generator=g)
+    oracle.reshape_and_cache(key, key, kc, vc, torch.tensor([6 * bs + 5, 8 * bs + 5]))
+    ctx = 2 * bs + 6
+    q = torch.randn(2, 2, D, generator=g)
+    tables = torch.tensor([b1, b2], dtype=torch.int32)
+    lens = torch.tensor([ctx, ctx], dtype=torch.int32)
+    out, _ = oracle.decode(q, kc, vc, tables, lens, 0.3)
+    # same query against beam 1's table with beam 2's appended row gives beam 2's answer
+    kc2, vc2 = kc.clone(), vc.clone()
+    kc2[6, :, 5], vc2[6, :, 5] = key[1], key[1]
+    out_b2_via_b1, _ = oracle.decode(q[1:], kc2, vc2, tables[:1], lens[:1], 0.3)
+    assert torch.equal(out[1], out_b2_via_b1[0])
+    assert not torch.equal(out[0], out[1])
+
+
+def test_swap_round_trip_and_errors():
+    g = torch.Generator().manual_seed(31)
+    dev_k = torch.randn(6, 2, 16, 8, generator=g).to(torch.bfloat16)
+    dev_v = torch.randn(6, 2, 16, 8, generator=g).to(torch.bfloat16)
+    host_k = torch.zeros(4, 2, 16, 8, dtype=torch.bfloat16)
+    host_v = torch.zeros_like(host_k)
+    out_map = torch.tensor([[5, 0], [1, 3]])
+    oracle.copy_blocks(dev_k, dev_v, host_k, host_v, out_map)
+    assert torch.equal(host_k[0], dev_k[5]) and torch.equal(host_v[3], dev_v[1])
+    assert torch.all(host_k[1] == 0) and torch.all(host_k[2] == 0)
+    back_k, back_v = torch.zeros_like(dev_k), torch.zeros_like(dev_v)
+    oracle.copy_blocks(host_k, host_v, back_k, back_v, out_map.flip(1))
+    assert torch.equal(back_k[5], dev_k[5]) and torch.equal(back_v[1], dev_v[1])
+    with pytest.raises(ValueError):
+        oracle.copy_blocks(dev_k, dev_v, host_k, host_v, torch.tensor([[6, 0]]))
+    with pytest.raises(ValueError):
+        oracle.copy_blocks(dev_k, dev_v, host_k, host_v, torch.tensor([[0, 4]]))
