@@ -260,11 +260,14 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
-def make_batch(name: str, seed: int, num_blocks=None):
+def make_batch(name: str, seed: int, num_blocks=None, block_size=None):
     from pagedattention_paged_kv_02_b200 import workloads as W
+    kw = {}
     if num_blocks:
-        return W.WORKLOADS[name](seed=seed, num_blocks=num_blocks)
-    return W.WORKLOADS[name](seed=seed)
+        kw["num_blocks"] = num_blocks
+    if block_size:
+        kw["block_size"] = block_size
+    return W.WORKLOADS[name](seed=seed, **kw)
 
 
 class Runner:
@@ -341,7 +344,8 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     dist = init_dist(world, "nccl")
-    batch = make_batch(args.workload, seed=rank, num_blocks=args.num_blocks)
+    batch = make_batch(args.workload, seed=rank, num_blocks=args.num_blocks,
+                       block_size=args.block_size)
     if args.partition is not None:
         batch.partition_size = args.partition
     r = Runner(batch, dev)
@@ -642,6 +646,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--partition", type=int, default=None,
                     help="decode KV partition tokens (0 automatic, <0 no split)")
+    ap.add_argument("--block-size", type=int, default=None, choices=[16, 32, 64],
+                    help="block size override for the decode workloads (pool bytes kept)")
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="physical pool size override (a smaller pool for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -21,6 +21,10 @@ Sources, by page title and section:
 * page "字节跳动 AI Infra (2)", table of algorithm-level optimisations,
   FlashDecoding row: split along the KV length (:func:`decode_partials`,
   :func:`lse_merge`).
+* page "字节跳动 AI Infra (2)", optimisation table, KV quantisation row, and
+  page "LLM推理优化", section 1.3 (quantised KV cache): FP8 E4M3 codes with a
+  scale per K/V head (:func:`e4m3_encode`, :func:`reshape_and_cache_e4m3`,
+  :func:`decode_e4m3`).
 * page "vLLM框架是怎么做推理加速的", section 3: chunked prefill; page
   "LLM推理优化", section 2.3: causal attention (:func:`prefill`).
 
@@ -75,8 +79,17 @@ def _load():
             lib.oracle_lse_merge.restype = None
             lib.oracle_prefill.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, I, I64, D, P]
             lib.oracle_copy_blocks.argtypes = [P, P, I64, P, P, I64, P, I64, I64]
+            lib.oracle_e4m3_encode_array.argtypes = [P, P, I64]
+            lib.oracle_e4m3_encode_array.restype = None
+            lib.oracle_e4m3_decode_array.argtypes = [P, P, I64]
+            lib.oracle_e4m3_decode_array.restype = None
+            lib.oracle_reshape_and_cache_e4m3.argtypes = [P, P, I, P, P, P, I64, I, I, I, I64, P,
+                                                          P]
+            lib.oracle_decode_e4m3.argtypes = [P, P, P, I, P, P, P, P, P, P, I, I, I, I, I, I,
+                                               I64, D, P]
             for f in ("oracle_reshape_and_cache", "oracle_decode", "oracle_decode_partials",
-                      "oracle_prefill", "oracle_copy_blocks"):
+                      "oracle_prefill", "oracle_copy_blocks", "oracle_reshape_and_cache_e4m3",
+                      "oracle_decode_e4m3"):
                 getattr(lib, f).restype = I
             _lib = lib
     return _lib
@@ -255,4 +268,63 @@ def copy_blocks(src_k, src_v, dst_k, dst_v, mapping) -> None:
                                     _ptr(dst_v), dst_k.shape[0], _ptr(mapping),
                                     mapping.shape[0] if mapping.numel() else 0, block_bytes)
     _check(rc, "copy_blocks")
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) KV cache
+# --------------------------------------------------------------------------
+def e4m3_encode(x) -> torch.Tensor:
+    """E4M3 codes (uint8) of fp32 values: nearest value, ties to the even
+    code, finite magnitudes beyond 448 saturated, NaN to 0x7F."""
+    x = _cpu(torch.as_tensor(x, dtype=torch.float32))
+    out = torch.empty(x.shape, dtype=torch.uint8)
+    _load().oracle_e4m3_encode_array(_ptr(x), _ptr(out), x.numel())
+    return out
+
+
+def e4m3_decode(codes) -> torch.Tensor:
+    """Values (float64) of E4M3 codes."""
+    codes = _cpu(torch.as_tensor(codes, dtype=torch.uint8))
+    out = torch.empty(codes.shape, dtype=torch.float64)
+    _load().oracle_e4m3_decode_array(_ptr(codes), _ptr(out), codes.numel())
+    return out
+
+
+def reshape_and_cache_e4m3(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale) -> None:
+    """The append step into uint8 E4M3 caches: code of fp32(x) / scale[h]."""
+    key, value = _cpu(key), _cpu(value)
+    slot_mapping = _cpu(slot_mapping, torch.int64)
+    k_scale = _cpu(k_scale, torch.float32)
+    v_scale = _cpu(v_scale, torch.float32)
+    for c in (k_cache, v_cache):
+        if not c.is_contiguous() or c.device.type != "cpu" or c.dtype != torch.uint8:
+            raise ValueError("caches must be contiguous uint8 host tensors")
+    NB, H_kv, bs, D = k_cache.shape
+    T = slot_mapping.numel()
+    rc = _load().oracle_reshape_and_cache_e4m3(_ptr(key), _ptr(value), _dtype_code(key),
+                                               _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                               T, H_kv, D, bs, NB, _ptr(k_scale), _ptr(v_scale))
+    _check(rc, "reshape_and_cache_e4m3")
+
+
+def decode_e4m3(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                select=None):
+    """fp64 paged decode over uint8 E4M3 caches with per-K/V-head scales."""
+    q = _cpu(q)
+    k_cache, v_cache = _cpu(k_cache, torch.uint8), _cpu(v_cache, torch.uint8)
+    k_scale, v_scale = _cpu(k_scale, torch.float32), _cpu(v_scale, torch.float32)
+    block_tables = _cpu(block_tables, torch.int32)
+    context_lens = _cpu(context_lens, torch.int32)
+    B, H_q, D = q.shape
+    NB, H_kv, bs, _ = k_cache.shape
+    MB = block_tables.shape[1]
+    sel = _select(select, B * H_q)
+    out = torch.zeros(B, H_q, D, dtype=torch.float64)
+    lse = torch.full((B, H_q), float("-inf"), dtype=torch.float64)
+    rc = _load().oracle_decode_e4m3(_ptr(out), _ptr(lse), _ptr(q), _dtype_code(q), _ptr(k_cache),
+                                    _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                    _ptr(block_tables), _ptr(context_lens), B, H_q, H_kv, D, bs,
+                                    MB, NB, float(scale), _ptr(sel))
+    _check(rc, "decode_e4m3")
+    return out, lse
 

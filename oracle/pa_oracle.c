@@ -22,6 +22,10 @@
  *  [FD]  page "字节跳动 AI Infra (2)", question "推理加速的综合策略有哪些",
  *        table of algorithm-level optimisations, row FlashDecoding: decode is
  *        parallelised by splitting along the KV length.
+ *  [Q8]  page "字节跳动 AI Infra (2)", optimisation table, row "KV量化(INT8)"
+ *        (store K/V in low precision, halving the cache), and page
+ *        "LLM推理优化", section 1.3 (quantise K/V from FP16 to INT8/INT4):
+ *        here FP8 E4M3 codes with one scale per K/V head, value = code*scale.
  *  [CP]  page "vLLM框架是怎么做推理加速的", section 3 (Chunked Prefill): a
  *        prompt is cut into chunks (512 tokens by default) that attend over
  *        the cache; page "LLM推理优化", section 2.3: prefill attention is
@@ -54,18 +58,64 @@
 #include <omp.h>
 #endif
 
-enum { OR_F32 = 0, OR_BF16 = 1 };
+enum { OR_F32 = 0, OR_BF16 = 1, OR_E4M3 = 2 };
 enum { OR_OK = 0, OR_BAD_SLOT = 1, OR_BAD_BLOCK = 2, OR_BAD_ARG = 3, OR_NO_MEM = 4 };
 
+/* [Q8] value of an FP8 E4M3 code (1 sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits; exponent field 0 holds the subnormals m * 2^-9; no
+ * infinities; S.1111.111 is NaN; largest finite magnitude 448). */
+static double e4m3_value(uint8_t c)
+{
+    int e = (c >> 3) & 0xF, m = c & 7;
+    double v;
+    if ((c & 0x7F) == 0x7F) return NAN;
+    if (e == 0)
+        v = m * ldexp(1.0, -9);
+    else
+        v = (1.0 + m / 8.0) * ldexp(1.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* [Q8] code of the E4M3 value nearest to x, ties to the even code, finite
+ * magnitudes beyond 448 (and infinities) saturated to +-448, NaN to 0x7F.
+ * Written as a plain search over the 127 non-negative codes. */
+uint8_t oracle_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    int k = 0; /* largest code with value <= a */
+    while (k + 1 <= 0x7E && e4m3_value((uint8_t)(k + 1)) <= a) ++k;
+    double lo = e4m3_value((uint8_t)k), hi = e4m3_value((uint8_t)(k + 1));
+    int code;
+    if (a - lo < hi - a)
+        code = k;
+    else if (a - lo > hi - a)
+        code = k + 1;
+    else
+        code = (k % 2 == 0) ? k : k + 1;
+    return sign | (uint8_t)code;
+}
+
+double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
+
 /* A stored element, widened exactly to double. bf16 is the top half of an
- * IEEE binary32, so shifting its 16 bits up gives the same number as a float. */
-static double stored(const void *base, int64_t i, int dtype)
+ * IEEE binary32, so shifting its 16 bits up gives the same number as a float.
+ * An E4M3 code is its value times the K/V head's scale (exact in double). */
+static double stored_scaled(const void *base, int64_t i, int dtype, double scale)
 {
     if (dtype == OR_F32) return (double)((const float *)base)[i];
+    if (dtype == OR_E4M3) return e4m3_value(((const uint8_t *)base)[i]) * scale;
     uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
     return (double)f;
+}
+
+static double stored(const void *base, int64_t i, int dtype)
+{
+    return stored_scaled(base, i, dtype, 1.0);
 }
 
 /* One sequence's view of the pool: where its block table row is and which
@@ -78,6 +128,7 @@ typedef struct {
     int H_kv, D, bs;
     int64_t NB;
     int kv_head;
+    double k_scale, v_scale; /* E4M3 caches: value = code * scale */
 } paged_seq;
 
 /* [PG] element index of K/V[position j][dim 0] of this sequence and head:
@@ -111,7 +162,8 @@ static int attend(double *o, double *lse, const double *q, const paged_seq *s,
         int64_t base = token_base(s, j);
         if (base < 0) return OR_BAD_BLOCK;
         double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += q[d] * stored(s->k_cache, base + d, s->dtype);
+        for (int d = 0; d < D; ++d)
+            dot += q[d] * stored_scaled(s->k_cache, base + d, s->dtype, s->k_scale);
         double sc = scale * dot;
         sbuf[j - j0] = sc;
         if (sc > m) m = sc;
@@ -125,7 +177,8 @@ static int attend(double *o, double *lse, const double *q, const paged_seq *s,
     for (int64_t j = j0; j < j1; ++j) {
         int64_t base = token_base(s, j);
         double w = sbuf[j - j0] / denom;
-        for (int d = 0; d < D; ++d) o[d] += w * stored(s->v_cache, base + d, s->dtype);
+        for (int d = 0; d < D; ++d)
+            o[d] += w * stored_scaled(s->v_cache, base + d, s->dtype, s->v_scale);
     }
     *lse = m + log(denom);
     return OR_OK;
@@ -197,7 +250,7 @@ int oracle_decode(double *out, double *lse, const void *q, const void *k_cache,
         if (select && !select[bh]) continue;
         int b = (int)(bh / H_q), h = (int)(bh % H_q);
         paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)b * MB, MB,
-                       H_kv, D, bs, NB, h / group};
+                       H_kv, D, bs, NB, h / group, 1.0, 1.0};
         double *qv = malloc(sizeof(double) * D);
         double *sbuf = malloc(sizeof(double) * (context_lens[b] > 0 ? context_lens[b] : 1));
         if (!qv || !sbuf) {
@@ -238,7 +291,7 @@ int oracle_decode_partials(double *o_parts, double *lse_parts, const void *q, co
     for (int64_t bh = 0; bh < (int64_t)B * H_q; ++bh) {
         int b = (int)(bh / H_q), h = (int)(bh % H_q);
         paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)b * MB, MB,
-                       H_kv, D, bs, NB, h / group};
+                       H_kv, D, bs, NB, h / group, 1.0, 1.0};
         double *qv = malloc(sizeof(double) * D);
         double *sbuf = malloc(sizeof(double) * partition_tokens);
         if (!qv || !sbuf) {
@@ -324,7 +377,7 @@ int oracle_prefill(double *out, double *lse, const void *q, const void *k_cache,
         int64_t i = row - query_start_loc[c];
         int64_t pos = (int64_t)context_lens[c] - C + i; /* this query's position */
         paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)c * MB, MB,
-                       H_kv, D, bs, NB, h / group};
+                       H_kv, D, bs, NB, h / group, 1.0, 1.0};
         double *qv = malloc(sizeof(double) * D);
         double *sbuf = malloc(sizeof(double) * (pos + 1));
         if (!qv || !sbuf) {
@@ -367,4 +420,92 @@ int oracle_copy_blocks(const void *src_k, const void *src_v, int64_t src_blocks,
         memcpy((char *)dst_v + d, (const char *)src_v + s, block_bytes);
     }
     return OR_OK;
+}
+
+/* [Q8]+[KV] the append step into an E4M3 cache: each element of the new
+ * token's K (V) row for K/V head h is stored as the code of the fp32 quotient
+ * x / k_scale[h] (x / v_scale[h]), computed as an IEEE single-precision
+ * division and encoded by oracle_e4m3_encode. key/value are fp32 or bf16
+ * (dtype); caches hold one byte per element. Slots as in
+ * oracle_reshape_and_cache. */
+int oracle_reshape_and_cache_e4m3(const void *key, const void *value, int dtype, uint8_t *k_cache,
+                                  uint8_t *v_cache, const int64_t *slot_mapping,
+                                  int64_t num_tokens, int num_kv_heads, int head_dim,
+                                  int block_size, int64_t num_blocks, const float *k_scale,
+                                  const float *v_scale)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return OR_BAD_ARG;
+    for (int64_t t = 0; t < num_tokens; ++t)
+        if (slot_mapping[t] >= num_blocks * (int64_t)block_size) return OR_BAD_SLOT;
+    for (int64_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        int64_t block = slot / block_size, offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            int64_t src = ((int64_t)t * num_kv_heads + h) * head_dim;
+            int64_t dst = ((block * num_kv_heads + h) * block_size + offset) * head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                float xk = (float)stored(key, src + d, dtype);
+                float xv = (float)stored(value, src + d, dtype);
+                float qk = xk / k_scale[h];
+                float qv = xv / v_scale[h];
+                k_cache[dst + d] = oracle_e4m3_encode(qk);
+                v_cache[dst + d] = oracle_e4m3_encode(qv);
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* [KV]+[PG]+[GQA]+[Q8] decode over an E4M3 cache: as oracle_decode, with
+ * q of dtype q_dtype and every cached element equal to its code's value times
+ * the K/V head's scale (k_scale / v_scale, one per K/V head). */
+int oracle_decode_e4m3(double *out, double *lse, const void *q, int q_dtype, const uint8_t *k_cache,
+                       const uint8_t *v_cache, const float *k_scale, const float *v_scale,
+                       const int32_t *block_tables, const int32_t *context_lens, int B, int H_q,
+                       int H_kv, int D, int bs, int MB, int64_t NB, double scale,
+                       const uint8_t *select)
+{
+    int rc = check_heads(H_q, H_kv, D, bs, MB, NB);
+    if (rc) return rc;
+    for (int b = 0; b < B; ++b)
+        if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)MB * bs) return OR_BAD_ARG;
+    const int group = H_q / H_kv;
+    int err = OR_OK;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : err)
+    for (int64_t bh = 0; bh < (int64_t)B * H_q; ++bh) {
+        if (select && !select[bh]) continue;
+        int b = (int)(bh / H_q), h = (int)(bh % H_q);
+        int kvh = h / group;
+        paged_seq s = {k_cache, v_cache, OR_E4M3, block_tables + (int64_t)b * MB, MB,
+                       H_kv, D, bs, NB, kvh, (double)k_scale[kvh], (double)v_scale[kvh]};
+        double *qv = malloc(sizeof(double) * D);
+        double *sbuf = malloc(sizeof(double) * (context_lens[b] > 0 ? context_lens[b] : 1));
+        if (!qv || !sbuf) {
+            free(qv); free(sbuf);
+            err = OR_NO_MEM > err ? OR_NO_MEM : err;
+            continue;
+        }
+        for (int d = 0; d < D; ++d) qv[d] = stored(q, bh * D + d, q_dtype);
+        double l;
+        int r = attend(out + bh * D, &l, qv, &s, 0, context_lens[b], scale, sbuf);
+        if (lse) lse[bh] = l;
+        if (r > err) err = r;
+        free(qv);
+        free(sbuf);
+    }
+    return err;
+}
+
+
+/* [Q8] element-wise helpers over arrays (for tests and fixtures). */
+void oracle_e4m3_encode_array(const float *x, uint8_t *codes, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode(x[i]);
+}
+
+void oracle_e4m3_decode_array(const uint8_t *codes, double *x, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) x[i] = e4m3_value(codes[i]);
 }

@@ -281,25 +281,29 @@ def tiny_fp32(seed: int = 0) -> Batch:
                         scale=1.0 / 8.0, name="tiny_fp32_b4_d64")
 
 
-def llama7b_decode(seed: int = 0, num_blocks: int = 16384) -> Batch:
+def llama7b_decode(seed: int = 0, num_blocks: int = 16384, block_size: int = 16) -> Batch:
     """Llama-2-7B-shaped decode: 64 sequences with lengths uniform in
     [128, 2048], 32/32 heads, head_dim 128, 16-token blocks, 16384-block pool,
     bf16, N(0,1)."""
     gen = torch.Generator().manual_seed(seed + 7919)
     lens = torch.randint(128, 2049, (64,), generator=gen).tolist()
-    return decode_batch(lens, 32, 32, 128, 16, num_blocks, torch.bfloat16, 1.0, seed,
-                        max_blocks_per_seq=128, name="llama7b_decode_b64_h32_d128_bs16")
+    nb, mb = num_blocks * 16 // block_size, 2048 // block_size  # same pool bytes
+    return decode_batch(lens, 32, 32, 128, block_size, nb, torch.bfloat16, 1.0, seed,
+                        max_blocks_per_seq=mb,
+                        name=f"llama7b_decode_b64_h32_d128_bs{block_size}")
 
 
-def gqa_decode(seed: int = 0, num_blocks: int = 32768) -> Batch:
+def gqa_decode(seed: int = 0, num_blocks: int = 32768, block_size: int = 16) -> Batch:
     """GQA decode: 128 sequences, lengths log-normal with median 1024 and
     sigma 0.75 (natural-log scale) clipped to [16, 4096], 64 q / 8 kv heads,
     head_dim 128, 16-token blocks, 32768-block pool, bf16, N(0,1)."""
     gen = torch.Generator().manual_seed(seed + 104729)
     z = torch.randn(128, generator=gen, dtype=torch.float64)
     lens = torch.exp(math.log(1024.0) + 0.75 * z).round().clamp(16, 4096).to(torch.int64).tolist()
-    return decode_batch(lens, 64, 8, 128, 16, num_blocks, torch.bfloat16, 1.0, seed,
-                        max_blocks_per_seq=256, name="gqa_decode_b128_h64kv8_d128_bs16")
+    nb, mb = num_blocks * 16 // block_size, 4096 // block_size  # same pool bytes
+    return decode_batch(lens, 64, 8, 128, block_size, nb, torch.bfloat16, 1.0, seed,
+                        max_blocks_per_seq=mb,
+                        name=f"gqa_decode_b128_h64kv8_d128_bs{block_size}")
 
 
 def long_context_decode(seed: int = 0, num_blocks: int = 8192) -> Batch:

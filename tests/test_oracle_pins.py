@@ -478,3 +478,82 @@ def test_swap_round_trip_and_errors():
         oracle.copy_blocks(dev_k, dev_v, host_k, host_v, torch.tensor([[6, 0]]))
     with pytest.raises(ValueError):
         oracle.copy_blocks(dev_k, dev_v, host_k, host_v, torch.tensor([[0, 4]]))
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) KV cache
+# ---------------------------------------------------------------------------
+def test_e4m3_decode_matches_library_for_all_codes():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ours = oracle.e4m3_decode(codes)
+    lib = codes.view(torch.float8_e4m3fn).to(torch.float64)
+    nan = torch.isnan(lib)
+    assert torch.equal(torch.isnan(ours), nan) and int(nan.sum()) == 2  # 0x7F, 0xFF
+    assert torch.equal(ours[~nan], lib[~nan])
+    assert ours.abs()[~nan].max() == 448.0
+
+
+def test_e4m3_encode_matches_library_in_range():
+    """Every bf16 bit pattern whose magnitude is below 448 (exhaustive)
+    encodes to the same code as torch's float8_e4m3fn conversion (nearest,
+    ties to even); outside that range the oracle saturates instead."""
+    bits = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16)
+    x = bits.view(torch.bfloat16).to(torch.float32)
+    keep = torch.isfinite(x) & (x.abs() < 448)
+    x = x[keep]
+    ours = oracle.e4m3_encode(x)
+    lib = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(ours, lib)
+
+
+def test_e4m3_saturation_and_ties():
+    x = torch.tensor([448.0, 460.0, 1e6, float("inf"), -1e30, float("-inf"), float("nan"),
+                      1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, -0.0])
+    c = oracle.e4m3_encode(x).tolist()
+    assert c[:6] == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE]
+    assert c[6] == 0x7F
+    # halfway cases go to the even code
+    assert c[7:11] == [0x38, 0x3A, 0x00, 0x02]
+    assert c[11] == 0x80
+
+
+def test_e4m3_reshape_is_divide_then_encode():
+    g = torch.Generator().manual_seed(50)
+    key = (torch.randn(3, 2, 8, generator=g) * 3).to(torch.bfloat16)
+    value = (torch.randn(3, 2, 8, generator=g) * 3).to(torch.bfloat16)
+    ks, vs = torch.tensor([0.05, 0.3]), torch.tensor([0.02, 7.0])
+    kc = torch.zeros(4, 2, 16, 8, dtype=torch.uint8)
+    vc = torch.zeros_like(kc)
+    slots = torch.tensor([5, -1, 63])
+    oracle.reshape_and_cache_e4m3(key, value, kc, vc, slots, ks, vs)
+    for t, s in ((0, 5), (2, 63)):
+        for h in range(2):
+            want_k = oracle.e4m3_encode(key[t, h].float() / ks[h])
+            want_v = oracle.e4m3_encode(value[t, h].float() / vs[h])
+            assert torch.equal(kc[s // 16, h, s % 16], want_k)
+            assert torch.equal(vc[s // 16, h, s % 16], want_v)
+    untouched = torch.ones(4, 16, dtype=torch.bool)
+    untouched[0, 5] = untouched[3, 15] = False
+    assert torch.all(kc.permute(0, 2, 1, 3)[untouched] == 0)
+
+
+def test_e4m3_decode_equals_decode_of_dequantized_cache():
+    """With power-of-two scales code*scale is exact in fp32, so decode over
+    the E4M3 cache equals decode over the dequantized fp32 cache bit for bit
+    (and it is close to torch's attention on the same values)."""
+    ctxs, H_q, H_kv, D, bs = [7, 33, 50], 8, 2, 16, 16
+    g = torch.Generator().manual_seed(51)
+    NB = 12
+    kc = torch.randint(0, 256, (NB, H_kv, bs, D), generator=g, dtype=torch.int32).to(torch.uint8)
+    vc = torch.randint(0, 256, (NB, H_kv, bs, D), generator=g, dtype=torch.int32).to(torch.uint8)
+    kc[(kc & 0x7F) == 0x7F] = 0x38  # no NaN codes
+    vc[(vc & 0x7F) == 0x7F] = 0x30
+    ks, vs = torch.tensor([0.0625, 0.5]), torch.tensor([0.25, 2.0 ** -6])
+    tables = torch.tensor([[3, 0, 0, 0], [1, 7, 2, 0], [4, 5, 6, 11]], dtype=torch.int32)
+    lens = torch.tensor(ctxs, dtype=torch.int32)
+    q = torch.randn(3, H_q, D, generator=g).to(torch.bfloat16)
+    out, lse = oracle.decode_e4m3(q, kc, vc, ks, vs, tables, lens, 0.2)
+    kd = (oracle.e4m3_decode(kc) * ks.double()[None, :, None, None]).float()
+    vd = (oracle.e4m3_decode(vc) * vs.double()[None, :, None, None]).float()
+    ref, ref_lse = oracle.decode(q.float(), kd, vd, tables, lens, 0.2)
+    assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
