@@ -102,10 +102,11 @@ def decode_bytes(batch) -> float:
     if batch.q is None or batch.num_seqs == 0:
         return 0.0
     e = batch.k_cache.element_size()
+    eq = batch.q.element_size()
     ctx = batch.context_lens.to(torch.int64)
     H_kv, D, bs = batch.num_kv_heads, batch.head_dim, batch.block_size
     kv = int((2 * ctx * H_kv * D * e).sum())
-    qo = 2 * batch.num_seqs * batch.num_q_heads * D * e
+    qo = 2 * batch.num_seqs * batch.num_q_heads * D * eq
     tbl = int((4 * ((ctx + bs - 1) // bs) * H_kv).sum())
     return float(kv + qo + tbl + 4 * batch.num_seqs)
 
@@ -309,14 +310,24 @@ class Runner:
         """The step's C-ABI calls with their arguments marshalled once."""
         pa = self.pa
         d = d or self.d
-        c = {"reshape": pa.prepare_reshape_and_cache(d.key, d.value, d.k_cache, d.v_cache,
-                                                     d.slot_mapping)}
+        if d.k_scale is not None:
+            c = {"reshape": pa.prepare_reshape_and_cache_fp8(d.key, d.value, d.k_cache, d.v_cache,
+                                                             d.slot_mapping, d.k_scale,
+                                                             d.v_scale)}
+        else:
+            c = {"reshape": pa.prepare_reshape_and_cache(d.key, d.value, d.k_cache, d.v_cache,
+                                                         d.slot_mapping)}
         if d.prefill_q is not None:
             c["prefill"] = pa.prepare_prefill_chunk(
                 pout if pout is not None else self.pout, d.prefill_q, d.k_cache, d.v_cache,
                 d.prefill_block_tables, d.prefill_context_lens, d.query_start_loc, self.max_q,
                 d.scale)
-        if d.q is not None and d.num_seqs:
+        if d.q is not None and d.num_seqs and d.k_scale is not None:
+            c["decode"] = pa.prepare_decode_fp8(out if out is not None else self.out, d.q,
+                                                d.k_cache, d.v_cache, d.k_scale, d.v_scale,
+                                                d.block_tables, d.context_lens, self.max_ctx,
+                                                d.scale, self.part, self.ws)
+        elif d.q is not None and d.num_seqs:
             c["decode"] = pa.prepare_decode(out if out is not None else self.out, d.q, d.k_cache,
                                             d.v_cache, d.block_tables, d.context_lens,
                                             self.max_ctx, d.scale, self.part, self.ws)
@@ -488,7 +499,8 @@ def run_ours(args, rank, world):
             "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if batch.dtype.itemsize == 2 else "f32",
+            "dtype": ("e4m3 KV / bf16 q" if batch.fp8 else
+                      "bf16" if batch.dtype.itemsize == 2 else "f32"),
             "data": "synthetic (seeded; one batch per rank)",
             "config": workload_config(batch, args.workload, world, r),
             "tokens_per_s": round(tok_total / (ms * 1e-3), 1),
@@ -541,6 +553,12 @@ def workload_config(batch, name, world, r=None):
 # --------------------------------------------------------------------------
 def _oracle_step(batch, k, v, select=None, pselect=None):
     import oracle
+    if batch.fp8:
+        oracle.reshape_and_cache_e4m3(batch.key, batch.value, k, v, batch.slot_mapping,
+                                      batch.k_scale, batch.v_scale)
+        oracle.decode_e4m3(batch.q, k, v, batch.k_scale, batch.v_scale, batch.block_tables,
+                           batch.context_lens, batch.scale, select=select)
+        return
     oracle.reshape_and_cache(batch.key, batch.value, k, v, batch.slot_mapping)
     if batch.prefill_q is not None:
         oracle.prefill(batch.prefill_q, k, v, batch.prefill_block_tables,
@@ -641,7 +659,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="llama7b_decode",
                     choices=["tiny_fp32", "llama7b_decode", "gqa_decode", "long_context_decode",
-                             "mixed_prefill_decode"])
+                             "mixed_prefill_decode", "llama7b_decode_fp8", "gqa_decode_fp8"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--partition", type=int, default=None,

@@ -137,6 +137,34 @@ PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const 
                     int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
                     cudaStream_t stream);
 
+/* FP8 KV cache (E4M3 codes, one byte per element, one dequantisation scale
+ * per K/V head for K and one for V): page "字节跳动 AI Infra (2)", optimisation
+ * table, KV quantisation row, and page "LLM推理优化", section 1.3 (store K/V
+ * in low precision). Element value = code * scale[kv head].
+ *
+ * pa_reshape_and_cache_fp8: as pa_reshape_and_cache, with k_cache/v_cache
+ * uint8 [num_blocks][num_kv_heads][block_size][head_dim] and key/value of
+ * `dtype` (fp32 or bf16); each element is stored as the E4M3 code nearest to
+ * the IEEE fp32 quotient x / scale[h] (ties to even; magnitudes beyond 448
+ * saturate to +-448). k_scale/v_scale: device float [num_kv_heads]. */
+PA_API pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache,
+                                          void *v_cache, const int64_t *slot_mapping,
+                                          int num_tokens, int num_kv_heads, int head_dim,
+                                          int block_size, int num_blocks, const float *k_scale,
+                                          const float *v_scale, pa_dtype dtype,
+                                          cudaStream_t stream);
+
+/* pa_decode_fp8: as pa_decode over E4M3 caches (uint8, layout as above) with
+ * per-K/V-head scales; q and out are bf16; head_dim must be 128. The same
+ * workspace sizes apply (pa_decode_workspace_size). */
+PA_API pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                               const float *k_scale, const float *v_scale,
+                               const int32_t *block_tables, const int32_t *context_lens,
+                               int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int num_blocks, int max_blocks_per_seq,
+                               int max_context_len, float scale, int partition_size,
+                               void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* pa_decode without a caller-provided workspace. The pages have no
  * counterpart: this exists for callers that cannot allocate device memory at
  * the call site (a plugin handed only its input and output buffers, or a

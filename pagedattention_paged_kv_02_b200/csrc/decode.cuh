@@ -43,6 +43,8 @@ struct DecodeArgs {
     const int32_t *context_lens;
     float *part_o;    // [B][H_q][S_max][D] (split mode only)
     float *part_lse;  // [B][H_q][S_max], base-2 log-sum-exp of scaled scores
+    const float *k_scale;  // FP8 caches: per K/V head dequantisation scales
+    const float *v_scale;
     int num_seqs, H_q, H_kv, group, bs, NB, MB, max_ctx, P, S_max, n_htiles;
     float scale_log2;  // scale * log2(e): scores are kept in the base-2 domain
     unsigned long long timeout_ns;
@@ -77,7 +79,8 @@ struct DecodeSmem {
 template <int D, int NW, int HT, typename OutT>
 __device__ __forceinline__ void decode_epilogue(const DecodeArgs &a, const float *red_o,
                                                 const float *red_m, const float *red_l, int b,
-                                                int h0, int nh, int s, int n_splits) {
+                                                int h0, int nh, int s, int n_splits,
+                                                float oscale = 1.f) {
     constexpr int OS = D + 4;  // padded row stride of red_o
     for (int idx = threadIdx.x; idx < nh * (D / 2); idx += NW * 32) {
         const int row = idx / (D / 2);
@@ -95,7 +98,7 @@ __device__ __forceinline__ void decode_epilogue(const DecodeArgs &a, const float
                 o1 += f * red_o[(w * HT + row) * OS + d + 1];
             }
         }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float inv = L > 0.f ? oscale / L : 0.f;
         const size_t bh = (size_t)b * a.H_q + h0 + row;
         if (n_splits <= 1) {
             if constexpr (sizeof(OutT) == 2) {

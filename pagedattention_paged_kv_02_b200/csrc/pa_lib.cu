@@ -18,6 +18,7 @@
 #include "pa_device.cuh"
 #include "reshape_and_cache.cuh"
 #include "decode.cuh"
+#include "decode_fp8.cuh"
 #include "prefill.cuh"
 #include "blocks.cuh"
 
@@ -82,7 +83,7 @@ int partition_tokens(int max_ctx, int partition_size) {
     }
     const int whole = ((max_ctx > 0 ? max_ctx : 1) + kChunk - 1) / kChunk * kChunk;
     if (partition_size < 0) return whole <= kMaxPartition ? whole : -1;
-    return max_ctx <= 1024 ? whole : 512;  // automatic
+    return max_ctx <= 1024 ? whole : 1024;  // automatic
 }
 
 size_t workspace_bytes(int B, int H_q, int D, int max_ctx, int P) {
@@ -175,6 +176,32 @@ pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const C
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return PA_ERR_CUDA;
     if ((long long)fa.numRegs * kPfThreads < kPfRegsNeeded) return PA_ERR_UNSUPPORTED;
     k<<<grid, kPfThreads, smem, st>>>(a, mq, mk, mv);
+    return launch_status();
+}
+
+// A 4-D view [num_blocks][H_kv][bs][128] of a one-byte (E4M3) cache with a
+// box of 16 tokens x 128 dims (128 bytes) and 128-byte swizzle.
+bool encode_cache_map_u8(CUtensorMap *m, const void *cache, int NB, int H_kv, int bs) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {128, (cuuint64_t)bs, (cuuint64_t)H_kv, (cuuint64_t)NB};
+    cuuint64_t strides[3] = {128, (cuuint64_t)bs * 128, (cuuint64_t)H_kv * bs * 128};
+    cuuint32_t box[4] = {128, (cuuint32_t)kChunk, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(cache), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NW, int NS>
+pa_status launch_decode_e4m3(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
+                             dim3 grid, cudaStream_t st) {
+    constexpr int STAGE = 2 * kChunk * 128;
+    using L = DecodeSmem<NW, NS, STAGE, kHeadsBf16, 128>;
+    const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
+    auto k = decode_split_e4m3<NW, NS>;
+    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
+    k<<<grid, NW * 32, smem, st>>>(a, mk, mv);
     return launch_status();
 }
 
@@ -330,6 +357,118 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                 decode_reduce<64, float><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
             st = launch_status();
         }
+    }
+    return st;
+}
+
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache,
+                                   void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                                   int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                   const float *k_scale, const float *v_scale, pa_dtype dtype,
+                                   cudaStream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (!head_dim_ok(head_dim) || !block_size_ok(block_size)) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping || !k_scale || !v_scale)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(slot_mapping, 8) || !aligned(k_scale, 4) ||
+        !aligned(v_scale, 4))
+        return PA_ERR_INVALID_ARG;
+    ReshapeFp8Args a;
+    a.key = key;
+    a.value = value;
+    a.k_cache = static_cast<uint4 *>(k_cache);
+    a.v_cache = static_cast<uint4 *>(v_cache);
+    a.slot_mapping = slot_mapping;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.vecs_per_row = head_dim / 16;
+    a.vecs_per_token = num_kv_heads * a.vecs_per_row;
+    a.total_vecs = (long long)num_tokens * a.vecs_per_token;
+    a.num_kv_heads = num_kv_heads;
+    a.block_size = block_size;
+    a.num_slots = (long long)num_blocks * block_size;
+    a.bf16_in = dtype == PA_BF16;
+    const long long blocks = (a.total_vecs + 255) / 256;
+    if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    reshape_and_cache_e4m3_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    return launch_status();
+}
+
+pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const float *k_scale, const float *v_scale, const int32_t *block_tables,
+                        const int32_t *context_lens, int num_seqs, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        int max_blocks_per_seq, int max_context_len, float scale,
+                        int partition_size, void *workspace, size_t workspace_bytes_given,
+                        cudaStream_t stream) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0 || head_dim != 128 || !block_size_ok(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size)
+        return PA_ERR_INVALID_ARG;
+    const int P = partition_tokens(max_context_len, partition_size);
+    if (P <= 0) return partition_size > 0 ? PA_ERR_INVALID_ARG : PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !k_scale ||
+        !v_scale)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(k_scale, 4) ||
+        !aligned(v_scale, 4))
+        return PA_ERR_INVALID_ARG;
+    const size_t need = workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, P);
+    if (need > 0 && (!workspace || workspace_bytes_given < need || !aligned(workspace, 256)))
+        return PA_ERR_WORKSPACE;
+    const int group = num_q_heads / num_kv_heads;
+    const int n_htiles = (group + kHeadsBf16 - 1) / kHeadsBf16;
+    const long long S = (max_context_len + P - 1) / P;
+    const long long gy = (long long)num_kv_heads * n_htiles;
+    if (gy > 65535 || num_seqs > 65535 || S > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    DecodeArgs a;
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    const long long S1 = S > 0 ? S : 1;
+    a.part_o = need ? static_cast<float *>(workspace) : nullptr;
+    a.part_lse = need ? reinterpret_cast<float *>(
+                            static_cast<char *>(workspace) +
+                            ((size_t)num_seqs * num_q_heads * S1 * head_dim * 4 + 255) / 256 * 256)
+                      : nullptr;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.num_seqs = num_seqs;
+    a.H_q = num_q_heads;
+    a.H_kv = num_kv_heads;
+    a.group = group;
+    a.bs = block_size;
+    a.NB = num_blocks;
+    a.MB = max_blocks_per_seq;
+    a.max_ctx = max_context_len;
+    a.P = P;
+    a.S_max = (int)S1;
+    a.n_htiles = n_htiles;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.timeout_ns = kWaitTimeoutNs;
+    CUtensorMap mk, mv;
+    if (!encode_cache_map_u8(&mk, k_cache, num_blocks, num_kv_heads, block_size) ||
+        !encode_cache_map_u8(&mv, v_cache, num_blocks, num_kv_heads, block_size))
+        return PA_ERR_CUDA;
+    const dim3 grid((unsigned)S1, (unsigned)gy, (unsigned)num_seqs);
+    pa_status st = launch_decode_e4m3<4, 4>(a, mk, mv, grid, stream);
+    if (st != PA_OK) return st;
+    if (S1 > 1) {
+        decode_reduce<128, __nv_bfloat16><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
+        st = launch_status();
     }
     return st;
 }

@@ -69,6 +69,8 @@ class Batch:
     prefill_context_lens: Optional[torch.Tensor] = None
     query_start_loc: Optional[torch.Tensor] = None
     partition_size: int = 0
+    k_scale: Optional[torch.Tensor] = None  # FP8 pools: float32 [H_kv] per-head scales
+    v_scale: Optional[torch.Tensor] = None
 
     @property
     def num_blocks(self) -> int:
@@ -89,7 +91,13 @@ class Batch:
 
     @property
     def dtype(self) -> torch.dtype:
-        return self.k_cache.dtype
+        """Element type of q, out and the new K/V rows."""
+        t = self.q if self.q is not None else self.prefill_q
+        return t.dtype
+
+    @property
+    def fp8(self) -> bool:
+        return self.k_cache.dtype == torch.uint8
 
     @property
     def num_seqs(self) -> int:
@@ -329,10 +337,43 @@ def mixed_prefill_decode(seed: int = 0, num_blocks: int = 16384) -> Batch:
                        1.0, seed, name="mixed_prefill8x512_decode192_h32kv8_d128_bs16")
 
 
+def to_fp8(batch: Batch, k_amax: float = 4.0, v_amax: float = 4.0) -> Batch:
+    """A copy of a decode batch whose pool holds FP8 E4M3 codes: each cached
+    value divided by its K/V head's scale (amax / 448, one per head for K
+    and one for V) and cast with torch's float8_e4m3fn conversion after
+    clamping to the E4M3 range. NaN poison stays NaN (code 0x7F). q and the
+    step's new K/V rows keep their type (the append quantises them)."""
+    H = batch.num_kv_heads
+    ks = torch.full((H,), k_amax / 448.0, dtype=torch.float32)
+    vs = torch.full((H,), v_amax / 448.0, dtype=torch.float32)
+
+    def enc(pool, sc):
+        x = pool.float() / sc[None, :, None, None]
+        x = torch.where(torch.isnan(x), x, x.clamp(-448.0, 448.0))
+        return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+    kw = dict(batch.__dict__)
+    kw.update(k_cache=enc(batch.k_cache, ks), v_cache=enc(batch.v_cache, vs), k_scale=ks,
+              v_scale=vs, name=batch.name + "_fp8")
+    return Batch(**kw)
+
+
+def llama7b_decode_fp8(seed: int = 0, num_blocks: int = 16384, block_size: int = 16) -> Batch:
+    """The Llama-2-7B-shaped decode batch with an FP8 E4M3 pool."""
+    return to_fp8(llama7b_decode(seed, num_blocks, block_size))
+
+
+def gqa_decode_fp8(seed: int = 0, num_blocks: int = 32768, block_size: int = 16) -> Batch:
+    """The GQA decode batch with an FP8 E4M3 pool."""
+    return to_fp8(gqa_decode(seed, num_blocks, block_size))
+
+
 WORKLOADS = {
     "tiny_fp32": tiny_fp32,
     "llama7b_decode": llama7b_decode,
     "gqa_decode": gqa_decode,
     "long_context_decode": long_context_decode,
     "mixed_prefill_decode": mixed_prefill_decode,
+    "llama7b_decode_fp8": llama7b_decode_fp8,
+    "gqa_decode_fp8": gqa_decode_fp8,
 }

@@ -70,9 +70,9 @@ def test_partition_and_workspace_arithmetic(L):
     # invalid explicit sizes
     assert pa.pa_decode_partition_tokens(1000, 24) == -1
     assert pa.pa_decode_partition_tokens(1000, 32768) == -1
-    # automatic: one partition for short contexts, 512 tokens otherwise
+    # automatic: one partition for short contexts, 1024 tokens otherwise
     assert pa.pa_decode_partition_tokens(40, 0) == 48
-    assert pa.pa_decode_partition_tokens(4096, 0) == 512
+    assert pa.pa_decode_partition_tokens(4096, 0) == 1024
 
 
 def _decode(L, **kw):
