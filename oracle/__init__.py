@@ -25,6 +25,8 @@ Sources, by page title and section:
   page "LLM推理优化", section 1.3 (quantised KV cache): FP8 E4M3 codes with a
   scale per K/V head (:func:`e4m3_encode`, :func:`reshape_and_cache_e4m3`,
   :func:`decode_e4m3`).
+* page "LLM推理优化", section 2.3 (window_size) and page "vLLM框架是怎么做推理加速的",
+  追问 3 (sliding window attention): :func:`decode_window`.
 * page "vLLM框架是怎么做推理加速的", section 3: chunked prefill; page
   "LLM推理优化", section 2.3: causal attention (:func:`prefill`).
 
@@ -79,6 +81,8 @@ def _load():
             lib.oracle_lse_merge.restype = None
             lib.oracle_prefill.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, I, I64, D, P]
             lib.oracle_copy_blocks.argtypes = [P, P, I64, P, P, I64, P, I64, I64]
+            lib.oracle_decode_window.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I64,
+                                                 D, I, P]
             lib.oracle_e4m3_encode_array.argtypes = [P, P, I64]
             lib.oracle_e4m3_encode_array.restype = None
             lib.oracle_e4m3_decode_array.argtypes = [P, P, I64]
@@ -89,7 +93,7 @@ def _load():
                                                I64, D, P]
             for f in ("oracle_reshape_and_cache", "oracle_decode", "oracle_decode_partials",
                       "oracle_prefill", "oracle_copy_blocks", "oracle_reshape_and_cache_e4m3",
-                      "oracle_decode_e4m3"):
+                      "oracle_decode_e4m3", "oracle_decode_window"):
                 getattr(lib, f).restype = I
             _lib = lib
     return _lib
@@ -326,5 +330,24 @@ def decode_e4m3(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_len
                                     _ptr(block_tables), _ptr(context_lens), B, H_q, H_kv, D, bs,
                                     MB, NB, float(scale), _ptr(sel))
     _check(rc, "decode_e4m3")
+    return out, lse
+
+
+def decode_window(q, k_cache, v_cache, block_tables, context_lens, scale, window, select=None):
+    """fp64 paged decode attending only the last ``window`` positions."""
+    q, k_cache, v_cache = _cpu(q), _cpu(k_cache), _cpu(v_cache)
+    block_tables = _cpu(block_tables, torch.int32)
+    context_lens = _cpu(context_lens, torch.int32)
+    B, H_q, D = q.shape
+    NB, H_kv, bs, _ = k_cache.shape
+    MB = block_tables.shape[1]
+    sel = _select(select, B * H_q)
+    out = torch.zeros(B, H_q, D, dtype=torch.float64)
+    lse = torch.full((B, H_q), float("-inf"), dtype=torch.float64)
+    rc = _load().oracle_decode_window(_ptr(out), _ptr(lse), _ptr(q), _ptr(k_cache),
+                                      _ptr(v_cache), _dtype_code(q), _ptr(block_tables),
+                                      _ptr(context_lens), B, H_q, H_kv, D, bs, MB, NB,
+                                      float(scale), int(window), _ptr(sel))
+    _check(rc, "decode_window")
     return out, lse
 

@@ -26,6 +26,9 @@
  *        (store K/V in low precision, halving the cache), and page
  *        "LLM推理优化", section 1.3 (quantise K/V from FP16 to INT8/INT4):
  *        here FP8 E4M3 codes with one scale per K/V head, value = code*scale.
+ *  [SW]  page "LLM推理优化", section 2.3 (flash_attn_func window_size) and page
+ *        "vLLM框架是怎么做推理加速的", 追问 3 (sliding window attention): a query
+ *        sees only the last `window` positions up to its own.
  *  [CP]  page "vLLM框架是怎么做推理加速的", section 3 (Chunked Prefill): a
  *        prompt is cut into chunks (512 tokens by default) that attend over
  *        the cache; page "LLM推理优化", section 2.3: prefill attention is
@@ -509,3 +512,44 @@ void oracle_e4m3_decode_array(const uint8_t *codes, double *x, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i) x[i] = e4m3_value(codes[i]);
 }
+
+/* [SW]+[KV]+[PG] decode with a sliding window: as oracle_decode, each query
+ * attending positions [max(0, ctx - window), ctx) only (window > 0). */
+int oracle_decode_window(double *out, double *lse, const void *q, const void *k_cache,
+                         const void *v_cache, int dtype, const int32_t *block_tables,
+                         const int32_t *context_lens, int B, int H_q, int H_kv, int D, int bs,
+                         int MB, int64_t NB, double scale, int window, const uint8_t *select)
+{
+    int rc = check_heads(H_q, H_kv, D, bs, MB, NB);
+    if (rc) return rc;
+    if (window <= 0) return OR_BAD_ARG;
+    for (int b = 0; b < B; ++b)
+        if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)MB * bs) return OR_BAD_ARG;
+    const int group = H_q / H_kv;
+    int err = OR_OK;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : err)
+    for (int64_t bh = 0; bh < (int64_t)B * H_q; ++bh) {
+        if (select && !select[bh]) continue;
+        int b = (int)(bh / H_q), h = (int)(bh % H_q);
+        paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)b * MB, MB,
+                       H_kv, D, bs, NB, h / group, 1.0, 1.0};
+        int64_t j1 = context_lens[b];
+        int64_t j0 = j1 - window > 0 ? j1 - window : 0;
+        double *qv = malloc(sizeof(double) * D);
+        double *sbuf = malloc(sizeof(double) * (j1 - j0 > 0 ? j1 - j0 : 1));
+        if (!qv || !sbuf) {
+            free(qv); free(sbuf);
+            err = OR_NO_MEM > err ? OR_NO_MEM : err;
+            continue;
+        }
+        for (int d = 0; d < D; ++d) qv[d] = stored(q, bh * D + d, dtype);
+        double l;
+        int r = attend(out + bh * D, &l, qv, &s, j0, j1, scale, sbuf);
+        if (lse) lse[bh] = l;
+        if (r > err) err = r;
+        free(qv);
+        free(sbuf);
+    }
+    return err;
+}
+

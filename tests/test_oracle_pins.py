@@ -557,3 +557,42 @@ def test_e4m3_decode_equals_decode_of_dequantized_cache():
     vd = (oracle.e4m3_decode(vc) * vs.double()[None, :, None, None]).float()
     ref, ref_lse = oracle.decode(q.float(), kd, vd, tables, lens, 0.2)
     assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+
+
+# ---------------------------------------------------------------------------
+# sliding window
+# ---------------------------------------------------------------------------
+def test_window_covering_everything_is_plain_decode():
+    q, ks, vs, kc, vc, tables, lens = random_paged([9, 30, 47], 4, 2, 8, 8, seed=70)
+    a = oracle.decode(q, kc, vc, tables, lens, 0.3)
+    b = oracle.decode_window(q, kc, vc, tables, lens, 0.3, 47)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_window_of_one_is_the_last_value():
+    q, ks, vs, kc, vc, tables, lens = random_paged([9, 30], 2, 2, 8, 8, seed=71)
+    out, _ = oracle.decode_window(q, kc, vc, tables, lens, 0.3, 1)
+    for b, c in enumerate([9, 30]):
+        assert torch.equal(out[b], vs[b][:, c - 1].double())
+
+
+def test_window_equals_decode_of_the_dropped_prefix():
+    """A window of W over ctx tokens equals plain decode of the sequence with
+    its first ctx - W tokens removed (here a whole number of blocks, so the
+    shortened table is the original minus its leading entries)."""
+    bs = 8
+    ctxs = [48, 37]
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, 4, 1, 8, bs, seed=72)
+    W = 24
+    out, lse = oracle.decode_window(q, kc, vc, tables, lens, 0.4, W)
+    for b, c in enumerate(ctxs):
+        drop = (c - W) // bs * bs
+        rest = c - drop
+        t = tables[b:b + 1, drop // bs:].contiguous()
+        ref, ref_lse = oracle.decode_window(q[b:b + 1], kc, vc, t,
+                                            torch.tensor([rest], dtype=torch.int32), 0.4, W)
+        plain, plain_lse = oracle.decode(q[b:b + 1], kc, vc, t,
+                                         torch.tensor([rest], dtype=torch.int32), 0.4)
+        if rest == W:
+            assert torch.equal(out[b], plain[0]) and torch.equal(lse[b], plain_lse[0])
+        assert torch.equal(out[b], ref[0])
