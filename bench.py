@@ -434,7 +434,7 @@ def run_ours(args, rank, world):
         bcalls.append(r.calls(d=dd, out=outs[-1], pout=pouts[-1]))
     d2h = out_hs[0].numel() * out_hs[0].element_size()
     comp = torch.cuda.current_stream()
-    cs = torch.cuda.Stream()
+    up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()  # uploads never queue behind downloads
     up_done = [torch.cuda.Event() for _ in range(2)]
     used = [torch.cuda.Event() for _ in range(2)]
     down_done = [torch.cuda.Event() for _ in range(2)]
@@ -443,18 +443,18 @@ def run_ours(args, rank, world):
 
     def e2e_step(i):
         k = i % 2
-        with torch.cuda.stream(cs):
-            cs.wait_event(used[k])          # buffer k's previous step is done with it
+        up_s.wait_event(used[k])          # buffer k's previous step is done with it
+        with torch.cuda.stream(up_s):
             d_flats[k].copy_(h_flat, non_blocking=True)
-            up_done[k].record(cs)
+        up_done[k].record(up_s)
         comp.wait_event(up_done[k])
-        comp.wait_event(down_done[k])       # its previous result has been read back
+        comp.wait_event(down_done[k])     # its previous result has been read back
         r.step(calls=bcalls[k])
         used[k].record(comp)
-        with torch.cuda.stream(cs):
-            cs.wait_event(used[k])
+        down_s.wait_event(used[k])
+        with torch.cuda.stream(down_s):
             out_hs[k].copy_(outs[k] if outs[k] is not None else pouts[k], non_blocking=True)
-            down_done[k].record(cs)
+        down_done[k].record(down_s)
 
     for i in range(max(3, args.warmup // 4)):
         e2e_step(i)
@@ -462,10 +462,12 @@ def run_ours(args, rank, world):
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(comp)
-    cs.wait_event(e0)
+    up_s.wait_event(e0)
+    down_s.wait_event(e0)
     for i in range(K):
         e2e_step(i)
-    comp.wait_stream(cs)
+    comp.wait_stream(up_s)
+    comp.wait_stream(down_s)
     e1.record(comp)
     torch.cuda.synchronize()
     barrier(world)
@@ -652,6 +654,55 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_block_copies(args, rank, world):
+    """Auxiliary workloads for the block-copy row: ``cow_copy`` copies 1024
+    whole blocks inside the Llama-7B-shaped pool (copy-on-write), ``swap_out``
+    moves 256 blocks to a pinned host pool. Bytes = read + write of K and V."""
+    import torch
+    from pagedattention_paged_kv_02_b200 import pa
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    H, bs, D, NB = 32, 16, 128, 4096
+    g = torch.Generator(device=dev).manual_seed(rank)
+    k = torch.randn(NB, H, bs, D, device=dev, generator=g).to(torch.bfloat16)
+    v = torch.randn(NB, H, bs, D, device=dev, generator=g).to(torch.bfloat16)
+    perm = torch.randperm(NB, generator=torch.Generator().manual_seed(rank))
+    if args.workload == "cow_copy":
+        n = 1024
+        mapping = torch.stack([perm[:n], perm[n:2 * n]], 1).contiguous().to(dev)
+        call = lambda: pa.pa_copy_blocks(k, v, mapping)
+        where = "device pool -> same pool"
+    else:
+        n = 256
+        hk = torch.empty(n, H, bs, D, dtype=torch.bfloat16).pin_memory()
+        hv = torch.empty_like(hk).pin_memory()
+        mapping = torch.stack([perm[:n], torch.arange(n)], 1).contiguous().to(dev)
+        call = lambda: pa.pa_swap_blocks(k, v, hk, hv, mapping)
+        where = "device pool -> pinned host pool"
+    block_bytes = H * bs * D * 2
+    nbytes = 2 * 2 * n * block_bytes  # K and V, read and write
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        call()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.steps
+    hbm, _, _, basis = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {"metric": f"whole-block copy GB/s ({where}; read+write bytes)", "value": round(gbs, 1),
+            "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": args.workload, "pairs": n,
+                                            "block_bytes_per_cache": block_bytes},
+            "frac_of_hbm_peak": round(gbs / hbm, 4) if args.workload == "cow_copy" else None,
+            "peak_basis": f"{basis} hbm_gbs", "gpu_launches": args.steps}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -659,7 +710,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="llama7b_decode",
                     choices=["tiny_fp32", "llama7b_decode", "gqa_decode", "long_context_decode",
-                             "mixed_prefill_decode", "llama7b_decode_fp8", "gqa_decode_fp8"])
+                             "mixed_prefill_decode", "llama7b_decode_fp8", "gqa_decode_fp8",
+                             "cow_copy", "swap_out"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--partition", type=int, default=None,
@@ -680,6 +732,9 @@ def main(argv=None):
         run_reference(args, rank, world)
         return
     pin_device(local, world)
+    if args.workload in ("cow_copy", "swap_out"):
+        run_block_copies(args, rank, world)
+        return
     run_ours(args, rank, world)
 
 

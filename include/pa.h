@@ -190,6 +190,23 @@ PA_API pa_status pa_decode_static_workspace(void *out, const void *q, const void
                                             float scale, int partition_size, pa_dtype dtype,
                                             cudaStream_t stream);
 
+/* pa_decode restricted to a sliding window (page "LLM推理优化", section 2.3,
+ * flash_attn_func window_size; page "vLLM框架是怎么做推理加速的", 追问 3,
+ * sliding window attention): sequence b's query attends only positions
+ * [max(0, context_lens[b] - sliding_window), context_lens[b]). Table entries
+ * of blocks wholly before the window are never read (an engine may have
+ * freed them). sliding_window must be > 0; other arguments, workspace sizes
+ * and errors as for pa_decode. */
+PA_API pa_status pa_decode_sliding_window(void *out, const void *q, const void *k_cache,
+                                          const void *v_cache, const int32_t *block_tables,
+                                          const int32_t *context_lens, int num_seqs,
+                                          int num_q_heads, int num_kv_heads, int head_dim,
+                                          int block_size, int num_blocks,
+                                          int max_blocks_per_seq, int max_context_len,
+                                          float scale, int sliding_window, int partition_size,
+                                          void *workspace, size_t workspace_bytes,
+                                          pa_dtype dtype, cudaStream_t stream);
+
 /* Chunked prefill: chunk c has C_c = query_start_loc[c+1] - query_start_loc[c]
  * queries and context_lens[c] tokens in the cache (its own C_c tokens
  * included, already written by pa_reshape_and_cache). Query i of the chunk

@@ -46,9 +46,20 @@ struct DecodeArgs {
     const float *k_scale;  // FP8 caches: per K/V head dequantisation scales
     const float *v_scale;
     int num_seqs, H_q, H_kv, group, bs, NB, MB, max_ctx, P, S_max, n_htiles;
+    int window;        // > 0: attend only the last `window` positions
     float scale_log2;  // scale * log2(e): scores are kept in the base-2 domain
     unsigned long long timeout_ns;
 };
+
+// First attended position of a sequence of ctx tokens (the sliding window's
+// start, 0 without a window), and the 16-aligned position its partitions
+// count from.
+__device__ __forceinline__ int window_lo(const DecodeArgs &a, int ctx) {
+    return a.window > 0 && ctx > a.window ? ctx - a.window : 0;
+}
+__device__ __forceinline__ int span_base(const DecodeArgs &a, int ctx) {
+    return window_lo(a, ctx) & ~(kChunk - 1);
+}
 
 // Context length of sequence b as the kernels use it: clamped to what the
 // host bound and the table row allow (anything outside is recorded).
@@ -151,13 +162,14 @@ __global__ void __launch_bounds__(NW * 32)
     const int nh = min(HT, a.group - ht * HT);
 
     const int ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
-    const int n_splits = (ctx + a.P - 1) / a.P;
+    const int lo = window_lo(a, ctx), base = span_base(a, ctx);
+    const int n_splits = (ctx - base + a.P - 1) / a.P;
     if (s >= (n_splits > 0 ? n_splits : 1)) return;
     if (ctx == 0) {
         write_zero_rows<D, __nv_bfloat16>(a, b, h0, nh);
         return;
     }
-    const int tok0 = s * a.P;
+    const int tok0 = base + s * a.P;
     const int tok1 = min(tok0 + a.P, ctx);
     const int n_chunks = (tok1 - tok0 + kChunk - 1) / kChunk;
     const int lb0 = tok0 / a.bs;
@@ -243,14 +255,16 @@ __global__ void __launch_bounds__(NW * 32)
         const int id = tbl[t / a.bs - lb0];
         if (id >= 0) {
             const int valid = min(kChunk, tok1 - t);
+            const int first = max(0, lo - t);  // rows before the window start
             const uint32_t kb = stage0 + st * STAGE;
             const uint32_t vb = kb + HALF;
-            if (valid < kChunk) {
-                // rows past the context may hold anything (NaN, Inf): zero
-                // the V rows so that P = 0 cannot turn them into NaN
-                const int nvec = (kChunk - valid) * (D / 8);
+            if (valid < kChunk || first > 0) {
+                // rows outside [first, valid) may hold anything (NaN, Inf):
+                // zero those V rows so that P = 0 cannot turn them into NaN
+                const int nvec = kChunk * (D / 8);
                 for (int e = lane; e < nvec; e += 32) {
-                    const int r = valid + e / (D / 8);
+                    const int r = e / (D / 8);
+                    if (r >= first && r < valid) continue;
                     const int u = e % (D / 8);
                     const uint32_t addr = vb + (u / 8) * SUBTILE + r * 128 + (u % 8) * 16;
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
@@ -280,7 +294,7 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int tok = nt * 8 + 2 * tig + (e & 1);
-                    sc[nt][e] = tok < valid ? sc[nt][e] * a.scale_log2 : -INFINITY;
+                    sc[nt][e] = tok < valid && tok >= first ? sc[nt][e] * a.scale_log2 : -INFINITY;
                 }
             mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
             mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
@@ -300,12 +314,16 @@ __global__ void __launch_bounds__(NW * 32)
             // the denominator sums the same rounded weights the numerator uses
             l0 = l0 * c0 + (bf16_lo(pa[0]) + bf16_hi(pa[0]) + bf16_lo(pa[2]) + bf16_hi(pa[2]));
             l1 = l1 * c1 + (bf16_lo(pa[1]) + bf16_hi(pa[1]) + bf16_lo(pa[3]) + bf16_hi(pa[3]));
+            // the running max rarely moves once a few chunks are in: rescale
+            // the accumulators only when it did for some row of this warp
+            if (__any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {
 #pragma unroll
-            for (int dt = 0; dt < DTILES; ++dt) {
-                o[dt][0] *= c0;
-                o[dt][1] *= c0;
-                o[dt][2] *= c1;
-                o[dt][3] *= c1;
+                for (int dt = 0; dt < DTILES; ++dt) {
+                    o[dt][0] *= c0;
+                    o[dt][1] *= c0;
+                    o[dt][2] *= c1;
+                    o[dt][3] *= c1;
+                }
             }
             // O += P V  (V^T fragments via transposed ldmatrix)
             {
@@ -386,13 +404,14 @@ __global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constan
     const int nh = min(HT, a.group - ht * HT);
 
     const int ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
-    const int n_splits = (ctx + a.P - 1) / a.P;
+    const int lo = window_lo(a, ctx), base = span_base(a, ctx);
+    const int n_splits = (ctx - base + a.P - 1) / a.P;
     if (s >= (n_splits > 0 ? n_splits : 1)) return;
     if (ctx == 0) {
         write_zero_rows<D, float>(a, b, h0, nh);
         return;
     }
-    const int tok0 = s * a.P;
+    const int tok0 = base + s * a.P;
     const int tok1 = min(tok0 + a.P, ctx);
     const int n_chunks = (tok1 - tok0 + kChunk - 1) / kChunk;
     const int lb0 = tok0 / a.bs;
@@ -467,9 +486,10 @@ __global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constan
         const int id = tbl[t / a.bs - lb0];
         if (id >= 0) {
             const int valid = min(kChunk, tok1 - t);
+            const int first = max(0, lo - t);
             const float *ks = reinterpret_cast<const float *>(smem + warp * NS * STAGE + st * STAGE);
             const float *vs = ks + kChunk * D;
-            for (int j = 0; j < valid; ++j) {  // tokens past the context are never touched
+            for (int j = first; j < valid; ++j) {  // tokens outside the span are never touched
                 float kk[VEC], vv[VEC];
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) {
@@ -535,7 +555,7 @@ __global__ void __launch_bounds__(128) decode_reduce(const __grid_constant__ Dec
     const int bh = blockIdx.x;
     const int b = bh / a.H_q;
     const int ctx = clamped_ctx(a, b, false);
-    const int n = (ctx + a.P - 1) / a.P;
+    const int n = (ctx - span_base(a, ctx) + a.P - 1) / a.P;
     if (n <= 1) return;
     const float *lse = a.part_lse + (size_t)bh * a.S_max;
     const float *po = a.part_o + (size_t)bh * a.S_max * D;

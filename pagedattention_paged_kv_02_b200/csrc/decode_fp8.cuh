@@ -62,13 +62,17 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
     return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
 }
 
-template <int NW, int NS>
+// CT: tokens per pipeline stage (16 or 32). A 32-token stage is two
+// 16-token page pieces (each inside one physical block, so each has its own
+// table lookup); it halves the softmax and hand-off work per byte.
+template <int NW, int NS, int CT>
 __global__ void __launch_bounds__(NW * 32)
     decode_split_e4m3(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
     constexpr int D = 128;
     constexpr int HT = kHeadsBf16;
-    constexpr int HALF = kChunk * D;  // bytes of one K (or V) chunk
+    constexpr int PIECES = CT / kChunk;
+    constexpr int HALF = CT * D;  // bytes of one K (or V) stage
     constexpr int STAGE = 2 * HALF;
     using L = DecodeSmem<NW, NS, STAGE, HT, D>;
 
@@ -86,15 +90,16 @@ __global__ void __launch_bounds__(NW * 32)
     const int nh = min(HT, a.group - ht * HT);
 
     const int ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
-    const int n_splits = (ctx + a.P - 1) / a.P;
+    const int lo = window_lo(a, ctx), base = span_base(a, ctx);
+    const int n_splits = (ctx - base + a.P - 1) / a.P;
     if (s >= (n_splits > 0 ? n_splits : 1)) return;
     if (ctx == 0) {
         write_zero_rows<D, __nv_bfloat16>(a, b, h0, nh);
         return;
     }
-    const int tok0 = s * a.P;
+    const int tok0 = base + s * a.P;
     const int tok1 = min(tok0 + a.P, ctx);
-    const int n_chunks = (tok1 - tok0 + kChunk - 1) / kChunk;
+    const int n_chunks = (tok1 - tok0 + CT - 1) / CT;
     const int lb0 = tok0 / a.bs;
     const int n_tbl = (tok1 - 1) / a.bs - lb0 + 1;
 
@@ -120,17 +125,28 @@ __global__ void __launch_bounds__(NW * 32)
     auto issue = [&](int i) {
         const int st = i % NS;
         const uint32_t bar = bar0 + st * 8;
-        const int t = tok0 + (warp + i * NW) * kChunk;
-        const int id = tbl[t / a.bs - lb0];
-        if (id < 0) {
+        const int t = tok0 + (warp + i * NW) * CT;
+        int ids[PIECES];
+        int n = 0;
+#pragma unroll
+        for (int p = 0; p < PIECES; ++p) {
+            const int tp = t + p * kChunk;
+            ids[p] = tp < tok1 ? tbl[tp / a.bs - lb0] : -1;
+            n += ids[p] >= 0;
+        }
+        if (n == 0) {
             mbar_arrive(bar);
             return;
         }
-        mbar_arrive_expect_tx(bar, STAGE);
+        mbar_arrive_expect_tx(bar, n * 2 * kChunk * D);
         const uint32_t kdst = stage0 + st * STAGE;
-        const int off = t % a.bs;
-        tma_load_4d(kdst, &tmk, bar, 0, off, kvh, id);
-        tma_load_4d(kdst + HALF, &tmv, bar, 0, off, kvh, id);
+#pragma unroll
+        for (int p = 0; p < PIECES; ++p) {
+            if (ids[p] < 0) continue;
+            const int off = (t + p * kChunk) % a.bs;
+            tma_load_4d(kdst + p * kChunk * D, &tmk, bar, 0, off, kvh, ids[p]);
+            tma_load_4d(kdst + HALF + p * kChunk * D, &tmv, bar, 0, off, kvh, ids[p]);
+        }
     };
     if (lane == 0) {
         for (int i = 0; i < NS && i < my_n; ++i) issue(i);
@@ -176,96 +192,129 @@ __global__ void __launch_bounds__(NW * 32)
             break;
         }
         done = i + 1;
-        const int t = tok0 + (warp + i * NW) * kChunk;
-        const int id = tbl[t / a.bs - lb0];
-        if (id >= 0) {
-            const int valid = min(kChunk, tok1 - t);
+        const int t = tok0 + (warp + i * NW) * CT;
+        // pieces that were loaded (inside the span, valid table entry)
+        int pok = 0;
+#pragma unroll
+        for (int p = 0; p < PIECES; ++p)
+            if (t + p * kChunk < tok1 && tbl[(t + p * kChunk) / a.bs - lb0] >= 0) pok |= 1 << p;
+        if (pok) {
+            const int valid = min(CT, tok1 - t);
+            const int first = max(0, lo - t);  // rows before the window start
             const uint32_t kb = stage0 + st * STAGE;
             const uint32_t vb = kb + HALF;
-            if (valid < kChunk) {
-                // rows past the context may hold anything: zero those V rows
-                const int nvec = (kChunk - valid) * 8;
-                for (int e = lane; e < nvec; e += 32) {
-                    const uint32_t addr = vb + (valid + e / 8) * 128 + (e % 8) * 16;
+            const bool full = valid == CT && first == 0 && pok == (1 << PIECES) - 1;
+            if (!full) {
+                // rows outside [first, valid) or in an unloaded piece may hold
+                // anything: zero those V rows so that P = 0 cannot meet a NaN
+                for (int e = lane; e < CT * 8; e += 32) {
+                    const int r = e / 8;
+                    if (r >= first && r < valid && ((pok >> (r / kChunk)) & 1)) continue;
+                    const uint32_t addr = vb + r * 128 + (e % 8) * 16;
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
                                  : "memory");
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            // S = Q K^T: matrices (tokens 0-7 | 8-15) x (16-dim units u, u+1)
-            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            // S = Q K^T per 16-token piece: matrices (tokens 0-7 | 8-15) x
+            // (16-dim units u, u+1)
+            float sc[2 * PIECES][4];
+#pragma unroll
+            for (int nt = 0; nt < 2 * PIECES; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
             {
                 const int mi = lane >> 3;
                 const int r = (mi & 1) * 8 + (lane & 7);
 #pragma unroll
-                for (int kp = 0; kp < 4; ++kp) {
-                    const int u = kp * 2 + (mi >> 1);
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4(kb + sw128(r, u), r0, r1, r2, r3);
-                    // r0: tokens 0-7, unit 2kp; r1: tokens 8-15, unit 2kp;
-                    // r2, r3: the same for unit 2kp+1
-                    mma_f16_16816(sc[0], qa[2 * kp], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r0 >> 16));
-                    mma_f16_16816(sc[1], qa[2 * kp], e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r1 >> 16));
-                    mma_f16_16816(sc[0], qa[2 * kp + 1], e4m3x2_to_f16x2(r2),
-                                  e4m3x2_to_f16x2(r2 >> 16));
-                    mma_f16_16816(sc[1], qa[2 * kp + 1], e4m3x2_to_f16x2(r3),
-                                  e4m3x2_to_f16x2(r3 >> 16));
-                }
-            }
+                for (int p = 0; p < PIECES; ++p)
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+                    for (int kp = 0; kp < 4; ++kp) {
+                        const int u = kp * 2 + (mi >> 1);
+                        uint32_t r0, r1, r2, r3;
+                        ldsm_x4(kb + p * kChunk * D + sw128(r, u), r0, r1, r2, r3);
+                        mma_f16_16816(sc[2 * p], qa[2 * kp], e4m3x2_to_f16x2(r0),
+                                      e4m3x2_to_f16x2(r0 >> 16));
+                        mma_f16_16816(sc[2 * p + 1], qa[2 * kp], e4m3x2_to_f16x2(r1),
+                                      e4m3x2_to_f16x2(r1 >> 16));
+                        mma_f16_16816(sc[2 * p], qa[2 * kp + 1], e4m3x2_to_f16x2(r2),
+                                      e4m3x2_to_f16x2(r2 >> 16));
+                        mma_f16_16816(sc[2 * p + 1], qa[2 * kp + 1], e4m3x2_to_f16x2(r3),
+                                      e4m3x2_to_f16x2(r3 >> 16));
+                    }
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2 * PIECES; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int tok = nt * 8 + 2 * tig + (e & 1);
-                    sc[nt][e] = tok < valid ? sc[nt][e] * sl2 : -INFINITY;
+                    const bool ok = tok < valid && tok >= first && ((pok >> (tok / kChunk)) & 1);
+                    sc[nt][e] = ok ? sc[nt][e] * sl2 : -INFINITY;
+                    if (e < 2)
+                        mx0 = fmaxf(mx0, sc[nt][e]);
+                    else
+                        mx1 = fmaxf(mx1, sc[nt][e]);
                 }
-            float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-            float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
             const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);
+            // a row with nothing visible yet keeps reference -inf: use 0 then
+            const float r0m = mn0 == -INFINITY ? 0.f : mn0, r1m = mn1 == -INFINITY ? 0.f : mn1;
+            const float c0 = exp2f(m0 - r0m), c1 = exp2f(m1 - r1m);
             m0 = mn0;
             m1 = mn1;
-            uint32_t pa[4];
-            pa[0] = pack_f16x2(exp2f(sc[0][0] - mn0), exp2f(sc[0][1] - mn0));
-            pa[1] = pack_f16x2(exp2f(sc[0][2] - mn1), exp2f(sc[0][3] - mn1));
-            pa[2] = pack_f16x2(exp2f(sc[1][0] - mn0), exp2f(sc[1][1] - mn0));
-            pa[3] = pack_f16x2(exp2f(sc[1][2] - mn1), exp2f(sc[1][3] - mn1));
-            l0 = l0 * c0 + (f16_lo(pa[0]) + f16_hi(pa[0]) + f16_lo(pa[2]) + f16_hi(pa[2]));
-            l1 = l1 * c1 + (f16_lo(pa[1]) + f16_hi(pa[1]) + f16_lo(pa[3]) + f16_hi(pa[3]));
+            uint32_t pa[PIECES][4];
+            float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-            for (int dt = 0; dt < 16; ++dt) {
-                o[dt][0] *= c0;
-                o[dt][1] *= c0;
-                o[dt][2] *= c1;
-                o[dt][3] *= c1;
+            for (int p = 0; p < PIECES; ++p) {
+                pa[p][0] = pack_f16x2(exp2f(sc[2 * p][0] - r0m), exp2f(sc[2 * p][1] - r0m));
+                pa[p][1] = pack_f16x2(exp2f(sc[2 * p][2] - r1m), exp2f(sc[2 * p][3] - r1m));
+                pa[p][2] = pack_f16x2(exp2f(sc[2 * p + 1][0] - r0m), exp2f(sc[2 * p + 1][1] - r0m));
+                pa[p][3] = pack_f16x2(exp2f(sc[2 * p + 1][2] - r1m), exp2f(sc[2 * p + 1][3] - r1m));
+                ps0 += f16_lo(pa[p][0]) + f16_hi(pa[p][0]) + f16_lo(pa[p][2]) + f16_hi(pa[p][2]);
+                ps1 += f16_lo(pa[p][1]) + f16_hi(pa[p][1]) + f16_lo(pa[p][3]) + f16_hi(pa[p][3]);
             }
-            // O += P V: matrices (tokens 0-7 | 8-15) x units (u, u+1), transposed
+            l0 = l0 * c0 + ps0;
+            l1 = l1 * c1 + ps1;
+            // the running max rarely moves once a few chunks are in: rescale
+            // the accumulators only when it did for some row of this warp
+            if (__any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {
+#pragma unroll
+                for (int dt = 0; dt < 16; ++dt) {
+                    o[dt][0] *= c0;
+                    o[dt][1] *= c0;
+                    o[dt][2] *= c1;
+                    o[dt][3] *= c1;
+                }
+            }
+            // O += P V per piece: matrices (tokens 0-7 | 8-15) x units (u,
+            // u+1), transposed; each register holds a token pair (2c, 2c+1)
+            // x a dim pair (2g, 2g+1) of its unit; a byte permute regroups
+            // it into (dim 2g: both tokens) and (dim 2g+1: both tokens)
             {
                 const int mi = lane >> 3;
                 const int r = (mi & 1) * 8 + (lane & 7);
 #pragma unroll
-                for (int up = 0; up < 4; ++up) {
-                    const int u = up * 2 + (mi >> 1);
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4_t(vb + sw128(r, u), r0, r1, r2, r3);
-                    // each register: token pair (2c, 2c+1) x dim pair (2g, 2g+1)
-                    // of its unit; regroup bytes into (dim 2g: both tokens) and
-                    // (dim 2g+1: both tokens)
-                    const uint32_t a0 = __byte_perm(r0, 0, 0x3120), a1 = __byte_perm(r1, 0, 0x3120);
-                    const uint32_t b0 = __byte_perm(r2, 0, 0x3120), b1 = __byte_perm(r3, 0, 0x3120);
-                    const int u0 = up * 2, u1 = up * 2 + 1;
-                    mma_f16_16816(o[2 * u0], pa, e4m3x2_to_f16x2(a0), e4m3x2_to_f16x2(a1));
-                    mma_f16_16816(o[2 * u0 + 1], pa, e4m3x2_to_f16x2(a0 >> 16),
-                                  e4m3x2_to_f16x2(a1 >> 16));
-                    mma_f16_16816(o[2 * u1], pa, e4m3x2_to_f16x2(b0), e4m3x2_to_f16x2(b1));
-                    mma_f16_16816(o[2 * u1 + 1], pa, e4m3x2_to_f16x2(b0 >> 16),
-                                  e4m3x2_to_f16x2(b1 >> 16));
-                }
+                for (int p = 0; p < PIECES; ++p)
+#pragma unroll
+                    for (int up = 0; up < 4; ++up) {
+                        const int u = up * 2 + (mi >> 1);
+                        uint32_t r0, r1, r2, r3;
+                        ldsm_x4_t(vb + p * kChunk * D + sw128(r, u), r0, r1, r2, r3);
+                        const uint32_t a0 = __byte_perm(r0, 0, 0x3120);
+                        const uint32_t a1 = __byte_perm(r1, 0, 0x3120);
+                        const uint32_t b0 = __byte_perm(r2, 0, 0x3120);
+                        const uint32_t b1 = __byte_perm(r3, 0, 0x3120);
+                        const int u0 = up * 2, u1 = up * 2 + 1;
+                        mma_f16_16816(o[2 * u0], pa[p], e4m3x2_to_f16x2(a0), e4m3x2_to_f16x2(a1));
+                        mma_f16_16816(o[2 * u0 + 1], pa[p], e4m3x2_to_f16x2(a0 >> 16),
+                                      e4m3x2_to_f16x2(a1 >> 16));
+                        mma_f16_16816(o[2 * u1], pa[p], e4m3x2_to_f16x2(b0), e4m3x2_to_f16x2(b1));
+                        mma_f16_16816(o[2 * u1 + 1], pa[p], e4m3x2_to_f16x2(b0 >> 16),
+                                      e4m3x2_to_f16x2(b1 >> 16));
+                    }
             }
         }
         __syncwarp();

@@ -118,6 +118,25 @@ Pipe decode_pipe() {
     return p;
 }
 
+// Launch shape of the FP8 split kernel: warps x stages x tokens per stage;
+// PA_DECODE_PIPE_FP8=<warps>x<stages>x<tokens> (built: 4x2x16, 4x4x16,
+// 4x2x32, 4x3x32, 2x4x32; default 4x2x32).
+struct PipeFp8 {
+    int nw, ns, ct;
+};
+
+PipeFp8 decode_pipe_fp8() {
+    static PipeFp8 p = [] {
+        PipeFp8 r{4, 2, 32};
+        if (const char *e = std::getenv("PA_DECODE_PIPE_FP8")) {
+            int w = 0, s = 0, c = 0;
+            if (sscanf(e, "%dx%dx%d", &w, &s, &c) == 3) r = PipeFp8{w, s, c};
+        }
+        return r;
+    }();
+    return p;
+}
+
 template <int D, int NW, int NS>
 pa_status launch_decode_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
                              dim3 grid, cudaStream_t st) {
@@ -193,13 +212,13 @@ bool encode_cache_map_u8(CUtensorMap *m, const void *cache, int NB, int H_kv, in
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NW, int NS>
+template <int NW, int NS, int CT>
 pa_status launch_decode_e4m3(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
                              dim3 grid, cudaStream_t st) {
-    constexpr int STAGE = 2 * kChunk * 128;
+    constexpr int STAGE = 2 * CT * 128;
     using L = DecodeSmem<NW, NS, STAGE, kHeadsBf16, 128>;
     const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
-    auto k = decode_split_e4m3<NW, NS>;
+    auto k = decode_split_e4m3<NW, NS, CT>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
     k<<<grid, NW * 32, smem, st>>>(a, mk, mv);
     return launch_status();
@@ -268,12 +287,15 @@ size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int head_dim, int
     return workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len, P);
 }
 
-pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
-                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
-                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                    int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
-                    int partition_size, void *workspace, size_t workspace_bytes_given,
-                    pa_dtype dtype, cudaStream_t stream) {
+}  // extern "C"
+
+static pa_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, const int32_t *context_lens,
+                             int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                             int block_size, int num_blocks, int max_blocks_per_seq,
+                             int max_context_len, float scale, int partition_size,
+                             void *workspace, size_t workspace_bytes_given, pa_dtype dtype,
+                             int window, cudaStream_t stream) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
         return PA_ERR_INVALID_ARG;
@@ -327,6 +349,8 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     a.n_htiles = n_htiles;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
+    a.window = window;
+    a.k_scale = a.v_scale = nullptr;
 
     const dim3 grid((unsigned)S1, (unsigned)gy, (unsigned)num_seqs);
     pa_status st;
@@ -359,6 +383,35 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
         }
     }
     return st;
+}
+
+extern "C" {
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                    int partition_size, void *workspace, size_t workspace_bytes_given,
+                    pa_dtype dtype, cudaStream_t stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       max_blocks_per_seq, max_context_len, scale, partition_size, workspace,
+                       workspace_bytes_given, dtype, 0, stream);
+}
+
+pa_status pa_decode_sliding_window(void *out, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *block_tables,
+                                   const int32_t *context_lens, int num_seqs, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int num_blocks, int max_blocks_per_seq, int max_context_len,
+                                   float scale, int sliding_window, int partition_size,
+                                   void *workspace, size_t workspace_bytes_given, pa_dtype dtype,
+                                   cudaStream_t stream) {
+    if (sliding_window <= 0) return PA_ERR_INVALID_ARG;
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       max_blocks_per_seq, max_context_len, scale, partition_size, workspace,
+                       workspace_bytes_given, dtype, sliding_window, stream);
 }
 
 pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache,
@@ -446,6 +499,7 @@ pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const voi
                       : nullptr;
     a.k_scale = k_scale;
     a.v_scale = v_scale;
+    a.window = 0;
     a.num_seqs = num_seqs;
     a.H_q = num_q_heads;
     a.H_kv = num_kv_heads;
@@ -464,7 +518,13 @@ pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const voi
         !encode_cache_map_u8(&mv, v_cache, num_blocks, num_kv_heads, block_size))
         return PA_ERR_CUDA;
     const dim3 grid((unsigned)S1, (unsigned)gy, (unsigned)num_seqs);
-    pa_status st = launch_decode_e4m3<4, 4>(a, mk, mv, grid, stream);
+    const PipeFp8 pp = decode_pipe_fp8();
+    pa_status st =
+        pp.nw == 4 && pp.ns == 2 && pp.ct == 16   ? launch_decode_e4m3<4, 2, 16>(a, mk, mv, grid, stream)
+        : pp.nw == 4 && pp.ns == 4 && pp.ct == 16 ? launch_decode_e4m3<4, 4, 16>(a, mk, mv, grid, stream)
+        : pp.nw == 4 && pp.ns == 3 && pp.ct == 32 ? launch_decode_e4m3<4, 3, 32>(a, mk, mv, grid, stream)
+        : pp.nw == 2 && pp.ns == 4 && pp.ct == 32 ? launch_decode_e4m3<2, 4, 32>(a, mk, mv, grid, stream)
+                                                  : launch_decode_e4m3<4, 2, 32>(a, mk, mv, grid, stream);
     if (st != PA_OK) return st;
     if (S1 > 1) {
         decode_reduce<128, __nv_bfloat16><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);

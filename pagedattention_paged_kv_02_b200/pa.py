@@ -26,7 +26,7 @@ EXPORTS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_partit
            "pa_decode", "pa_prefill_chunk", "pa_check_tables", "pa_device_error",
            "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
            "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
-           "pa_reshape_and_cache_fp8", "pa_decode_fp8")
+           "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window")
 
 
 class PAError(RuntimeError):
@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_static_workspace.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I,
                                                  I, P]
         L.pa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P]
+        L.pa_decode_sliding_window.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,
+                                               P, SZ, I, P]
         L.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, I, P]
         L.pa_decode_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, SZ,
                                     P]
@@ -68,7 +70,7 @@ def lib() -> ctypes.CDLL:
         L.pa_status_string.restype = ctypes.c_char_p
         for f in ("pa_reshape_and_cache", "pa_decode", "pa_decode_static_workspace",
                   "pa_prefill_chunk", "pa_check_tables", "pa_copy_blocks", "pa_swap_blocks",
-                  "pa_reshape_and_cache_fp8", "pa_decode_fp8",
+                  "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window",
                   "pa_device_error", "pa_selftest_bounded_wait", "pa_decode_partition_tokens",
                   "pa_version"):
             getattr(L, f).restype = I
@@ -158,6 +160,24 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
     _call("pa_decode", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
           _p(context_lens), B, H_q, H_kv, D, bs, NB, MB, int(max_context_len), float(scale),
           int(partition_size), _p(workspace), ws_bytes, _dt(q), _stream(stream))
+
+
+def pa_decode_sliding_window(out, q, k_cache, v_cache, block_tables, context_lens,
+                             max_context_len: int, scale: float, sliding_window: int,
+                             partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                             stream=None) -> None:
+    """pa_decode attending only the last ``sliding_window`` positions."""
+    _check_int(block_tables, torch.int32, "block_tables")
+    _check_int(context_lens, torch.int32, "context_lens")
+    B, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
+        raise ValueError("out must match q; caches must share head_dim")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _call("pa_decode_sliding_window", _p(out), _p(q), _p(k_cache), _p(v_cache),
+          _p(block_tables), _p(context_lens), B, H_q, H_kv, D, bs, NB, block_tables.shape[1],
+          int(max_context_len), float(scale), int(sliding_window), int(partition_size),
+          _p(workspace), ws_bytes, _dt(q), _stream(stream))
 
 
 def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_lens,
