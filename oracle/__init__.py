@@ -80,6 +80,8 @@ def _load():
             lib.oracle_lse_merge.argtypes = [P, P, P, P, I64, I, I]
             lib.oracle_lse_merge.restype = None
             lib.oracle_prefill.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, I, I64, D, P]
+            lib.oracle_prefill_window.argtypes = [P, P, P, P, P, I, P, P, P, I, I, I, I, I, I,
+                                                  I64, D, I, P]
             lib.oracle_copy_blocks.argtypes = [P, P, I64, P, P, I64, P, I64, I64]
             lib.oracle_decode_window.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I64,
                                                  D, I, P]
@@ -93,7 +95,7 @@ def _load():
                                                I64, D, P]
             for f in ("oracle_reshape_and_cache", "oracle_decode", "oracle_decode_partials",
                       "oracle_prefill", "oracle_copy_blocks", "oracle_reshape_and_cache_e4m3",
-                      "oracle_decode_e4m3", "oracle_decode_window"):
+                      "oracle_decode_e4m3", "oracle_decode_window", "oracle_prefill_window"):
                 getattr(lib, f).restype = I
             _lib = lib
     return _lib
@@ -255,6 +257,31 @@ def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, sc
                                 _dtype_code(q), _ptr(block_tables), _ptr(context_lens), _ptr(qsl),
                                 n_chunks, H_q, H_kv, D, bs, MB, NB, float(scale), _ptr(sel))
     _check(rc, "prefill")
+    return out, lse
+
+
+def prefill_window(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
+                   window, select=None):
+    """fp64 chunked prefill with a sliding window: query i of chunk c, at
+    position pos = ctx - C + i, attends positions [max(0, pos - window + 1),
+    pos] only. Shapes as ``prefill``."""
+    q, k_cache, v_cache = _cpu(q), _cpu(k_cache), _cpu(v_cache)
+    block_tables = _cpu(block_tables, torch.int32)
+    context_lens = _cpu(context_lens, torch.int32)
+    qsl = _cpu(query_start_loc, torch.int32)
+    total_q, H_q, D = q.shape
+    NB, H_kv, bs, _ = k_cache.shape
+    n_chunks = qsl.numel() - 1
+    MB = block_tables.shape[1]
+    assert int(qsl[-1]) == total_q
+    sel = _select(select, total_q * H_q)
+    out = torch.zeros(total_q, H_q, D, dtype=torch.float64)
+    lse = torch.full((total_q, H_q), float("-inf"), dtype=torch.float64)
+    rc = _load().oracle_prefill_window(_ptr(out), _ptr(lse), _ptr(q), _ptr(k_cache),
+                                       _ptr(v_cache), _dtype_code(q), _ptr(block_tables),
+                                       _ptr(context_lens), _ptr(qsl), n_chunks, H_q, H_kv, D, bs,
+                                       MB, NB, float(scale), int(window), _ptr(sel))
+    _check(rc, "prefill_window")
     return out, lse
 
 

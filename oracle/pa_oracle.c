@@ -352,15 +352,15 @@ void oracle_lse_merge(double *out, double *lse, const double *o_parts, const dou
  * Query i attends positions [0, ctx - C + i] (causal, bottom-right aligned).
  * out: [total_q][H_q][D]; lse: [total_q][H_q] (may be NULL); select as in
  * oracle_decode over (row, head). */
-int oracle_prefill(double *out, double *lse, const void *q, const void *k_cache,
-                   const void *v_cache, int dtype, const int32_t *block_tables,
-                   const int32_t *context_lens, const int32_t *query_start_loc, int n_chunks,
-                   int H_q, int H_kv, int D, int bs, int MB, int64_t NB, double scale,
-                   const uint8_t *select)
+static int prefill_impl(double *out, double *lse, const void *q, const void *k_cache,
+                        const void *v_cache, int dtype, const int32_t *block_tables,
+                        const int32_t *context_lens, const int32_t *query_start_loc,
+                        int n_chunks, int H_q, int H_kv, int D, int bs, int MB, int64_t NB,
+                        double scale, int window, const uint8_t *select)
 {
     int rc = check_heads(H_q, H_kv, D, bs, MB, NB);
     if (rc) return rc;
-    if (n_chunks < 0 || query_start_loc[0] != 0) return OR_BAD_ARG;
+    if (n_chunks < 0 || query_start_loc[0] != 0 || window < 0) return OR_BAD_ARG;
     for (int c = 0; c < n_chunks; ++c) {
         int64_t C = (int64_t)query_start_loc[c + 1] - query_start_loc[c];
         if (C < 0 || context_lens[c] < C || (int64_t)context_lens[c] > (int64_t)MB * bs)
@@ -379,6 +379,7 @@ int oracle_prefill(double *out, double *lse, const void *q, const void *k_cache,
         int64_t C = (int64_t)query_start_loc[c + 1] - query_start_loc[c];
         int64_t i = row - query_start_loc[c];
         int64_t pos = (int64_t)context_lens[c] - C + i; /* this query's position */
+        int64_t j0 = window > 0 && pos + 1 - window > 0 ? pos + 1 - window : 0;
         paged_seq s = {k_cache, v_cache, dtype, block_tables + (int64_t)c * MB, MB,
                        H_kv, D, bs, NB, h / group, 1.0, 1.0};
         double *qv = malloc(sizeof(double) * D);
@@ -390,13 +391,40 @@ int oracle_prefill(double *out, double *lse, const void *q, const void *k_cache,
         }
         for (int d = 0; d < D; ++d) qv[d] = stored(q, rh * D + d, dtype);
         double l;
-        int r = attend(out + rh * D, &l, qv, &s, 0, pos + 1, scale, sbuf);
+        int r = attend(out + rh * D, &l, qv, &s, j0, pos + 1, scale, sbuf);
         if (lse) lse[rh] = l;
         if (r > err) err = r;
         free(qv);
         free(sbuf);
     }
     return err;
+}
+
+int oracle_prefill(double *out, double *lse, const void *q, const void *k_cache,
+                   const void *v_cache, int dtype, const int32_t *block_tables,
+                   const int32_t *context_lens, const int32_t *query_start_loc, int n_chunks,
+                   int H_q, int H_kv, int D, int bs, int MB, int64_t NB, double scale,
+                   const uint8_t *select)
+{
+    return prefill_impl(out, lse, q, k_cache, v_cache, dtype, block_tables, context_lens,
+                        query_start_loc, n_chunks, H_q, H_kv, D, bs, MB, NB, scale, 0, select);
+}
+
+/* [SW]+[CP] chunked prefill with a sliding window: as oracle_prefill, query i
+ * (at position pos = ctx - C + i) attending positions
+ * [max(0, pos - window + 1), pos] only: the window's last `window` positions
+ * end at the query's own, as a decode query at position ctx - 1 attends
+ * [ctx - window, ctx). window > 0. */
+int oracle_prefill_window(double *out, double *lse, const void *q, const void *k_cache,
+                          const void *v_cache, int dtype, const int32_t *block_tables,
+                          const int32_t *context_lens, const int32_t *query_start_loc,
+                          int n_chunks, int H_q, int H_kv, int D, int bs, int MB, int64_t NB,
+                          double scale, int window, const uint8_t *select)
+{
+    if (window <= 0) return OR_BAD_ARG;
+    return prefill_impl(out, lse, q, k_cache, v_cache, dtype, block_tables, context_lens,
+                        query_start_loc, n_chunks, H_q, H_kv, D, bs, MB, NB, scale, window,
+                        select);
 }
 
 /* Block copies of the paged pool, whole blocks (every K/V head) at a time:

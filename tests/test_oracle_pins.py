@@ -596,3 +596,86 @@ def test_window_equals_decode_of_the_dropped_prefix():
         if rest == W:
             assert torch.equal(out[b], plain[0]) and torch.equal(lse[b], plain_lse[0])
         assert torch.equal(out[b], ref[0])
+
+
+def test_prefill_window_no_cache_is_banded_attention():
+    """Chunks with nothing cached and identity tables equal torch's attention
+    under an explicit band mask: query i sees keys j with i - W < j <= i."""
+    Cs, H_q, H_kv, D, bs, W = [5, 16, 23], 4, 2, 8, 4, 6
+    g = torch.Generator().manual_seed(73)
+    ks = [torch.randn(H_kv, c, D, generator=g) for c in Cs]
+    vs = [torch.randn(H_kv, c, D, generator=g) for c in Cs]
+    rows, at = [], 0
+    for c in Cs:
+        n = -(-c // bs)
+        rows.append(list(range(at, at + n)))
+        at += n
+    kc, vc = place(ks, vs, rows, at + 1, bs)
+    tables = pad_tables(rows, max(len(r) for r in rows), at)
+    qsl = torch.tensor([0] + list(np.cumsum(Cs)), dtype=torch.int32)
+    q = torch.randn(sum(Cs), H_q, D, generator=g)
+    out, _ = oracle.prefill_window(q, kc, vc, tables, torch.tensor(Cs, dtype=torch.int32), qsl,
+                                   0.35, W)
+    for c, C in enumerate(Cs):
+        i = torch.arange(C)[:, None]
+        j = torch.arange(C)[None, :]
+        band = (j <= i) & (j > i - W)
+        qc = q[qsl[c]:qsl[c + 1]].transpose(0, 1).to(F64)
+        ref = F.scaled_dot_product_attention(qc[None], ks[c][None].to(F64), vs[c][None].to(F64),
+                                             attn_mask=band, scale=0.35,
+                                             enable_gqa=True)[0].transpose(0, 1)
+        torch.testing.assert_close(out[qsl[c]:qsl[c + 1]], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_window_covering_everything_is_plain_prefill():
+    ctxs, H_q, H_kv, D, bs = [37, 70], 4, 2, 8, 16
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=74)
+    qp = torch.randn(21, H_q, D, generator=torch.Generator().manual_seed(75))
+    qsl = torch.tensor([0, 9, 21], dtype=torch.int32)
+    a = oracle.prefill(qp, kc, vc, tables, lens, qsl, 0.3)
+    b = oracle.prefill_window(qp, kc, vc, tables, lens, qsl, 0.3, 70)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_prefill_window_query_equals_windowed_decode_at_its_position():
+    """Query i of a windowed chunk equals a windowed decode over the first
+    pos + 1 tokens (the decode query sits at position pos)."""
+    ctxs, H_q, H_kv, D, bs, W = [37, 70], 4, 1, 8, 16, 13
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=76)
+    Cs = [9, 20]
+    qp = torch.randn(sum(Cs), H_q, D, generator=torch.Generator().manual_seed(77))
+    qsl = torch.tensor([0, Cs[0], Cs[0] + Cs[1]], dtype=torch.int32)
+    out, lse = oracle.prefill_window(qp, kc, vc, tables, lens, qsl, 0.3, W)
+    for c, C in enumerate(Cs):
+        for i in range(C):
+            row = int(qsl[c]) + i
+            pos = ctxs[c] - C + i
+            d, dl = oracle.decode_window(qp[row][None], kc, vc, tables[c:c + 1],
+                                         torch.tensor([pos + 1], dtype=torch.int32), 0.3, W)
+            assert torch.equal(out[row], d[0]) and torch.equal(lse[row], dl[0])
+
+
+def test_prefill_window_ignores_keys_outside_the_band():
+    """Changing keys/values more than W - 1 positions before a query, or
+    after it, leaves that query's output bit-identical; changing one inside
+    its band does not."""
+    ctxs, H_q, H_kv, D, bs, W = [40], 2, 1, 8, 8, 10
+    q, ks, vs, kc, vc, tables, lens = random_paged(ctxs, H_q, H_kv, D, bs, seed=78)
+    qp = torch.randn(12, H_q, D, generator=torch.Generator().manual_seed(79))
+    qsl = torch.tensor([0, 12], dtype=torch.int32)
+    out, _ = oracle.prefill_window(qp, kc, vc, tables, lens, qsl, 0.3, W)
+    # query i sits at position 28 + i and sees [19 + i, 28 + i]
+    ks2 = [ks[0].clone()]
+    vs2 = [vs[0].clone()]
+    ks2[0][:, :19] += 3.0
+    vs2[0][:, :19] -= 2.0
+    ks2[0][:, 39:] += 3.0
+    kc2, vc2 = place(ks2, vs2, [tables[0].tolist()], kc.shape[0], bs)
+    out2, _ = oracle.prefill_window(qp, kc2, vc2, tables, lens, qsl, 0.3, W)
+    assert torch.equal(out[:11], out2[:11])  # rows 0..10 see [19, 38]
+    assert not torch.equal(out[11], out2[11])  # row 11 sees position 39
+    vs3 = [vs[0].clone()]
+    vs3[0][:, 25] += 1.0  # inside the band of rows 0..6
+    kc3, vc3 = place(ks, vs3, [tables[0].tolist()], kc.shape[0], bs)
+    out3, _ = oracle.prefill_window(qp, kc3, vc3, tables, lens, qsl, 0.3, W)
+    assert not torch.equal(out[:7], out3[:7]) and torch.equal(out[7:], out3[7:])
