@@ -105,9 +105,13 @@ def decode_bytes(batch) -> float:
     eq = batch.q.element_size()
     ctx = batch.context_lens.to(torch.int64)
     H_kv, D, bs = batch.num_kv_heads, batch.head_dim, batch.block_size
-    kv = int((2 * ctx * H_kv * D * e).sum())
+    lo = torch.zeros_like(ctx)
+    if batch.sliding_window > 0:  # only the window's tokens and blocks
+        lo = (ctx - batch.sliding_window).clamp(min=0)
+    kv = int((2 * (ctx - lo) * H_kv * D * e).sum())
     qo = 2 * batch.num_seqs * batch.num_q_heads * D * eq
-    tbl = int((4 * ((ctx + bs - 1) // bs) * H_kv).sum())
+    nblk = torch.where(ctx > lo, (ctx - 1) // bs - lo // bs + 1, torch.zeros_like(ctx))
+    tbl = int((4 * nblk * H_kv).sum())
     return float(kv + qo + tbl + 4 * batch.num_seqs)
 
 
@@ -121,17 +125,22 @@ def reshape_bytes(batch) -> float:
 
 def prefill_flops(batch) -> float:
     """Algorithmic FLOPs of the chunked prefill: Q.K^T and P.V over each
-    query's causal range (4 D H_q per query-key pair)."""
+    query's causal range, or its band under a sliding window (4 D H_q per
+    query-key pair)."""
     if batch.prefill_q is None:
         return 0.0
     qsl = batch.query_start_loc.tolist()
     ctx = batch.prefill_context_lens.tolist()
-    H_q, D = batch.num_q_heads, batch.head_dim
+    H_q, D, W = batch.num_q_heads, batch.head_dim, batch.sliding_window
     f = 0
     for c in range(len(ctx)):
         C = qsl[c + 1] - qsl[c]
         cached = ctx[c] - C
-        f += 4 * D * H_q * (C * cached + C * (C + 1) // 2)
+        if W > 0:  # query at position p sees min(p + 1, W) keys
+            pairs = sum(min(p + 1, W) for p in range(cached, ctx[c]))
+        else:
+            pairs = C * cached + C * (C + 1) // 2
+        f += 4 * D * H_q * pairs
     return float(f)
 
 
@@ -321,7 +330,7 @@ class Runner:
             c["prefill"] = pa.prepare_prefill_chunk(
                 pout if pout is not None else self.pout, d.prefill_q, d.k_cache, d.v_cache,
                 d.prefill_block_tables, d.prefill_context_lens, d.query_start_loc, self.max_q,
-                d.scale)
+                d.scale, self.host.sliding_window)
         if d.q is not None and d.num_seqs and d.k_scale is not None:
             c["decode"] = pa.prepare_decode_fp8(out if out is not None else self.out, d.q,
                                                 d.k_cache, d.v_cache, d.k_scale, d.v_scale,
@@ -330,7 +339,8 @@ class Runner:
         elif d.q is not None and d.num_seqs:
             c["decode"] = pa.prepare_decode(out if out is not None else self.out, d.q, d.k_cache,
                                             d.v_cache, d.block_tables, d.context_lens,
-                                            self.max_ctx, d.scale, self.part, self.ws)
+                                            self.max_ctx, d.scale, self.part, self.ws,
+                                            self.host.sliding_window)
         return c
 
     def step(self, ev=None, calls=None):
@@ -359,6 +369,7 @@ def run_ours(args, rank, world):
                        block_size=args.block_size)
     if args.partition is not None:
         batch.partition_size = args.partition
+    batch.sliding_window = args.window
     r = Runner(batch, dev)
     hbm, bf16, bf16_sus, basis = load_peaks()
 
@@ -475,6 +486,7 @@ def run_ours(args, rank, world):
     _, e2e_ms = aggregate(0.0, e2e_ms_local, world, dev)
 
     line = None
+    wtag = f"_window{args.window}" if args.window else ""
     if rank == 0:
         if r.dominant == "decode":
             value = dbytes_total / (ms * 1e-3) / 1e9
@@ -485,7 +497,7 @@ def run_ours(args, rank, world):
                     "peak_basis": f"{basis} hbm_gbs",
                     "kernel": "pa_decode (decode_split + decode_reduce)",
                     "alg_bytes_per_launch": dbytes,
-                    "traffic": profiled_traffic(f"decode_{args.workload}.md",
+                    "traffic": profiled_traffic(f"decode_{args.workload}{wtag}.md",
                                                 DECODE_SOURCES)}
         else:
             value = dbytes_total / (ms * 1e-3) / 1e9
@@ -495,7 +507,7 @@ def run_ours(args, rank, world):
                     "unit": "TFLOP/s", "frac": round(achieved / bf16_sus, 4),
                     "peak_basis": f"{basis} bf16_tflops_sustained",
                     "kernel": "pa_prefill_chunk", "alg_flops_per_launch": pflops,
-                    "traffic": profiled_traffic(f"prefill_{args.workload}.md",
+                    "traffic": profiled_traffic(f"prefill_{args.workload}{wtag}.md",
                                                 PREFILL_SOURCES)}
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
@@ -547,6 +559,8 @@ def workload_config(batch, name, world, r=None):
     if batch.prefill_q is not None:
         c.update({"prefill_chunks": batch.query_start_loc.numel() - 1,
                   "prefill_tokens": batch.prefill_q.shape[0]})
+    if batch.sliding_window > 0:
+        c["sliding_window"] = batch.sliding_window
     return c
 
 
@@ -562,13 +576,23 @@ def _oracle_step(batch, k, v, select=None, pselect=None):
                            batch.context_lens, batch.scale, select=select)
         return
     oracle.reshape_and_cache(batch.key, batch.value, k, v, batch.slot_mapping)
+    W = batch.sliding_window
     if batch.prefill_q is not None:
-        oracle.prefill(batch.prefill_q, k, v, batch.prefill_block_tables,
-                       batch.prefill_context_lens, batch.query_start_loc, batch.scale,
-                       select=pselect)
+        if W > 0:
+            oracle.prefill_window(batch.prefill_q, k, v, batch.prefill_block_tables,
+                                  batch.prefill_context_lens, batch.query_start_loc, batch.scale,
+                                  W, select=pselect)
+        else:
+            oracle.prefill(batch.prefill_q, k, v, batch.prefill_block_tables,
+                           batch.prefill_context_lens, batch.query_start_loc, batch.scale,
+                           select=pselect)
     if batch.q is not None and batch.num_seqs:
-        oracle.decode(batch.q, k, v, batch.block_tables, batch.context_lens, batch.scale,
-                      select=select)
+        if W > 0:
+            oracle.decode_window(batch.q, k, v, batch.block_tables, batch.context_lens,
+                                 batch.scale, W, select=select)
+        else:
+            oracle.decode(batch.q, k, v, batch.block_tables, batch.context_lens, batch.scale,
+                          select=select)
 
 
 def _sample_masks(batch, frac: float, offset: int):
@@ -623,6 +647,7 @@ def run_reference(args, rank, world):
         return
     import oracle
     batch = make_batch(args.workload, seed=0, num_blocks=args.num_blocks)
+    batch.sliding_window = args.window
     k, v = batch.k_cache, batch.v_cache
     total = args.steps + args.warmup
     t = time.perf_counter()
@@ -720,11 +745,16 @@ def main(argv=None):
                     help="block size override for the decode workloads (pool bytes kept)")
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="physical pool size override (a smaller pool for profiler captures)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window: each query sees only its last W positions "
+                         "(0: the whole context); not for the FP8 workloads")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.window < 0 or (args.window and args.workload.endswith("_fp8")):
+        ap.error("--window takes W > 0 and a bf16/fp32 workload")
     rank, local, world = rank_env()
     if world != args.gpus and world > 1:
         print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)

@@ -226,6 +226,25 @@ PA_API pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache,
                            int num_blocks, int max_blocks_per_seq, float scale, pa_dtype dtype,
                            cudaStream_t stream);
 
+/* pa_prefill_chunk restricted to a sliding window (page "LLM推理优化",
+ * section 2.3, flash_attn_func window_size; page "vLLM框架是怎么做推理加速的",
+ * 追问 3, sliding window attention): query i of chunk c, at position p,
+ * attends positions [max(0, p - sliding_window + 1), p] only, the band a
+ * pa_decode_sliding_window query at position context_lens[b] - 1 sees.
+ * Table entries of blocks wholly before the chunk's first query's band are
+ * never read (an engine may have freed them). sliding_window must be > 0;
+ * other arguments and errors as for pa_prefill_chunk. */
+PA_API pa_status pa_prefill_chunk_sliding_window(void *out, const void *q, const void *k_cache,
+                                                 const void *v_cache, const int32_t *block_tables,
+                                                 const int32_t *context_lens,
+                                                 const int32_t *query_start_loc, int num_chunks,
+                                                 int num_query_tokens, int max_query_len,
+                                                 int num_q_heads, int num_kv_heads, int head_dim,
+                                                 int block_size, int num_blocks,
+                                                 int max_blocks_per_seq, float scale,
+                                                 int sliding_window, pa_dtype dtype,
+                                                 cudaStream_t stream);
+
 /* Copy-on-write of whole blocks inside one pool: for each pair i of
  * block_mapping (int64 [num_pairs][2], device-readable), block
  * block_mapping[i][1] := block block_mapping[i][0], every kv head, K and V,

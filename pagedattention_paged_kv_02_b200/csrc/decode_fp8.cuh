@@ -49,6 +49,29 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
     return r;
 }
 
+// 2^x on the special-function unit, subnormal results flushed to zero (a
+// softmax weight below 2^-126 of the row's largest does not register).
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Four E4M3 codes w = [c0 c1 c2 c3] (c0 the low byte) -> the f16 pairs
+// {c0, c2} (even) and {c1, c3} (odd), each half equal to its code's value
+// times 2^-8, on the integer pipe: the code's sign goes to bit 15 and its
+// seven magnitude bits to bits 13..7, so the 4-bit exponent field becomes the
+// low four bits of f16's 5-bit field (biases 7 and 15: a factor 2^-8) and the
+// 3-bit mantissa the top of f16's; subnormal codes become f16 subnormals with
+// the same factor. Exact for every finite code; the two NaN codes (0x7f,
+// 0xff), which the quantising append never writes, come out finite (+-480
+// once the 2^8 is put back).
+__device__ __forceinline__ void e4m3x4_to_f16x2_scaled(uint32_t w, uint32_t &even,
+                                                       uint32_t &odd) {
+    odd = (w & 0x80008000u) | ((w >> 1) & 0x3F803F80u);
+    even = ((w << 8) & 0x80008000u) | ((w << 7) & 0x3F803F80u);
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -65,7 +88,13 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
 // CT: tokens per pipeline stage (16 or 32). A 32-token stage is two
 // 16-token page pieces (each inside one physical block, so each has its own
 // table lookup); it halves the softmax and hand-off work per byte.
-template <int NW, int NS, int CT>
+// CV: where codes become f16. 0: the conversion instruction for K and V;
+// 1: K on the integer pipe (e4m3x4_to_f16x2_scaled), V by instruction;
+// 2: both on the integer pipe; the 2^-8 of the integer form folds into the
+// scales. The conversion instruction shares a narrow pipe with the
+// exponentials, but the integer form costs 3.5 instructions per pair and
+// measured slower on B200, so 0 is the default.
+template <int NW, int NS, int CT, int CV>
 __global__ void __launch_bounds__(NW * 32)
     decode_split_e4m3(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -89,6 +118,7 @@ __global__ void __launch_bounds__(NW * 32)
     const int h0 = kvh * a.group + ht * HT;
     const int nh = min(HT, a.group - ht * HT);
 
+    allow_dependent_launch();
     const int ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
     const int lo = window_lo(a, ctx), base = span_base(a, ctx);
     const int n_splits = (ctx - base + a.P - 1) / a.P;
@@ -152,12 +182,14 @@ __global__ void __launch_bounds__(NW * 32)
         for (int i = 0; i < NS && i < my_n; ++i) issue(i);
     }
 
-    const float sl2 = a.scale_log2 * __ldg(a.k_scale + kvh);
-    const float vsc = __ldg(a.v_scale + kvh);
+    const float sl2 = a.scale_log2 * __ldg(a.k_scale + kvh) * (CV >= 1 ? 256.f : 1.f);
+    const float vsc = __ldg(a.v_scale + kvh) * (CV >= 2 ? 256.f : 1.f);
 
     // Q fragments in f16, dims permuted to match the K fragments: slot
     // 2c+j (j = 0,1) of k-step ks holds dim 16ks+4c+j, slot 2c+8+j holds
-    // dim 16ks+4c+2+j (c = lane % 4)
+    // dim 16ks+4c+2+j (c = lane % 4); with K converted on the integer pipe
+    // (even and odd codes of a word) slot 2c+j holds dim 16ks+4c+2j and slot
+    // 2c+8+j dim 16ks+4c+1+2j
     const int g = lane >> 2, tig = lane & 3;
     uint32_t qa[8][4];
     {
@@ -171,10 +203,17 @@ __global__ void __launch_bounds__(NW * 32)
                 uint2 v = make_uint2(0u, 0u);
                 if (qr < nh)
                     v = __ldg(reinterpret_cast<const uint2 *>(qb + qr * D + ks * 16 + 4 * tig));
-                qa[ks][hr] = pack_f16x2(bf16_lo(v.x), bf16_hi(v.x));      // dims +0, +1
-                qa[ks][hr + 2] = pack_f16x2(bf16_lo(v.y), bf16_hi(v.y));  // dims +2, +3
+                if (CV >= 1) {
+                    qa[ks][hr] = pack_f16x2(bf16_lo(v.x), bf16_lo(v.y));      // dims +0, +2
+                    qa[ks][hr + 2] = pack_f16x2(bf16_hi(v.x), bf16_hi(v.y));  // dims +1, +3
+                } else {
+                    qa[ks][hr] = pack_f16x2(bf16_lo(v.x), bf16_hi(v.x));      // dims +0, +1
+                    qa[ks][hr + 2] = pack_f16x2(bf16_lo(v.y), bf16_hi(v.y));  // dims +2, +3
+                }
             }
     }
+
+    const bool hi_rows = nh > 8;
 
     // O fragments of 16 virtual n-tiles: tile 2u+p, column n <-> dim 16u+2n+p
     float o[16][4];
@@ -232,29 +271,55 @@ __global__ void __launch_bounds__(NW * 32)
                         const int u = kp * 2 + (mi >> 1);
                         uint32_t r0, r1, r2, r3;
                         ldsm_x4(kb + p * kChunk * D + sw128(r, u), r0, r1, r2, r3);
-                        mma_f16_16816(sc[2 * p], qa[2 * kp], e4m3x2_to_f16x2(r0),
-                                      e4m3x2_to_f16x2(r0 >> 16));
-                        mma_f16_16816(sc[2 * p + 1], qa[2 * kp], e4m3x2_to_f16x2(r1),
-                                      e4m3x2_to_f16x2(r1 >> 16));
-                        mma_f16_16816(sc[2 * p], qa[2 * kp + 1], e4m3x2_to_f16x2(r2),
-                                      e4m3x2_to_f16x2(r2 >> 16));
-                        mma_f16_16816(sc[2 * p + 1], qa[2 * kp + 1], e4m3x2_to_f16x2(r3),
-                                      e4m3x2_to_f16x2(r3 >> 16));
+                        if constexpr (CV >= 1) {
+                            uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
+                            e4m3x4_to_f16x2_scaled(r0, e0, o0);
+                            e4m3x4_to_f16x2_scaled(r1, e1, o1);
+                            e4m3x4_to_f16x2_scaled(r2, e2, o2);
+                            e4m3x4_to_f16x2_scaled(r3, e3, o3);
+                            mma_f16_16816(sc[2 * p], qa[2 * kp], e0, o0);
+                            mma_f16_16816(sc[2 * p + 1], qa[2 * kp], e1, o1);
+                            mma_f16_16816(sc[2 * p], qa[2 * kp + 1], e2, o2);
+                            mma_f16_16816(sc[2 * p + 1], qa[2 * kp + 1], e3, o3);
+                        } else {
+                            mma_f16_16816(sc[2 * p], qa[2 * kp], e4m3x2_to_f16x2(r0),
+                                          e4m3x2_to_f16x2(r0 >> 16));
+                            mma_f16_16816(sc[2 * p + 1], qa[2 * kp], e4m3x2_to_f16x2(r1),
+                                          e4m3x2_to_f16x2(r1 >> 16));
+                            mma_f16_16816(sc[2 * p], qa[2 * kp + 1], e4m3x2_to_f16x2(r2),
+                                          e4m3x2_to_f16x2(r2 >> 16));
+                            mma_f16_16816(sc[2 * p + 1], qa[2 * kp + 1], e4m3x2_to_f16x2(r3),
+                                          e4m3x2_to_f16x2(r3 >> 16));
+                        }
                     }
             }
             float mx0 = -INFINITY, mx1 = -INFINITY;
+            if (full) {
 #pragma unroll
-            for (int nt = 0; nt < 2 * PIECES; ++nt)
+                for (int nt = 0; nt < 2 * PIECES; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int tok = nt * 8 + 2 * tig + (e & 1);
-                    const bool ok = tok < valid && tok >= first && ((pok >> (tok / kChunk)) & 1);
-                    sc[nt][e] = ok ? sc[nt][e] * sl2 : -INFINITY;
-                    if (e < 2)
-                        mx0 = fmaxf(mx0, sc[nt][e]);
-                    else
-                        mx1 = fmaxf(mx1, sc[nt][e]);
-                }
+                    for (int e = 0; e < 4; ++e) {
+                        sc[nt][e] *= sl2;
+                        if (e < 2)
+                            mx0 = fmaxf(mx0, sc[nt][e]);
+                        else
+                            mx1 = fmaxf(mx1, sc[nt][e]);
+                    }
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < 2 * PIECES; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int tok = nt * 8 + 2 * tig + (e & 1);
+                        const bool ok =
+                            tok < valid && tok >= first && ((pok >> (tok / kChunk)) & 1);
+                        sc[nt][e] = ok ? sc[nt][e] * sl2 : -INFINITY;
+                        if (e < 2)
+                            mx0 = fmaxf(mx0, sc[nt][e]);
+                        else
+                            mx1 = fmaxf(mx1, sc[nt][e]);
+                    }
+            }
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
             mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
             mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
@@ -262,19 +327,29 @@ __global__ void __launch_bounds__(NW * 32)
             const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
             // a row with nothing visible yet keeps reference -inf: use 0 then
             const float r0m = mn0 == -INFINITY ? 0.f : mn0, r1m = mn1 == -INFINITY ? 0.f : mn1;
-            const float c0 = exp2f(m0 - r0m), c1 = exp2f(m1 - r1m);
+            const float c0 = ex2_fast(m0 - r0m), c1 = ex2_fast(m1 - r1m);
             m0 = mn0;
             m1 = mn1;
             uint32_t pa[PIECES][4];
             float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
             for (int p = 0; p < PIECES; ++p) {
-                pa[p][0] = pack_f16x2(exp2f(sc[2 * p][0] - r0m), exp2f(sc[2 * p][1] - r0m));
-                pa[p][1] = pack_f16x2(exp2f(sc[2 * p][2] - r1m), exp2f(sc[2 * p][3] - r1m));
-                pa[p][2] = pack_f16x2(exp2f(sc[2 * p + 1][0] - r0m), exp2f(sc[2 * p + 1][1] - r0m));
-                pa[p][3] = pack_f16x2(exp2f(sc[2 * p + 1][2] - r1m), exp2f(sc[2 * p + 1][3] - r1m));
+                pa[p][0] = pack_f16x2(ex2_fast(sc[2 * p][0] - r0m), ex2_fast(sc[2 * p][1] - r0m));
+                pa[p][2] =
+                    pack_f16x2(ex2_fast(sc[2 * p + 1][0] - r0m), ex2_fast(sc[2 * p + 1][1] - r0m));
                 ps0 += f16_lo(pa[p][0]) + f16_hi(pa[p][0]) + f16_lo(pa[p][2]) + f16_hi(pa[p][2]);
-                ps1 += f16_lo(pa[p][1]) + f16_hi(pa[p][1]) + f16_lo(pa[p][3]) + f16_hi(pa[p][3]);
+            }
+            if (hi_rows) {  // rows g+8 hold query heads only when the tile has more than 8
+#pragma unroll
+                for (int p = 0; p < PIECES; ++p) {
+                    pa[p][1] = pack_f16x2(ex2_fast(sc[2 * p][2] - r1m), ex2_fast(sc[2 * p][3] - r1m));
+                    pa[p][3] = pack_f16x2(ex2_fast(sc[2 * p + 1][2] - r1m),
+                                          ex2_fast(sc[2 * p + 1][3] - r1m));
+                    ps1 += f16_lo(pa[p][1]) + f16_hi(pa[p][1]) + f16_lo(pa[p][3]) + f16_hi(pa[p][3]);
+                }
+            } else {
+#pragma unroll
+                for (int p = 0; p < PIECES; ++p) pa[p][1] = pa[p][3] = 0u;
             }
             l0 = l0 * c0 + ps0;
             l1 = l1 * c1 + ps1;
@@ -303,11 +378,24 @@ __global__ void __launch_bounds__(NW * 32)
                         const int u = up * 2 + (mi >> 1);
                         uint32_t r0, r1, r2, r3;
                         ldsm_x4_t(vb + p * kChunk * D + sw128(r, u), r0, r1, r2, r3);
+                        const int u0 = up * 2, u1 = up * 2 + 1;
+                        if constexpr (CV >= 2) {
+                            // even codes of a word: dim 2g, odd codes: dim 2g+1
+                            uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
+                            e4m3x4_to_f16x2_scaled(r0, e0, o0);
+                            e4m3x4_to_f16x2_scaled(r1, e1, o1);
+                            e4m3x4_to_f16x2_scaled(r2, e2, o2);
+                            e4m3x4_to_f16x2_scaled(r3, e3, o3);
+                            mma_f16_16816(o[2 * u0], pa[p], e0, e1);
+                            mma_f16_16816(o[2 * u0 + 1], pa[p], o0, o1);
+                            mma_f16_16816(o[2 * u1], pa[p], e2, e3);
+                            mma_f16_16816(o[2 * u1 + 1], pa[p], o2, o3);
+                            continue;
+                        }
                         const uint32_t a0 = __byte_perm(r0, 0, 0x3120);
                         const uint32_t a1 = __byte_perm(r1, 0, 0x3120);
                         const uint32_t b0 = __byte_perm(r2, 0, 0x3120);
                         const uint32_t b1 = __byte_perm(r3, 0, 0x3120);
-                        const int u0 = up * 2, u1 = up * 2 + 1;
                         mma_f16_16816(o[2 * u0], pa[p], e4m3x2_to_f16x2(a0), e4m3x2_to_f16x2(a1));
                         mma_f16_16816(o[2 * u0 + 1], pa[p], e4m3x2_to_f16x2(a0 >> 16),
                                       e4m3x2_to_f16x2(a1 >> 16));

@@ -118,19 +118,22 @@ Pipe decode_pipe() {
     return p;
 }
 
-// Launch shape of the FP8 split kernel: warps x stages x tokens per stage;
-// PA_DECODE_PIPE_FP8=<warps>x<stages>x<tokens> (built: 4x2x16, 4x4x16,
-// 4x2x32, 4x3x32, 2x4x32; default 4x2x32).
+// Launch shape of the FP8 split kernel: warps x stages x tokens per stage x
+// code conversion (decode_split_e4m3's CV);
+// PA_DECODE_PIPE_FP8=<warps>x<stages>x<tokens>x<cv> (built: 4x2x32x0,
+// 4x2x32x2, 4x2x16x0, 4x3x32x0; default 4x2x32x0: on B200 the conversion
+// instruction beat the integer-pipe form, 0.62 vs 0.55 of the HBM peak on
+// the Llama-7B batch).
 struct PipeFp8 {
-    int nw, ns, ct;
+    int nw, ns, ct, cv;
 };
 
 PipeFp8 decode_pipe_fp8() {
     static PipeFp8 p = [] {
-        PipeFp8 r{4, 2, 32};
+        PipeFp8 r{4, 2, 32, 0};
         if (const char *e = std::getenv("PA_DECODE_PIPE_FP8")) {
-            int w = 0, s = 0, c = 0;
-            if (sscanf(e, "%dx%dx%d", &w, &s, &c) == 3) r = PipeFp8{w, s, c};
+            int w = 0, s = 0, c = 0, v = 0;
+            if (sscanf(e, "%dx%dx%dx%d", &w, &s, &c, &v) == 4) r = PipeFp8{w, s, c, v};
         }
         return r;
     }();
@@ -184,10 +187,10 @@ int prefill_poly() {
     return v;
 }
 
-template <int POLY>
+template <int POLY, bool WIN>
 pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                             const CUtensorMap &mv, dim3 grid, size_t smem, cudaStream_t st) {
-    auto k = prefill_tc_kernel<POLY>;
+    auto k = prefill_tc_kernel<POLY, WIN>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
     // the kernel's register split must fit the registers it launches with,
     // or the warpgroups that grow would wait forever
@@ -212,15 +215,43 @@ bool encode_cache_map_u8(CUtensorMap *m, const void *cache, int NB, int H_kv, in
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NW, int NS, int CT>
+template <int NW, int NS, int CT, int CV>
 pa_status launch_decode_e4m3(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
                              dim3 grid, cudaStream_t st) {
     constexpr int STAGE = 2 * CT * 128;
     using L = DecodeSmem<NW, NS, STAGE, kHeadsBf16, 128>;
     const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
-    auto k = decode_split_e4m3<NW, NS, CT>;
+    auto k = decode_split_e4m3<NW, NS, CT, CV>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
     k<<<grid, NW * 32, smem, st>>>(a, mk, mv);
+    return launch_status();
+}
+
+// The LSE merge behind a split launch, as a programmatic dependent launch
+// (its CTAs may start while the split grid's last CTAs run; they wait for
+// that grid's completion before reading partials).
+template <int D, typename OutT>
+pa_status launch_reduce(const DecodeArgs &a, cudaStream_t st) {
+    const long long heads = (long long)a.num_seqs * a.H_q;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.stream = st;
+    cfg.dynamicSmemBytes = 0;
+    if (a.S_max <= kWarpMergeMax) {
+        cfg.gridDim = dim3((unsigned)((heads + 7) / 8));
+        cfg.blockDim = dim3(256);
+        if (cudaLaunchKernelEx(&cfg, decode_reduce_warp<D, OutT>, a) != cudaSuccess)
+            return PA_ERR_CUDA;
+    } else {
+        cfg.gridDim = dim3((unsigned)heads);
+        cfg.blockDim = dim3(128);
+        if (cudaLaunchKernelEx(&cfg, decode_reduce<D, OutT>, a) != cudaSuccess)
+            return PA_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -364,22 +395,16 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
                              : dispatch_bf16<64>(a, mk, mv, grid, stream);
         if (st != PA_OK) return st;
         if (S1 > 1) {
-            if (head_dim == 128)
-                decode_reduce<128, __nv_bfloat16><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
-            else
-                decode_reduce<64, __nv_bfloat16><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
-            st = launch_status();
+            st = head_dim == 128 ? launch_reduce<128, __nv_bfloat16>(a, stream)
+                                 : launch_reduce<64, __nv_bfloat16>(a, stream);
         }
     } else {
         st = head_dim == 128 ? launch_decode_f32<128, 4, 2>(a, grid, stream)
                              : launch_decode_f32<64, 4, 2>(a, grid, stream);
         if (st != PA_OK) return st;
         if (S1 > 1) {
-            if (head_dim == 128)
-                decode_reduce<128, float><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
-            else
-                decode_reduce<64, float><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
-            st = launch_status();
+            st = head_dim == 128 ? launch_reduce<128, float>(a, stream)
+                                 : launch_reduce<64, float>(a, stream);
         }
     }
     return st;
@@ -519,26 +544,25 @@ pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const voi
         return PA_ERR_CUDA;
     const dim3 grid((unsigned)S1, (unsigned)gy, (unsigned)num_seqs);
     const PipeFp8 pp = decode_pipe_fp8();
-    pa_status st =
-        pp.nw == 4 && pp.ns == 2 && pp.ct == 16   ? launch_decode_e4m3<4, 2, 16>(a, mk, mv, grid, stream)
-        : pp.nw == 4 && pp.ns == 4 && pp.ct == 16 ? launch_decode_e4m3<4, 4, 16>(a, mk, mv, grid, stream)
-        : pp.nw == 4 && pp.ns == 3 && pp.ct == 32 ? launch_decode_e4m3<4, 3, 32>(a, mk, mv, grid, stream)
-        : pp.nw == 2 && pp.ns == 4 && pp.ct == 32 ? launch_decode_e4m3<2, 4, 32>(a, mk, mv, grid, stream)
-                                                  : launch_decode_e4m3<4, 2, 32>(a, mk, mv, grid, stream);
+    auto is = [&](int w, int n, int c, int v) {
+        return pp.nw == w && pp.ns == n && pp.ct == c && pp.cv == v;
+    };
+    pa_status st = is(4, 2, 32, 2)   ? launch_decode_e4m3<4, 2, 32, 2>(a, mk, mv, grid, stream)
+                   : is(4, 2, 16, 0) ? launch_decode_e4m3<4, 2, 16, 0>(a, mk, mv, grid, stream)
+                   : is(4, 3, 32, 0) ? launch_decode_e4m3<4, 3, 32, 0>(a, mk, mv, grid, stream)
+                                     : launch_decode_e4m3<4, 2, 32, 0>(a, mk, mv, grid, stream);
     if (st != PA_OK) return st;
-    if (S1 > 1) {
-        decode_reduce<128, __nv_bfloat16><<<num_seqs * num_q_heads, 128, 0, stream>>>(a);
-        st = launch_status();
-    }
+    if (S1 > 1) st = launch_reduce<128, __nv_bfloat16>(a, stream);
     return st;
 }
 
-pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
-                           const int32_t *block_tables, const int32_t *context_lens,
-                           const int32_t *query_start_loc, int num_chunks, int num_query_tokens,
-                           int max_query_len, int num_q_heads, int num_kv_heads, int head_dim,
-                           int block_size, int num_blocks, int max_blocks_per_seq, float scale,
-                           pa_dtype dtype, cudaStream_t stream) {
+static pa_status prefill_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_tables, const int32_t *context_lens,
+                              const int32_t *query_start_loc, int num_chunks,
+                              int num_query_tokens, int max_query_len, int num_q_heads,
+                              int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                              int max_blocks_per_seq, float scale, int window, pa_dtype dtype,
+                              cudaStream_t stream) {
     if (num_chunks < 0 || num_query_tokens < 0 || max_query_len < 0 || num_q_heads <= 0 ||
         num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0)
@@ -588,12 +612,43 @@ pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const 
     a.bs = block_size;
     a.NB = num_blocks;
     a.MB = max_blocks_per_seq;
+    a.window = window;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
     const size_t smem = 1024 + kPfSmem;
     const dim3 grid((unsigned)qtiles, (unsigned)num_q_heads, (unsigned)num_chunks);
-    if (prefill_poly() == 4) return launch_prefill_tc<4>(a, mq, mk, mv, grid, smem, stream);
-    return launch_prefill_tc<0>(a, mq, mk, mv, grid, smem, stream);
+    if (window > 0) return launch_prefill_tc<0, true>(a, mq, mk, mv, grid, smem, stream);
+    if (prefill_poly() == 4) return launch_prefill_tc<4, false>(a, mq, mk, mv, grid, smem, stream);
+    return launch_prefill_tc<0, false>(a, mq, mk, mv, grid, smem, stream);
+}
+
+pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *block_tables, const int32_t *context_lens,
+                           const int32_t *query_start_loc, int num_chunks, int num_query_tokens,
+                           int max_query_len, int num_q_heads, int num_kv_heads, int head_dim,
+                           int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                           pa_dtype dtype, cudaStream_t stream) {
+    return prefill_impl(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                        num_chunks, num_query_tokens, max_query_len, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, max_blocks_per_seq, scale, 0, dtype,
+                        stream);
+}
+
+pa_status pa_prefill_chunk_sliding_window(void *out, const void *q, const void *k_cache,
+                                          const void *v_cache, const int32_t *block_tables,
+                                          const int32_t *context_lens,
+                                          const int32_t *query_start_loc, int num_chunks,
+                                          int num_query_tokens, int max_query_len,
+                                          int num_q_heads, int num_kv_heads, int head_dim,
+                                          int block_size, int num_blocks,
+                                          int max_blocks_per_seq, float scale,
+                                          int sliding_window, pa_dtype dtype,
+                                          cudaStream_t stream) {
+    if (sliding_window <= 0) return PA_ERR_INVALID_ARG;
+    return prefill_impl(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                        num_chunks, num_query_tokens, max_query_len, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
+                        sliding_window, dtype, stream);
 }
 
 }  // extern "C"

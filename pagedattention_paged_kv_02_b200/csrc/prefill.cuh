@@ -10,24 +10,33 @@
 // "vLLM与PagedAttention的原理"), and the softmax is computed tile by tile with
 // a running max and sum (page "LLM推理优化", section 2.1).
 //
-// One CTA = 128 query rows of one query head of one chunk (the tcgen05 M
-// tile); keys are processed in tiles of 128. Six warps:
-//   warp 4 (one lane)  TMA: the Q tile once, then each key tile's K and V as
-//                      16-token page pieces (128-byte swizzle) gathered
-//                      through the block table; K and V each single-buffered
-//                      with their own full/free barriers, so K(j+1) streams in
-//                      while tile j's softmax and P.V run.
-//   warp 5 (one lane)  MMA: S = Q K^T (8 x 128x128x16, both operands K-major
-//                      in shared memory) into tensor memory columns [0,128);
-//                      then O += P V with P read from tensor memory and V
-//                      MN-major in shared memory, into columns [128,256).
-//   warps 0-3          softmax: thread r owns row r (tensor-memory lane r):
-//                      row max, exp2, the running sum, bf16 P written back
-//                      over the consumed S columns; O is rescaled in tensor
-//                      memory only when a row's max grows by more than 2^8
-//                      (the result is exact for any reference max as long as
-//                      O and the sum share it); the epilogue divides by the
-//                      sum and writes bf16 rows.
+// With a sliding window of W positions (page "LLM推理优化", section 2.3 on
+// attention masks, read as a band), query i sees keys cached+i-W+1 ..
+// cached+i only; key tiles wholly before a query tile's band are neither
+// loaded nor multiplied.
+//
+// One CTA = two 128-row query tiles (the tcgen05 M) of one query head of one
+// chunk, sharing every K/V tile; keys are processed in tiles of 128. Twelve
+// warps:
+//   warp 8   TMA: both Q tiles once, then each key tile's K and V as
+//            16-token page pieces (128-byte swizzle) gathered through the
+//            block table, one piece per lane, into two-stage K and V rings
+//            with full/free barriers.
+//   warp 9   MMA (one lane) and the tensor-memory allocation: S_x = Q_x K^T
+//            (8 x 128x128x16, both operands K-major in shared memory) into
+//            tensor-memory columns [128x, 128x+128); O_x += P_x V with P_x
+//            read from tensor memory (bf16, over S_x's first 64 columns) and
+//            V MN-major in shared memory, into columns [256+128x, ...).
+//            After P_x.V_j it issues S_x for tile j+1 (the tensor core runs
+//            one thread's operations in order), so one query tile's softmax
+//            overlaps the other tile's multiplications.
+//   warps 0-3 / 4-7   softmax of query tile 0 / 1: thread r owns row r
+//            (tensor-memory lane r): row max, exp2, the running sum, bf16 P
+//            written back over the consumed S columns; O is rescaled in
+//            tensor memory only when a row's max grows by more than 2^8 (the
+//            result is exact for any reference max as long as O and the sum
+//            share it); the epilogue divides by the sum and writes bf16 rows.
+//   warps 10-11 idle (they give their registers to the softmax warpgroups).
 // All waits are bounded; a wait that runs out records PA_ERR_TIMEOUT, makes
 // every role leave its loop, drains outstanding copies and tensor-core work,
 // and frees the tensor memory.
@@ -60,6 +69,7 @@ struct PrefillArgs {
     const int32_t *context_lens;
     const int32_t *qsl;
     int n_chunks, total_q, H_q, H_kv, group, bs, NB, MB;
+    int window;  // > 0: query at position p sees keys p-window+1 .. p only
     float scale_log2;
     unsigned long long timeout_ns;
 };
@@ -224,7 +234,9 @@ __device__ __forceinline__ float ex2_poly(float x) {
 
 // POLY: every POLY-th pair of exponentials in a full (unmasked) tile is
 // computed with ex2_poly instead of the special-function unit (0 = none).
-template <int POLY>
+// WIN: the sliding-window build; without it the band logic folds away at
+// compile time and the causal kernel keeps its tighter code.
+template <int POLY, bool WIN>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
@@ -252,13 +264,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         return;
     }
     const int cached = ctx - C;
-    // rows and K/V tiles of each Q tile (a Q tile past the chunk has none)
+    // Rows of each Q tile (a Q tile past the chunk has none) and the K/V
+    // tiles [jlo_x, jhi_x) it needs: up to its last row's position, from its
+    // first row's band start. Key positions below the chunk's smallest band
+    // start (chunk_lo) are never needed: their blocks may have been freed.
     const int rows0 = min(kPfRows, C - row0);
     const int rows1 = max(0, min(kPfRows, C - row0 - kPfRows));
-    const int ntile0 = (cached + row0 + rows0 - 1) / kPfKeys + 1;
-    const int ntile1 = rows1 > 0 ? (cached + row0 + kPfRows + rows1 - 1) / kPfKeys + 1 : 0;
-    auto ntile = [&](int x) { return x == 0 ? ntile0 : ntile1; };
-    const int n_kv = max(ntile0, ntile1);
+    const int W = WIN ? a.window : 0;
+    const int chunk_lo = W > 0 ? max(0, cached - W + 1) : 0;
+    const int pf0 = cached + row0, pf1 = pf0 + kPfRows;  // first positions
+    const int jlo0 = (W > 0 ? max(0, pf0 - W + 1) : 0) / kPfKeys;
+    const int jlo1 = (W > 0 ? max(0, pf1 - W + 1) : 0) / kPfKeys;
+    const int jhi0 = (pf0 + rows0 - 1) / kPfKeys + 1;
+    const int jhi1 = rows1 > 0 ? (pf1 + rows1 - 1) / kPfKeys + 1 : jlo1;
+    auto jlo = [&](int x) { return x == 0 ? jlo0 : jlo1; };
+    auto jhi = [&](int x) { return x == 0 ? jhi0 : jhi1; };
+    auto active = [&](int x, int j) { return j >= jlo(x) && j < jhi(x); };
+    const int jmin = jlo0, jmax = max(jhi0, jhi1);  // K/V tiles this CTA streams
     const int kvh = h / a.group;
 
     if (threadIdx.x == 0) {
@@ -282,15 +304,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_alloc(smem_u32(&bars->tmem_base), 512);
         tmem_relinquish();
     }
-    // the chunk's block-table slice, checked once, into shared memory (the
-    // first kPfTblMax entries; a longer context reads the rest from global)
+    // the block-table slice this CTA streams, from its first key tile's
+    // block, checked once, into shared memory (kPfTblMax entries; a longer
+    // span reads the rest from global). Blocks wholly before chunk_lo are
+    // neither read nor checked.
     const int n_blk = (ctx + a.bs - 1) / a.bs;
+    const int blk0 = jmin * kPfKeys / a.bs, blk_lo = chunk_lo / a.bs;
     const int32_t *trow = a.block_tables + (size_t)c * a.MB;
-    for (int e = threadIdx.x; e < min(n_blk, kPfTblMax); e += kPfThreads) {
-        int id = __ldg(trow + e);
-        if (id < 0 || id >= a.NB) {
-            flag_error(PA_ERR_BAD_TABLE);
-            id = -1;
+    for (int e = threadIdx.x; e < min(n_blk - blk0, kPfTblMax); e += kPfThreads) {
+        int id = -1;
+        if (blk0 + e >= blk_lo) {
+            id = __ldg(trow + blk0 + e);
+            if (id < 0 || id >= a.NB) {
+                flag_error(PA_ERR_BAD_TABLE);
+                id = -1;
+            }
         }
         tbl[e] = id;
     }
@@ -314,10 +342,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j) {
             const int key = j * kPfKeys + s16 * 16;
             int id = -1;
-            if (lane < 16 && key < ctx) {
+            if (lane < 16 && key < ctx && (!WIN || key + 15 >= chunk_lo)) {
                 const int lb = key / a.bs;
-                if (lb < kPfTblMax) {
-                    id = tbl[lb];
+                if (lb - blk0 < kPfTblMax) {
+                    id = tbl[lb - blk0];
                 } else {
                     id = __ldg(trow + lb);
                     if (id < 0 || id >= a.NB) {
@@ -341,18 +369,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tma_load_3d(sQ + x * kPfTileBytes + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64,
                         h, q0 + row0 + x * kPfRows);
         }
-        int k_issued = 0, v_issued = 0;
-        for (int j = 0; j < n_kv; ++j) {
-            const int st = j % kPfStages;
-            const uint32_t use = j / kPfStages;
+        int k_issued = 0, v_issued = 0;  // counted from jmin
+        for (int j = jmin; j < jmax; ++j) {
+            const int st = (j - jmin) % kPfStages;
+            const uint32_t use = (j - jmin) / kPfStages;
             if (use > 0 && !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
                 break;
             issue(sK + st * kPfTileBytes, &tmk, &bars->k_full[st], j);
-            k_issued = j + 1;
+            k_issued = j - jmin + 1;
             if (use > 0 && !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
                 break;
             issue(sV + st * kPfTileBytes, &tmv, &bars->v_full[st], j);
-            v_issued = j + 1;
+            v_issued = j - jmin + 1;
         }
         if (bars->abort && lane == 0) {  // let copies already in flight land
             mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
@@ -369,8 +397,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             constexpr uint32_t kIdQK = f16_idesc(128, 128, false);
             constexpr uint32_t kIdPV = f16_idesc(128, 128, true);
             auto issue_s = [&](int x, int j) -> bool {  // S_x = Q_x K_j^T
-                const int st = j % kPfStages;
-                if (!pf_wait(bars, &bars->k_full[st], (j / kPfStages) & 1, a.timeout_ns, false))
+                const int st = (j - jmin) % kPfStages;
+                if (!pf_wait(bars, &bars->k_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
+                             false))
                     return false;
                 tc_fence_after();
                 const uint32_t q = sQ + x * kPfTileBytes, k = sK + st * kPfTileBytes;
@@ -384,9 +413,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 return true;
             };
             auto issue_pv = [&](int x, int j) -> bool {  // O_x += P_x V_j
-                const int st = j % kPfStages;
-                if (!pf_wait(bars, &bars->p_full[x], j & 1, a.timeout_ns, false)) return false;
-                if (!pf_wait(bars, &bars->v_full[st], (j / kPfStages) & 1, a.timeout_ns, false))
+                const int st = (j - jmin) % kPfStages;
+                if (!pf_wait(bars, &bars->p_full[x], (j - jlo(x)) & 1, a.timeout_ns, false))
+                    return false;
+                if (!pf_wait(bars, &bars->v_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
+                             false))
                     return false;
                 tc_fence_after();
                 const uint32_t v = sV + st * kPfTileBytes;
@@ -394,28 +425,30 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 for (int ks = 0; ks < 8; ++ks)
                     mma_ts(tmem + 256 + x * 128, tmem + x * 128 + ks * 8,
                            sw128_desc(v + ks * 2048, 16384, 1024), kIdPV,
-                           (j > 0 || ks > 0) ? 1u : 0u);
+                           (j > jlo(x) || ks > 0) ? 1u : 0u);
                 tc_commit(smem_u32(&bars->o_full[x]));
                 return true;
             };
             bool ok = pf_wait(bars, &bars->q_full, 0, a.timeout_ns, false);
-            // S for the first K tile of every Q tile, then per K/V tile j:
-            // P.V of each Q tile and, behind it in issue order (the tensor
-            // core runs one thread's operations in order, so S may reuse the
-            // P columns), S of the next tile
-            ok = ok && issue_s(0, 0);
-            if (ok && ntile1 > 0) ok = issue_s(1, 0);
+            // S of every Q tile that starts at the first K tile, then per K/V
+            // tile j: P.V of each Q tile that uses it and, behind it in issue
+            // order (the tensor core runs one thread's operations in order,
+            // so S may reuse the P columns), S of each Q tile that uses tile
+            // j+1 (a Q tile whose band starts one tile later starts there)
+#pragma unroll
+            for (int x = 0; x < kPfQTiles; ++x)
+                if (ok && active(x, jmin)) ok = issue_s(x, jmin);
             if (ok) tc_commit(smem_u32(&bars->k_free[0]));
-            for (int j = 0; ok && j < n_kv; ++j) {
+            for (int j = jmin; ok && j < jmax; ++j) {
 #pragma unroll
                 for (int x = 0; x < kPfQTiles; ++x) {
-                    if (!ok || j >= ntile(x)) continue;
-                    ok = issue_pv(x, j);
-                    if (ok && j + 1 < ntile(x)) ok = issue_s(x, j + 1);
+                    if (ok && active(x, j)) ok = issue_pv(x, j);
+                    if (ok && active(x, j + 1)) ok = issue_s(x, j + 1);
                 }
                 if (!ok) break;
-                if (j + 1 < n_kv) tc_commit(smem_u32(&bars->k_free[(j + 1) % kPfStages]));
-                tc_commit(smem_u32(&bars->v_free[j % kPfStages]));
+                if (j + 1 < jmax)
+                    tc_commit(smem_u32(&bars->k_free[(j + 1 - jmin) % kPfStages]));
+                tc_commit(smem_u32(&bars->v_free[(j - jmin) % kPfStages]));
             }
             // every tensor-core operation issued above completes before teardown
             tc_commit(smem_u32(&bars->fin));
@@ -430,19 +463,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int i = row0 + x * kPfRows + r;         // query index in the chunk
         const bool row_valid = i < C;
         const int pos = cached + min(i, C - 1);       // keys <= pos are visible
+        const int lo = W > 0 ? pos - W + 1 : 0;       // ... and keys >= lo
         const int pos_first = cached + row0 + x * kPfRows;  // smallest pos of the tile
+        const int lo_last = W > 0 ? pos_first + (x == 0 ? rows0 : rows1) - W : 0;  // largest lo
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + x * 128 + lane_off;
         const uint32_t tO = tmem + 256 + x * 128 + lane_off;
         const float sl2 = a.scale_log2;
-        const int nt = ntile(x);
+        const int j0 = jlo(x), j1 = jhi(x);
         // the warpgroup that first consumes the last K/V tile clears its
-        // rows past the context
-        const bool zeroes_tail = nt == n_kv && (x == 0 || ntile0 < n_kv);
+        // rows past the context; query tile 0, always the first consumer of
+        // the first K/V tile, clears its rows before chunk_lo
+        const bool zeroes_tail = j1 == jmax && (x == 0 || jhi0 < jmax);
         float m = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
-            if (!pf_wait(bars, &bars->s_full[x], j & 1, a.timeout_ns, true)) {
+        for (int j = j0; j < j1; ++j) {
+            if (!pf_wait(bars, &bars->s_full[x], (j - j0) & 1, a.timeout_ns, true)) {
                 ok = false;
                 break;
             }
@@ -454,11 +490,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
             tmem_ld_wait();
             const int key0 = j * kPfKeys;
-            const bool diag = key0 + kPfKeys - 1 > pos_first;  // some key masked for some row
+            // some key masked for some row: past the first row's position,
+            // or before the last row's band start
+            const bool diag = key0 + kPfKeys - 1 > pos_first || (WIN && key0 < lo_last);
             if (diag) {
 #pragma unroll
                 for (int e = 0; e < 128; ++e)
-                    if (key0 + e > pos) sv[e] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
+                    if (key0 + e > pos || (WIN && key0 + e < lo))
+                        sv[e] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
             }
             // the row's largest scaled score (raw max, or raw min for a
             // negative scale)
@@ -487,7 +526,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
             const float m_tile = isinf(ext) ? -INFINITY : ext * sl2;
             const float m_new = fmaxf(m, m_tile);
-            if (j == 0) {
+            if (j == j0) {
                 m = m_new;
             } else if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
                 // re-reference O and the sum to the new max
@@ -510,9 +549,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (diag) {
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
-                    const float p0 = key0 + 2 * e <= pos
+                    const int k0 = key0 + 2 * e;
+                    const float p0 = k0 <= pos && (!WIN || k0 >= lo)
                                          ? ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m)) : 0.f;
-                    const float p1 = key0 + 2 * e + 1 <= pos
+                    const float p1 = k0 + 1 <= pos && (!WIN || k0 + 1 >= lo)
                                          ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m)) : 0.f;
                     ls[e & 3] += p0 + p1;
                     pk[e] = pack_bf16x2(p0, p1);
@@ -521,7 +561,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
                     float p0, p1;
-                    if (POLY > 0 && e % POLY == POLY - 1) {
+                    if (POLY > 0 && e % (POLY > 0 ? POLY : 1) == POLY - 1) {
                         p0 = ex2_poly(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m));
                         p1 = ex2_poly(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m));
                     } else {
@@ -536,18 +576,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
             tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
             tmem_st_wait();
-            if (zeroes_tail && j == nt - 1 && key0 + kPfKeys > ctx) {
-                // V rows past the context hold stale or unloaded data: zero
-                // them so that P = 0 cannot meet a NaN there
-                const int st = j % kPfStages;
-                if (!pf_wait(bars, &bars->v_full[st], (j / kPfStages) & 1, a.timeout_ns, true)) {
+            // V rows past the context, or before chunk_lo, hold stale or
+            // unloaded data: zero them so that P = 0 cannot meet a NaN there
+            const int z0 = WIN && x == 0 && j == jmin ? max(0, chunk_lo - key0) : 0;
+            const int z1 = zeroes_tail && j == j1 - 1 ? min(kPfKeys, ctx - key0) : kPfKeys;
+            if (z0 > 0 || z1 < kPfKeys) {
+                const int st = (j - jmin) % kPfStages;
+                if (!pf_wait(bars, &bars->v_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
+                             true)) {
                     ok = false;
                     break;
                 }
-                const int vr = ctx - key0;
                 const uint32_t vb = sV + st * kPfTileBytes;
-                for (int e = r; e < (kPfKeys - vr) * 16; e += 128) {
-                    const int row = vr + e / 16, u = e % 16;
+                const int nz = z0 + (kPfKeys - z1);  // rows [0, z0) and [z1, 128)
+                for (int e = r; e < nz * 16; e += 128) {
+                    const int zr = e / 16, u = e % 16;
+                    const int row = zr < z0 ? zr : z1 + (zr - z0);
                     const uint32_t addr = vb + (u / 8) * 16384 + row * 128 + (u % 8) * 16;
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
                                  : "memory");
@@ -557,7 +601,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tc_fence_before();
             mbar_arrive(smem_u32(&bars->p_full[x]));
         }
-        if (ok && nt > 0 && pf_wait(bars, &bars->o_full[x], (nt - 1) & 1, a.timeout_ns, true)) {
+        if (ok && j1 > j0 &&
+            pf_wait(bars, &bars->o_full[x], (j1 - j0 - 1) & 1, a.timeout_ns, true)) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + h) * 128;

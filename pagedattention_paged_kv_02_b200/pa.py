@@ -26,7 +26,8 @@ EXPORTS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_partit
            "pa_decode", "pa_prefill_chunk", "pa_check_tables", "pa_device_error",
            "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
            "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
-           "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window")
+           "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window",
+           "pa_prefill_chunk_sliding_window")
 
 
 class PAError(RuntimeError):
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_static_workspace.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I,
                                                  I, P]
         L.pa_prefill_chunk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P]
+        L.pa_prefill_chunk_sliding_window.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I,
+                                                      I, I, F, I, I, P]
         L.pa_decode_sliding_window.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,
                                                P, SZ, I, P]
         L.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, I, P]
@@ -71,8 +74,8 @@ def lib() -> ctypes.CDLL:
         for f in ("pa_reshape_and_cache", "pa_decode", "pa_decode_static_workspace",
                   "pa_prefill_chunk", "pa_check_tables", "pa_copy_blocks", "pa_swap_blocks",
                   "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window",
-                  "pa_device_error", "pa_selftest_bounded_wait", "pa_decode_partition_tokens",
-                  "pa_version"):
+                  "pa_prefill_chunk_sliding_window", "pa_device_error",
+                  "pa_selftest_bounded_wait", "pa_decode_partition_tokens", "pa_version"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -200,9 +203,7 @@ def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_l
           float(scale), int(partition_size), _dt(q), _stream(stream))
 
 
-def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
-                     max_query_len: int, scale: float, stream=None) -> None:
-    """Chunked prefill into ``out`` [total_q, H_q, D]."""
+def _prefill_args(out, q, k_cache, block_tables, context_lens, query_start_loc):
     for t, n in ((block_tables, "block_tables"), (context_lens, "context_lens"),
                  (query_start_loc, "query_start_loc")):
         _check_int(t, torch.int32, n)
@@ -210,11 +211,30 @@ def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query
     NB, H_kv, bs, D2 = k_cache.shape
     if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
         raise ValueError("out must match q; caches must share head_dim")
-    n_chunks = query_start_loc.numel() - 1
-    MB = block_tables.shape[1]
+    return query_start_loc.numel() - 1, total_q, H_q, H_kv, D, bs, NB, block_tables.shape[1]
+
+
+def pa_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                     max_query_len: int, scale: float, stream=None) -> None:
+    """Chunked prefill into ``out`` [total_q, H_q, D]."""
+    n_chunks, total_q, H_q, H_kv, D, bs, NB, MB = _prefill_args(
+        out, q, k_cache, block_tables, context_lens, query_start_loc)
     _call("pa_prefill_chunk", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
           _p(context_lens), _p(query_start_loc), n_chunks, total_q, int(max_query_len), H_q,
           H_kv, D, bs, NB, MB, float(scale), _dt(q), _stream(stream))
+
+
+def pa_prefill_chunk_sliding_window(out, q, k_cache, v_cache, block_tables, context_lens,
+                                    query_start_loc, max_query_len: int, scale: float,
+                                    sliding_window: int, stream=None) -> None:
+    """Chunked prefill where the query at position p sees positions
+    p - sliding_window + 1 .. p only."""
+    n_chunks, total_q, H_q, H_kv, D, bs, NB, MB = _prefill_args(
+        out, q, k_cache, block_tables, context_lens, query_start_loc)
+    _call("pa_prefill_chunk_sliding_window", _p(out), _p(q), _p(k_cache), _p(v_cache),
+          _p(block_tables), _p(context_lens), _p(query_start_loc), n_chunks, total_q,
+          int(max_query_len), H_q, H_kv, D, bs, NB, MB, float(scale), int(sliding_window),
+          _dt(q), _stream(stream))
 
 
 def _fp8_pool(k_cache, v_cache, k_scale, v_scale):
@@ -353,7 +373,9 @@ def prepare_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping) -> Pre
 
 def prepare_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len: int,
                    scale: float, partition_size: int = 0,
-                   workspace: Optional[torch.Tensor] = None) -> Prepared:
+                   workspace: Optional[torch.Tensor] = None,
+                   sliding_window: int = 0) -> Prepared:
+    """``pa_decode`` (or, with ``sliding_window`` > 0, ``pa_decode_sliding_window``)."""
     _check_int(block_tables, torch.int32, "block_tables")
     _check_int(context_lens, torch.int32, "context_lens")
     B, H_q, D = q.shape
@@ -361,14 +383,18 @@ def prepare_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_con
     if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
         raise ValueError("out must match q; caches must share head_dim")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    return Prepared("pa_decode", (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
-                                  _p(context_lens), B, H_q, H_kv, D, bs, NB,
-                                  block_tables.shape[1], int(max_context_len), float(scale),
-                                  int(partition_size), _p(workspace), ws_bytes, _dt(q)))
+    head = (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens), B,
+            H_q, H_kv, D, bs, NB, block_tables.shape[1], int(max_context_len), float(scale))
+    tail = (int(partition_size), _p(workspace), ws_bytes, _dt(q))
+    if sliding_window > 0:
+        return Prepared("pa_decode_sliding_window", head + (int(sliding_window),) + tail)
+    return Prepared("pa_decode", head + tail)
 
 
 def prepare_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
-                          max_query_len: int, scale: float) -> Prepared:
+                          max_query_len: int, scale: float, sliding_window: int = 0) -> Prepared:
+    """``pa_prefill_chunk`` (or, with ``sliding_window`` > 0,
+    ``pa_prefill_chunk_sliding_window``)."""
     for t, n in ((block_tables, "block_tables"), (context_lens, "context_lens"),
                  (query_start_loc, "query_start_loc")):
         _check_int(t, torch.int32, n)
@@ -376,11 +402,13 @@ def prepare_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, 
     NB, H_kv, bs, D2 = k_cache.shape
     if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
         raise ValueError("out must match q; caches must share head_dim")
-    return Prepared("pa_prefill_chunk", (_p(out), _p(q), _p(k_cache), _p(v_cache),
-                                         _p(block_tables), _p(context_lens), _p(query_start_loc),
-                                         query_start_loc.numel() - 1, total_q, int(max_query_len),
-                                         H_q, H_kv, D, bs, NB, block_tables.shape[1],
-                                         float(scale), _dt(q)))
+    head = (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+            _p(query_start_loc), query_start_loc.numel() - 1, total_q, int(max_query_len), H_q,
+            H_kv, D, bs, NB, block_tables.shape[1], float(scale))
+    if sliding_window > 0:
+        return Prepared("pa_prefill_chunk_sliding_window",
+                        head + (int(sliding_window), _dt(q)))
+    return Prepared("pa_prefill_chunk", head + (_dt(q),))
 
 
 def prepare_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale,

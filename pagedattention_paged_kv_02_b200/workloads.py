@@ -71,6 +71,7 @@ class Batch:
     partition_size: int = 0
     k_scale: Optional[torch.Tensor] = None  # FP8 pools: float32 [H_kv] per-head scales
     v_scale: Optional[torch.Tensor] = None
+    sliding_window: int = 0  # > 0: every query sees only its last sliding_window positions
 
     @property
     def num_blocks(self) -> int:

@@ -146,6 +146,24 @@ def test_prefill_host_checks(L):
     assert f(*b) == pa.PA_OK
 
 
+def test_prefill_window_host_checks(L):
+    from pagedattention_paged_kv_02_b200 import pa
+    f = L.pa_prefill_chunk_sliding_window
+    # as pa_prefill_chunk with the window before dtype
+    base = [FAKE] * 7 + [2, 1024, 512, 32, 8, 128, 16, 64, 64, 0.1, 256, 1, None]
+    assert len(base) == 20
+    for w in (0, -5):
+        b = list(base)
+        b[17] = w
+        assert f(*b) == pa.PA_ERR_INVALID_ARG
+    b = list(base)
+    b[18] = 0
+    assert f(*b) == pa.PA_ERR_UNSUPPORTED  # fp32 has no tensor-core path
+    b = list(base)
+    b[7] = 0
+    assert f(*b) == pa.PA_OK
+
+
 def test_service_host_checks(L):
     from pagedattention_paged_kv_02_b200 import pa
     bad = ctypes.c_int(-1)
