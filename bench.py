@@ -397,7 +397,9 @@ def run_ours(args, rank, world):
     clk = clocks.stop()
     barrier(world)
     ms_local = t0.elapsed_time(t1) / K
-    dom_ms = statistics.fmean(a.elapsed_time(b) for a, b in evs)
+    dom_all = sorted(a.elapsed_time(b) for a, b in evs)
+    dom_ms = statistics.fmean(dom_all)
+    pct = lambda q: dom_all[min(len(dom_all) - 1, int(q * len(dom_all)))]
 
     units = dbytes if r.dominant == "decode" else pflops
     total_units, ms = aggregate(units, ms_local, world, dev)
@@ -495,10 +497,12 @@ def run_ours(args, rank, world):
             roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                     "unit": "GB/s", "frac": round(achieved / hbm, 4),
                     "peak_basis": f"{basis} hbm_gbs",
-                    "kernel": "pa_decode (decode_split + decode_reduce)",
+                    "kernel": ("pa_decode_fp8 (decode_split_e4m3 + merge)" if batch.fp8 else
+                               "pa_decode (decode_split + merge)"),
                     "alg_bytes_per_launch": dbytes,
                     "traffic": profiled_traffic(f"decode_{args.workload}{wtag}.md",
-                                                DECODE_SOURCES)}
+                                                DECODE_FP8_SOURCES if batch.fp8
+                                                else DECODE_SOURCES)}
         else:
             value = dbytes_total / (ms * 1e-3) / 1e9
             unit = "GB/s"
@@ -526,6 +530,8 @@ def run_ours(args, rank, world):
                     "ms_per_step": round(e2e_ms, 5)},
             "gpu_launches": K * r.launches_per_step(),
             "clocks": clk,
+            "dominant_call_ms": {"mean": round(dom_ms, 5), "p10": round(pct(0.1), 5),
+                                 "p50": round(pct(0.5), 5), "p90": round(pct(0.9), 5)},
         }
         if r.dominant != "decode":
             line["prefill_tflops"] = round(pflops * world / (ms * 1e-3) / 1e12, 1)
@@ -542,6 +548,7 @@ DECODE_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/decode.cuh",
                   "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
 PREFILL_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/prefill.cuh",
                    "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
+DECODE_FP8_SOURCES = DECODE_SOURCES + ["pagedattention_paged_kv_02_b200/csrc/decode_fp8.cuh"]
 
 
 def workload_config(batch, name, world, r=None):

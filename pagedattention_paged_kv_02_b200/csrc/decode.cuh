@@ -1,4 +1,5 @@
-// decode.cuh -- paged decode attention: split-KV kernel and log-sum-exp merge.
+// decode.cuh -- paged decode attention: the split-KV kernel (the merge of
+// its partials is in decode_merge.cuh).
 //
 // What is computed (page "字节跳动 AI Infra (2)", question "KV Cache原理与优化"):
 // for each sequence b and query head h, softmax(scale * q . K^T) V over the
@@ -74,15 +75,10 @@ __device__ __forceinline__ int clamped_ctx(const DecodeArgs &a, int b, bool repo
 }
 
 // Programmatic dependent launch: a split CTA lets the merge kernel queued
-// behind it be scheduled as soon as every split CTA has started (its CTAs
-// then fill the SMs the split grid's tail leaves idle); the merge kernel
-// waits for the split grid to finish, with its writes visible, before it
-// reads any partial.
+// behind it (decode_merge.cuh) be scheduled as soon as every split CTA has
+// started; its CTAs then fill the SMs the split grid's tail leaves idle.
 __device__ __forceinline__ void allow_dependent_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void wait_for_primary_grid() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Shared-memory plan of a split CTA: the stage ring (reused after the main
@@ -557,120 +553,6 @@ __global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constan
     }
     __syncthreads();
     decode_epilogue<D, NW, HT, float>(a, red_o, red_m, red_l, b, h0, nh, s, n_splits);
-}
-
-// ------------------------------------------------------------- LSE merge
-// out = sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M), M = max_s lse_s, for
-// every (sequence, query head) with more than one partition.
-//
-// Few partitions per head (S_max <= kWarpMergeMax): one warp per
-// (sequence, head), eight per CTA, each lane owning D/32 dimensions and
-// walking the partitions in order; heads with one partition cost a warp a
-// length read.
-constexpr int kWarpMergeMax = 16;
-
-template <int D, typename OutT>
-__global__ void __launch_bounds__(256) decode_reduce_warp(const __grid_constant__ DecodeArgs a) {
-    constexpr int VEC = D / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x * 8 + warp;
-    if (bh >= a.num_seqs * a.H_q) return;
-    const int b = bh / a.H_q;
-    const int ctx = clamped_ctx(a, b, false);
-    const int n = (ctx - span_base(a, ctx) + a.P - 1) / a.P;
-    if (n <= 1) return;
-    wait_for_primary_grid();
-    const float *lse = a.part_lse + (size_t)bh * a.S_max;
-    const float *po = a.part_o + (size_t)bh * a.S_max * D + lane * VEC;
-    float M = lane < n ? __ldcg(lse + lane) : -INFINITY;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float acc[VEC];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-    float W = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < n; ++s) {
-            const float w = exp2f(__ldcg(lse + s) - M);
-            W += w;
-            if constexpr (VEC == 4) {
-                const float4 x = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)s * D));
-                acc[0] = fmaf(w, x.x, acc[0]);
-                acc[1] = fmaf(w, x.y, acc[1]);
-                acc[2] = fmaf(w, x.z, acc[2]);
-                acc[3] = fmaf(w, x.w, acc[3]);
-            } else {
-                const float2 x = __ldcg(reinterpret_cast<const float2 *>(po + (size_t)s * D));
-                acc[0] = fmaf(w, x.x, acc[0]);
-                acc[1] = fmaf(w, x.y, acc[1]);
-            }
-        }
-    }
-    OutT *dst = reinterpret_cast<OutT *>(a.out) + (size_t)bh * D + lane * VEC;
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) dst[v] = OutT(W > 0.f ? acc[v] / W : 0.f);
-}
-
-// Many partitions per head: one CTA (4 warps) per (sequence, head), the
-// warps taking every 4th partition.
-template <int D, typename OutT>
-__global__ void __launch_bounds__(128) decode_reduce(const __grid_constant__ DecodeArgs a) {
-    constexpr int NWR = 4;
-    constexpr int VEC = D / 32;
-    const int bh = blockIdx.x;
-    const int b = bh / a.H_q;
-    const int ctx = clamped_ctx(a, b, false);
-    const int n = (ctx - span_base(a, ctx) + a.P - 1) / a.P;
-    if (n <= 1) return;
-    wait_for_primary_grid();
-    const float *lse = a.part_lse + (size_t)bh * a.S_max;
-    const float *po = a.part_o + (size_t)bh * a.S_max * D;
-    __shared__ float red[NWR][D + 1];
-    __shared__ float wsum[NWR];
-    __shared__ float smax[NWR];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    float M = -INFINITY;
-    for (int s = threadIdx.x; s < n; s += 128) M = fmaxf(M, lse[s]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) smax[warp] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(smax[0], smax[1]), fmaxf(smax[2], smax[3]));
-
-    float acc[VEC];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-    float W = 0.f;
-    if (M != -INFINITY) {
-        for (int s = warp; s < n; s += NWR) {
-            const float w = exp2f(lse[s] - M);
-            W += w;
-            const float *src = po + (size_t)s * D + lane * VEC;
-            if constexpr (VEC == 4) {
-                const float4 x = *reinterpret_cast<const float4 *>(src);
-                acc[0] = fmaf(w, x.x, acc[0]);
-                acc[1] = fmaf(w, x.y, acc[1]);
-                acc[2] = fmaf(w, x.z, acc[2]);
-                acc[3] = fmaf(w, x.w, acc[3]);
-            } else {
-                const float2 x = *reinterpret_cast<const float2 *>(src);
-                acc[0] = fmaf(w, x.x, acc[0]);
-                acc[1] = fmaf(w, x.y, acc[1]);
-            }
-        }
-    }
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) red[warp][lane * VEC + v] = acc[v];
-    if (lane == 0) wsum[warp] = W;
-    __syncthreads();
-    if (threadIdx.x < D) {
-        const int d = threadIdx.x;
-        const float Wt = wsum[0] + wsum[1] + wsum[2] + wsum[3];
-        const float x = red[0][d] + red[1][d] + red[2][d] + red[3][d];
-        const float r = Wt > 0.f ? x / Wt : 0.f;
-        reinterpret_cast<OutT *>(a.out)[(size_t)bh * D + d] = OutT(r);
-    }
 }
 
 }  // namespace pa

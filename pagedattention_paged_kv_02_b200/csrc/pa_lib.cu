@@ -18,6 +18,7 @@
 #include "pa_device.cuh"
 #include "reshape_and_cache.cuh"
 #include "decode.cuh"
+#include "decode_merge.cuh"
 #include "decode_fp8.cuh"
 #include "prefill.cuh"
 #include "blocks.cuh"
@@ -248,7 +249,7 @@ pa_status launch_reduce(const DecodeArgs &a, cudaStream_t st) {
             return PA_ERR_CUDA;
     } else {
         cfg.gridDim = dim3((unsigned)heads);
-        cfg.blockDim = dim3(128);
+        cfg.blockDim = dim3(512);
         if (cudaLaunchKernelEx(&cfg, decode_reduce<D, OutT>, a) != cudaSuccess)
             return PA_ERR_CUDA;
     }
