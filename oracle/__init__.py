@@ -86,6 +86,12 @@ def _load():
             lib.oracle_decode_window.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, I64,
                                                  D, I, P]
             lib.oracle_e4m3_encode_array.argtypes = [P, P, I64]
+            lib.oracle_int8_encode_array.argtypes = [P, P, I64]
+            lib.oracle_int8_encode_array.restype = None
+            lib.oracle_reshape_and_cache_int8.argtypes = [P, P, I, P, P, P, I64, I, I, I, I64, P,
+                                                          P]
+            lib.oracle_decode_int8.argtypes = [P, P, P, I, P, P, P, P, P, P, I, I, I, I, I, I,
+                                               I64, D, P]
             lib.oracle_e4m3_encode_array.restype = None
             lib.oracle_e4m3_decode_array.argtypes = [P, P, I64]
             lib.oracle_e4m3_decode_array.restype = None
@@ -95,7 +101,8 @@ def _load():
                                                I64, D, P]
             for f in ("oracle_reshape_and_cache", "oracle_decode", "oracle_decode_partials",
                       "oracle_prefill", "oracle_copy_blocks", "oracle_reshape_and_cache_e4m3",
-                      "oracle_decode_e4m3", "oracle_decode_window", "oracle_prefill_window"):
+                      "oracle_decode_e4m3", "oracle_decode_window", "oracle_prefill_window",
+                      "oracle_reshape_and_cache_int8", "oracle_decode_int8"):
                 getattr(lib, f).restype = I
             _lib = lib
     return _lib
@@ -357,6 +364,54 @@ def decode_e4m3(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_len
                                     _ptr(block_tables), _ptr(context_lens), B, H_q, H_kv, D, bs,
                                     MB, NB, float(scale), _ptr(sel))
     _check(rc, "decode_e4m3")
+    return out, lse
+
+
+def int8_encode(q) -> torch.Tensor:
+    """INT8 codes (int8) of fp32 quotients x / scale: nearest integer, ties to
+    even, saturated to [-127, 127], NaN to 0."""
+    q = _cpu(torch.as_tensor(q, dtype=torch.float32))
+    out = torch.empty(q.shape, dtype=torch.int8)
+    _load().oracle_int8_encode_array(_ptr(q), _ptr(out), q.numel())
+    return out
+
+
+def reshape_and_cache_int8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale) -> None:
+    """The append step into int8 caches: code of fp32(x) / scale[h]."""
+    key, value = _cpu(key), _cpu(value)
+    slot_mapping = _cpu(slot_mapping, torch.int64)
+    k_scale = _cpu(k_scale, torch.float32)
+    v_scale = _cpu(v_scale, torch.float32)
+    for c in (k_cache, v_cache):
+        if not c.is_contiguous() or c.device.type != "cpu" or c.dtype != torch.int8:
+            raise ValueError("caches must be contiguous int8 host tensors")
+    NB, H_kv, bs, D = k_cache.shape
+    T = slot_mapping.numel()
+    rc = _load().oracle_reshape_and_cache_int8(_ptr(key), _ptr(value), _dtype_code(key),
+                                               _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                               T, H_kv, D, bs, NB, _ptr(k_scale), _ptr(v_scale))
+    _check(rc, "reshape_and_cache_int8")
+
+
+def decode_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                select=None):
+    """fp64 paged decode over int8 caches with per-K/V-head scales."""
+    q = _cpu(q)
+    k_cache, v_cache = _cpu(k_cache, torch.int8), _cpu(v_cache, torch.int8)
+    k_scale, v_scale = _cpu(k_scale, torch.float32), _cpu(v_scale, torch.float32)
+    block_tables = _cpu(block_tables, torch.int32)
+    context_lens = _cpu(context_lens, torch.int32)
+    B, H_q, D = q.shape
+    NB, H_kv, bs, _ = k_cache.shape
+    MB = block_tables.shape[1]
+    sel = _select(select, B * H_q)
+    out = torch.zeros(B, H_q, D, dtype=torch.float64)
+    lse = torch.full((B, H_q), float("-inf"), dtype=torch.float64)
+    rc = _load().oracle_decode_int8(_ptr(out), _ptr(lse), _ptr(q), _dtype_code(q), _ptr(k_cache),
+                                    _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                    _ptr(block_tables), _ptr(context_lens), B, H_q, H_kv, D, bs,
+                                    MB, NB, float(scale), _ptr(sel))
+    _check(rc, "decode_int8")
     return out, lse
 
 

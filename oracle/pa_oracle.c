@@ -25,7 +25,8 @@
  *  [Q8]  page "字节跳动 AI Infra (2)", optimisation table, row "KV量化(INT8)"
  *        (store K/V in low precision, halving the cache), and page
  *        "LLM推理优化", section 1.3 (quantise K/V from FP16 to INT8/INT4):
- *        here FP8 E4M3 codes with one scale per K/V head, value = code*scale.
+ *        here INT8 codes or FP8 E4M3 codes, one scale per K/V head,
+ *        value = code * scale.
  *  [SW]  page "LLM推理优化", section 2.3 (flash_attn_func window_size) and page
  *        "vLLM框架是怎么做推理加速的", 追问 3 (sliding window attention): a query
  *        sees only the last `window` positions up to its own.
@@ -61,7 +62,7 @@
 #include <omp.h>
 #endif
 
-enum { OR_F32 = 0, OR_BF16 = 1, OR_E4M3 = 2 };
+enum { OR_F32 = 0, OR_BF16 = 1, OR_E4M3 = 2, OR_I8 = 3 };
 enum { OR_OK = 0, OR_BAD_SLOT = 1, OR_BAD_BLOCK = 2, OR_BAD_ARG = 3, OR_NO_MEM = 4 };
 
 /* [Q8] value of an FP8 E4M3 code (1 sign bit, 4 exponent bits with bias 7,
@@ -103,13 +104,27 @@ uint8_t oracle_e4m3_encode(float x)
 
 double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
 
+/* [Q8] INT8 code of q, an fp32 quotient x / scale: the nearest integer, ties
+ * to even (the default rounding mode of nearbyint), saturated to the
+ * symmetric range [-127, 127]; NaN gives 0. */
+int8_t oracle_int8_encode(float q)
+{
+    if (isnan(q)) return 0;
+    double r = nearbyint((double)q);
+    if (r > 127.0) r = 127.0;
+    if (r < -127.0) r = -127.0;
+    return (int8_t)r;
+}
+
 /* A stored element, widened exactly to double. bf16 is the top half of an
  * IEEE binary32, so shifting its 16 bits up gives the same number as a float.
- * An E4M3 code is its value times the K/V head's scale (exact in double). */
+ * An E4M3 or INT8 code is its value times the K/V head's scale (exact in
+ * double). */
 static double stored_scaled(const void *base, int64_t i, int dtype, double scale)
 {
     if (dtype == OR_F32) return (double)((const float *)base)[i];
     if (dtype == OR_E4M3) return e4m3_value(((const uint8_t *)base)[i]) * scale;
+    if (dtype == OR_I8) return (double)((const int8_t *)base)[i] * scale;
     uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
@@ -131,7 +146,7 @@ typedef struct {
     int H_kv, D, bs;
     int64_t NB;
     int kv_head;
-    double k_scale, v_scale; /* E4M3 caches: value = code * scale */
+    double k_scale, v_scale; /* 8-bit caches: value = code * scale */
 } paged_seq;
 
 /* [PG] element index of K/V[position j][dim 0] of this sequence and head:
@@ -453,17 +468,16 @@ int oracle_copy_blocks(const void *src_k, const void *src_v, int64_t src_blocks,
     return OR_OK;
 }
 
-/* [Q8]+[KV] the append step into an E4M3 cache: each element of the new
+/* [Q8]+[KV] the append step into an 8-bit cache: each element of the new
  * token's K (V) row for K/V head h is stored as the code of the fp32 quotient
  * x / k_scale[h] (x / v_scale[h]), computed as an IEEE single-precision
- * division and encoded by oracle_e4m3_encode. key/value are fp32 or bf16
- * (dtype); caches hold one byte per element. Slots as in
- * oracle_reshape_and_cache. */
-int oracle_reshape_and_cache_e4m3(const void *key, const void *value, int dtype, uint8_t *k_cache,
-                                  uint8_t *v_cache, const int64_t *slot_mapping,
-                                  int64_t num_tokens, int num_kv_heads, int head_dim,
-                                  int block_size, int64_t num_blocks, const float *k_scale,
-                                  const float *v_scale)
+ * division and encoded by oracle_e4m3_encode (fmt OR_E4M3) or
+ * oracle_int8_encode (fmt OR_I8). key/value are fp32 or bf16 (dtype); caches
+ * hold one byte per element. Slots as in oracle_reshape_and_cache. */
+static int reshape_q8(const void *key, const void *value, int dtype, uint8_t *k_cache,
+                      uint8_t *v_cache, const int64_t *slot_mapping, int64_t num_tokens,
+                      int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                      const float *k_scale, const float *v_scale, int fmt)
 {
     if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
         return OR_BAD_ARG;
@@ -481,22 +495,49 @@ int oracle_reshape_and_cache_e4m3(const void *key, const void *value, int dtype,
                 float xv = (float)stored(value, src + d, dtype);
                 float qk = xk / k_scale[h];
                 float qv = xv / v_scale[h];
-                k_cache[dst + d] = oracle_e4m3_encode(qk);
-                v_cache[dst + d] = oracle_e4m3_encode(qv);
+                if (fmt == OR_I8) {
+                    k_cache[dst + d] = (uint8_t)oracle_int8_encode(qk);
+                    v_cache[dst + d] = (uint8_t)oracle_int8_encode(qv);
+                } else {
+                    k_cache[dst + d] = oracle_e4m3_encode(qk);
+                    v_cache[dst + d] = oracle_e4m3_encode(qv);
+                }
             }
         }
     }
     return OR_OK;
 }
 
-/* [KV]+[PG]+[GQA]+[Q8] decode over an E4M3 cache: as oracle_decode, with
- * q of dtype q_dtype and every cached element equal to its code's value times
- * the K/V head's scale (k_scale / v_scale, one per K/V head). */
-int oracle_decode_e4m3(double *out, double *lse, const void *q, int q_dtype, const uint8_t *k_cache,
-                       const uint8_t *v_cache, const float *k_scale, const float *v_scale,
-                       const int32_t *block_tables, const int32_t *context_lens, int B, int H_q,
-                       int H_kv, int D, int bs, int MB, int64_t NB, double scale,
-                       const uint8_t *select)
+int oracle_reshape_and_cache_e4m3(const void *key, const void *value, int dtype, uint8_t *k_cache,
+                                  uint8_t *v_cache, const int64_t *slot_mapping,
+                                  int64_t num_tokens, int num_kv_heads, int head_dim,
+                                  int block_size, int64_t num_blocks, const float *k_scale,
+                                  const float *v_scale)
+{
+    return reshape_q8(key, value, dtype, k_cache, v_cache, slot_mapping, num_tokens,
+                      num_kv_heads, head_dim, block_size, num_blocks, k_scale, v_scale, OR_E4M3);
+}
+
+int oracle_reshape_and_cache_int8(const void *key, const void *value, int dtype, int8_t *k_cache,
+                                  int8_t *v_cache, const int64_t *slot_mapping,
+                                  int64_t num_tokens, int num_kv_heads, int head_dim,
+                                  int block_size, int64_t num_blocks, const float *k_scale,
+                                  const float *v_scale)
+{
+    return reshape_q8(key, value, dtype, (uint8_t *)k_cache, (uint8_t *)v_cache, slot_mapping,
+                      num_tokens, num_kv_heads, head_dim, block_size, num_blocks, k_scale,
+                      v_scale, OR_I8);
+}
+
+/* [KV]+[PG]+[GQA]+[Q8] decode over an 8-bit cache (fmt OR_E4M3 or OR_I8): as
+ * oracle_decode, with q of dtype q_dtype and every cached element equal to
+ * its code's value times the K/V head's scale (k_scale / v_scale, one per K/V
+ * head). */
+static int decode_q8(double *out, double *lse, const void *q, int q_dtype, const void *k_cache,
+                     const void *v_cache, const float *k_scale, const float *v_scale,
+                     const int32_t *block_tables, const int32_t *context_lens, int B, int H_q,
+                     int H_kv, int D, int bs, int MB, int64_t NB, double scale,
+                     const uint8_t *select, int fmt)
 {
     int rc = check_heads(H_q, H_kv, D, bs, MB, NB);
     if (rc) return rc;
@@ -509,7 +550,7 @@ int oracle_decode_e4m3(double *out, double *lse, const void *q, int q_dtype, con
         if (select && !select[bh]) continue;
         int b = (int)(bh / H_q), h = (int)(bh % H_q);
         int kvh = h / group;
-        paged_seq s = {k_cache, v_cache, OR_E4M3, block_tables + (int64_t)b * MB, MB,
+        paged_seq s = {k_cache, v_cache, fmt, block_tables + (int64_t)b * MB, MB,
                        H_kv, D, bs, NB, kvh, (double)k_scale[kvh], (double)v_scale[kvh]};
         double *qv = malloc(sizeof(double) * D);
         double *sbuf = malloc(sizeof(double) * (context_lens[b] > 0 ? context_lens[b] : 1));
@@ -530,7 +571,32 @@ int oracle_decode_e4m3(double *out, double *lse, const void *q, int q_dtype, con
 }
 
 
+int oracle_decode_e4m3(double *out, double *lse, const void *q, int q_dtype, const uint8_t *k_cache,
+                       const uint8_t *v_cache, const float *k_scale, const float *v_scale,
+                       const int32_t *block_tables, const int32_t *context_lens, int B, int H_q,
+                       int H_kv, int D, int bs, int MB, int64_t NB, double scale,
+                       const uint8_t *select)
+{
+    return decode_q8(out, lse, q, q_dtype, k_cache, v_cache, k_scale, v_scale, block_tables,
+                     context_lens, B, H_q, H_kv, D, bs, MB, NB, scale, select, OR_E4M3);
+}
+
+int oracle_decode_int8(double *out, double *lse, const void *q, int q_dtype, const int8_t *k_cache,
+                       const int8_t *v_cache, const float *k_scale, const float *v_scale,
+                       const int32_t *block_tables, const int32_t *context_lens, int B, int H_q,
+                       int H_kv, int D, int bs, int MB, int64_t NB, double scale,
+                       const uint8_t *select)
+{
+    return decode_q8(out, lse, q, q_dtype, k_cache, v_cache, k_scale, v_scale, block_tables,
+                     context_lens, B, H_q, H_kv, D, bs, MB, NB, scale, select, OR_I8);
+}
+
 /* [Q8] element-wise helpers over arrays (for tests and fixtures). */
+void oracle_int8_encode_array(const float *q, int8_t *codes, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) codes[i] = oracle_int8_encode(q[i]);
+}
+
 void oracle_e4m3_encode_array(const float *x, uint8_t *codes, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i) codes[i] = oracle_e4m3_encode(x[i]);

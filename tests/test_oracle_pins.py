@@ -560,6 +560,71 @@ def test_e4m3_decode_equals_decode_of_dequantized_cache():
 
 
 # ---------------------------------------------------------------------------
+# INT8 KV cache
+# ---------------------------------------------------------------------------
+def test_int8_encode_special_values():
+    """Halfway cases go to the even integer; integers stay; the range is the
+    symmetric [-127, 127]; NaN encodes as 0."""
+    q = torch.tensor([0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 126.5, -126.5, 3.0, -7.0, 0.49999997,
+                      127.0, 127.49, 128.0, 1e30, float("inf"), -127.6, -1e30, float("-inf"),
+                      float("nan"), -0.0])
+    want = [0, 2, 2, 0, -2, -2, 126, -126, 3, -7, 0, 127, 127, 127, 127, 127, -127, -127, -127,
+            0, 0]
+    assert oracle.int8_encode(q).tolist() == want
+
+
+def test_int8_encode_is_nearest_integer():
+    """Over a dense grid of fp32 quotients every code is an integer within
+    1/2 of the quotient, and the encoding never decreases."""
+    q = torch.arange(-130 * 256, 130 * 256 + 1, dtype=torch.float32) / 256
+    c = oracle.int8_encode(q).double()
+    inside = q.abs() <= 127
+    assert torch.all((c[inside] - q[inside].double()).abs() <= 0.5)
+    assert torch.all(c[~inside].abs() == 127)
+    assert torch.all(c[1:] >= c[:-1])
+
+
+def test_int8_reshape_is_divide_then_encode():
+    g = torch.Generator().manual_seed(52)
+    key = (torch.randn(3, 2, 8, generator=g) * 3).to(torch.bfloat16)
+    value = (torch.randn(3, 2, 8, generator=g) * 3).to(torch.bfloat16)
+    ks, vs = torch.tensor([0.05, 0.3]), torch.tensor([0.01, 7.0])  # some values saturate
+    kc = torch.zeros(4, 2, 16, 8, dtype=torch.int8)
+    vc = torch.zeros_like(kc)
+    slots = torch.tensor([5, -1, 63])
+    oracle.reshape_and_cache_int8(key, value, kc, vc, slots, ks, vs)
+    for t, s in ((0, 5), (2, 63)):
+        for h in range(2):
+            want_k = oracle.int8_encode(key[t, h].float() / ks[h])
+            want_v = oracle.int8_encode(value[t, h].float() / vs[h])
+            assert torch.equal(kc[s // 16, h, s % 16], want_k)
+            assert torch.equal(vc[s // 16, h, s % 16], want_v)
+    assert vc.abs().max() == 127  # value / 0.01 saturates
+    untouched = torch.ones(4, 16, dtype=torch.bool)
+    untouched[0, 5] = untouched[3, 15] = False
+    assert torch.all(kc.permute(0, 2, 1, 3)[untouched] == 0)
+
+
+def test_int8_decode_equals_decode_of_dequantized_cache():
+    """code*scale is exact in fp32 for power-of-two scales, so decode over the
+    INT8 cache equals decode over the dequantized fp32 cache bit for bit."""
+    ctxs, H_q, H_kv, D, bs = [7, 33, 50], 8, 2, 16, 16
+    g = torch.Generator().manual_seed(53)
+    NB = 12
+    kc = torch.randint(-127, 128, (NB, H_kv, bs, D), generator=g, dtype=torch.int32).to(torch.int8)
+    vc = torch.randint(-127, 128, (NB, H_kv, bs, D), generator=g, dtype=torch.int32).to(torch.int8)
+    ks, vs = torch.tensor([0.0625, 2.0 ** -7]), torch.tensor([0.25, 2.0 ** -6])
+    tables = torch.tensor([[3, 0, 0, 0], [1, 7, 2, 0], [4, 5, 6, 11]], dtype=torch.int32)
+    lens = torch.tensor(ctxs, dtype=torch.int32)
+    q = torch.randn(3, H_q, D, generator=g).to(torch.bfloat16)
+    out, lse = oracle.decode_int8(q, kc, vc, ks, vs, tables, lens, 0.2)
+    kd = (kc.double() * ks.double()[None, :, None, None]).float()
+    vd = (vc.double() * vs.double()[None, :, None, None]).float()
+    ref, ref_lse = oracle.decode(q.float(), kd, vd, tables, lens, 0.2)
+    assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+
+
+# ---------------------------------------------------------------------------
 # sliding window
 # ---------------------------------------------------------------------------
 def test_window_covering_everything_is_plain_decode():
