@@ -180,9 +180,10 @@ def profiled_traffic(profile: str, kernel_files, units_scale: float = 1.0):
         return None
     fields = {}
     for line in text.splitlines():
-        if ":" in line and line.lstrip().startswith(("source-sha256", "dram-bytes-per-launch")):
+        line = line.strip().lstrip("-* ")  # list items: "- key: `value`"
+        if ":" in line and line.startswith(("source-sha256", "dram-bytes-per-launch")):
             k, v = line.split(":", 1)
-            fields[k.strip().lstrip("-* ")] = v.strip().strip("`")
+            fields[k.strip()] = v.strip().strip("`")
     if fields.get("source-sha256") != source_digest(kernel_files):
         return None
     try:
@@ -497,11 +498,12 @@ def run_ours(args, rank, world):
             roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                     "unit": "GB/s", "frac": round(achieved / hbm, 4),
                     "peak_basis": f"{basis} hbm_gbs",
-                    "kernel": ("pa_decode_fp8 (decode_split_e4m3 + merge)" if batch.fp8 else
+                    "kernel": ("pa_decode_fp8 (decode_split_q8 + merge)" if batch.fp8 else
+                               "pa_decode_int8 (decode_split_q8 + merge)" if batch.int8 else
                                "pa_decode (decode_split + merge)"),
                     "alg_bytes_per_launch": dbytes,
                     "traffic": profiled_traffic(f"decode_{args.workload}{wtag}.md",
-                                                DECODE_FP8_SOURCES if batch.fp8
+                                                DECODE_FP8_SOURCES if batch.quantized
                                                 else DECODE_SOURCES)}
         else:
             value = dbytes_total / (ms * 1e-3) / 1e9
@@ -517,7 +519,7 @@ def run_ours(args, rank, world):
             "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": ("e4m3 KV / bf16 q" if batch.fp8 else
+            "dtype": ("e4m3 KV / bf16 q" if batch.fp8 else "int8 KV / bf16 q" if batch.int8 else
                       "bf16" if batch.dtype.itemsize == 2 else "f32"),
             "data": "synthetic (seeded; one batch per rank)",
             "config": workload_config(batch, args.workload, world, r),
@@ -580,6 +582,12 @@ def _oracle_step(batch, k, v, select=None, pselect=None):
         oracle.reshape_and_cache_e4m3(batch.key, batch.value, k, v, batch.slot_mapping,
                                       batch.k_scale, batch.v_scale)
         oracle.decode_e4m3(batch.q, k, v, batch.k_scale, batch.v_scale, batch.block_tables,
+                           batch.context_lens, batch.scale, select=select)
+        return
+    if batch.int8:
+        oracle.reshape_and_cache_int8(batch.key, batch.value, k, v, batch.slot_mapping,
+                                      batch.k_scale, batch.v_scale)
+        oracle.decode_int8(batch.q, k, v, batch.k_scale, batch.v_scale, batch.block_tables,
                            batch.context_lens, batch.scale, select=select)
         return
     oracle.reshape_and_cache(batch.key, batch.value, k, v, batch.slot_mapping)
@@ -743,6 +751,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama7b_decode",
                     choices=["tiny_fp32", "llama7b_decode", "gqa_decode", "long_context_decode",
                              "mixed_prefill_decode", "llama7b_decode_fp8", "gqa_decode_fp8",
+                             "llama7b_decode_int8", "gqa_decode_int8",
                              "cow_copy", "swap_out"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -760,7 +769,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.window < 0 or (args.window and args.workload.endswith("_fp8")):
+    if args.window < 0 or (args.window and args.workload.endswith(("_fp8", "_int8"))):
         ap.error("--window takes W > 0 and a bf16/fp32 workload")
     rank, local, world = rank_env()
     if world != args.gpus and world > 1:

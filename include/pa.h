@@ -165,6 +165,31 @@ PA_API pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, co
                                int max_context_len, float scale, int partition_size,
                                void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* INT8 KV cache (one int8 code per element, one dequantisation scale per K/V
+ * head for K and one for V): page "字节跳动 AI Infra (2)", optimisation table,
+ * row "KV量化(INT8)", and page "LLM推理优化", section 1.3 (INT8 K/V). Element
+ * value = code * scale[kv head].
+ *
+ * pa_reshape_and_cache_int8: as pa_reshape_and_cache_fp8 with int8 caches;
+ * each element is stored as the integer nearest to the IEEE fp32 quotient
+ * x / scale[h] (ties to even), saturated to [-127, 127]; NaN stores 0. */
+PA_API pa_status pa_reshape_and_cache_int8(const void *key, const void *value, void *k_cache,
+                                           void *v_cache, const int64_t *slot_mapping,
+                                           int num_tokens, int num_kv_heads, int head_dim,
+                                           int block_size, int num_blocks, const float *k_scale,
+                                           const float *v_scale, pa_dtype dtype,
+                                           cudaStream_t stream);
+
+/* pa_decode_int8: as pa_decode_fp8 over INT8 caches (int8, same layout and
+ * arguments). */
+PA_API pa_status pa_decode_int8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                const float *k_scale, const float *v_scale,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                int block_size, int num_blocks, int max_blocks_per_seq,
+                                int max_context_len, float scale, int partition_size,
+                                void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* pa_decode without a caller-provided workspace. The pages have no
  * counterpart: this exists for callers that cannot allocate device memory at
  * the call site (a plugin handed only its input and output buffers, or a

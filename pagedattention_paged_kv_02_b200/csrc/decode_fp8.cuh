@@ -1,12 +1,13 @@
-// decode_fp8.cuh -- paged decode over an FP8 (E4M3) KV cache.
+// decode_fp8.cuh -- paged decode over an 8-bit KV cache: FP8 (E4M3) or INT8
+// codes.
 //
-// Page "字节跳动 AI Infra (2)", optimisation table, row on KV quantisation,
-// and page "LLM推理优化", section 1.3: store K/V in low precision to shrink
-// the cache; decode is bound by KV reads (page "vLLM框架是怎么做推理加速的",
-// section 3), so halving the bytes per element halves its cost. Here each
-// element is an E4M3 code and value = code * scale[kv head]; the scales fold
-// into the score scale (K) and into the output (V), so the tensor-core
-// products run on the exact code values.
+// Page "字节跳动 AI Infra (2)", optimisation table, row "KV量化(INT8)", and
+// page "LLM推理优化", section 1.3 (INT8/INT4 K/V): store K/V in low precision
+// to shrink the cache; decode is bound by KV reads (page
+// "vLLM框架是怎么做推理加速的", section 3), so halving the bytes per element
+// halves its cost. Here each element is an E4M3 or INT8 code and value =
+// code * scale[kv head]; the scales fold into the score scale (K) and into
+// the output (V), so the tensor-core products run on the exact code values.
 //
 // Same work decomposition and pipeline as the bf16 split kernel (one CTA per
 // (partition, kv head [x 16-head tile], sequence), per-warp TMA rings of
@@ -23,8 +24,8 @@
 //     lane) plus one byte permute, giving two f16 token pairs for two
 //     adjacent dims; the output columns come out permuted accordingly and
 //     are put back in order in the merge;
-//   * the tensor-core type is f16 (E4M3 -> f16 is exact), P is rounded to
-//     f16 and the denominator sums the same rounded weights.
+//   * the tensor-core type is f16 (E4M3 -> f16 and INT8 -> f16 are exact), P
+//     is rounded to f16 and the denominator sums the same rounded weights.
 #pragma once
 
 #include "decode.cuh"
@@ -72,6 +73,29 @@ __device__ __forceinline__ void e4m3x4_to_f16x2_scaled(uint32_t w, uint32_t &eve
     even = ((w << 8) & 0x80008000u) | ((w << 7) & 0x3F803F80u);
 }
 
+// Four INT8 codes w = [c0 c1 c2 c3] (c0 the low byte) -> the f16 pairs
+// {c0, c2} (even) and {c1, c3} (odd), exact, without the conversion pipe:
+// flipping the sign bits makes each byte c + 128 in 0..255; a byte under the
+// f16 pattern 0x64 reads 1024 + (c + 128) (the ulp at 1024 is 1), and one
+// packed f16 subtraction of 1152 leaves c.
+__device__ __forceinline__ void int8x4_to_f16x2(uint32_t w, uint32_t &even, uint32_t &odd) {
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t e = __byte_perm(u, 0x64646464u, 0x4240);  // [c0', 0x64, c2', 0x64]
+    const uint32_t o = __byte_perm(u, 0x64646464u, 0x4341);  // [c1', 0x64, c3', 0x64]
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(even) : "r"(e), "r"(0x64806480u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(odd) : "r"(o), "r"(0x64806480u));
+}
+
+// The even/odd f16 pairs of a word of four codes, for the integer-pipe forms
+// of decode_split_q8 (CV 1, 2: E4M3 times 2^-8; CV 3: INT8).
+template <int CV>
+__device__ __forceinline__ void codes_to_f16x2(uint32_t w, uint32_t &even, uint32_t &odd) {
+    if constexpr (CV == 3)
+        int8x4_to_f16x2(w, even, odd);
+    else
+        e4m3x4_to_f16x2_scaled(w, even, odd);
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -88,15 +112,17 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
 // CT: tokens per pipeline stage (16 or 32). A 32-token stage is two
 // 16-token page pieces (each inside one physical block, so each has its own
 // table lookup); it halves the softmax and hand-off work per byte.
-// CV: where codes become f16. 0: the conversion instruction for K and V;
-// 1: K on the integer pipe (e4m3x4_to_f16x2_scaled), V by instruction;
-// 2: both on the integer pipe; the 2^-8 of the integer form folds into the
-// scales. The conversion instruction shares a narrow pipe with the
-// exponentials, but the integer form costs 3.5 instructions per pair and
-// measured slower on B200, so 0 is the default.
+// CV: the code format and where codes become f16. E4M3: 0 = the conversion
+// instruction for K and V; 1 = K on the integer pipe
+// (e4m3x4_to_f16x2_scaled), V by instruction; 2 = both on the integer pipe
+// (the 2^-8 of the integer form folds into the scales). The conversion
+// instruction shares a narrow pipe with the exponentials, but the E4M3
+// integer form costs 3.5 instructions per pair and measured slower on B200,
+// so 0 is the E4M3 default. INT8: 3 = both on the integer and FMA pipes
+// (int8x4_to_f16x2, 2.5 instructions per pair).
 template <int NW, int NS, int CT, int CV>
 __global__ void __launch_bounds__(NW * 32)
-    decode_split_e4m3(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+    decode_split_q8(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
     constexpr int D = 128;
     constexpr int HT = kHeadsBf16;
@@ -182,8 +208,8 @@ __global__ void __launch_bounds__(NW * 32)
         for (int i = 0; i < NS && i < my_n; ++i) issue(i);
     }
 
-    const float sl2 = a.scale_log2 * __ldg(a.k_scale + kvh) * (CV >= 1 ? 256.f : 1.f);
-    const float vsc = __ldg(a.v_scale + kvh) * (CV >= 2 ? 256.f : 1.f);
+    const float sl2 = a.scale_log2 * __ldg(a.k_scale + kvh) * (CV == 1 || CV == 2 ? 256.f : 1.f);
+    const float vsc = __ldg(a.v_scale + kvh) * (CV == 2 ? 256.f : 1.f);
 
     // Q fragments in f16, dims permuted to match the K fragments: slot
     // 2c+j (j = 0,1) of k-step ks holds dim 16ks+4c+j, slot 2c+8+j holds
@@ -273,10 +299,10 @@ __global__ void __launch_bounds__(NW * 32)
                         ldsm_x4(kb + p * kChunk * D + sw128(r, u), r0, r1, r2, r3);
                         if constexpr (CV >= 1) {
                             uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
-                            e4m3x4_to_f16x2_scaled(r0, e0, o0);
-                            e4m3x4_to_f16x2_scaled(r1, e1, o1);
-                            e4m3x4_to_f16x2_scaled(r2, e2, o2);
-                            e4m3x4_to_f16x2_scaled(r3, e3, o3);
+                            codes_to_f16x2<CV>(r0, e0, o0);
+                            codes_to_f16x2<CV>(r1, e1, o1);
+                            codes_to_f16x2<CV>(r2, e2, o2);
+                            codes_to_f16x2<CV>(r3, e3, o3);
                             mma_f16_16816(sc[2 * p], qa[2 * kp], e0, o0);
                             mma_f16_16816(sc[2 * p + 1], qa[2 * kp], e1, o1);
                             mma_f16_16816(sc[2 * p], qa[2 * kp + 1], e2, o2);
@@ -382,10 +408,10 @@ __global__ void __launch_bounds__(NW * 32)
                         if constexpr (CV >= 2) {
                             // even codes of a word: dim 2g, odd codes: dim 2g+1
                             uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
-                            e4m3x4_to_f16x2_scaled(r0, e0, o0);
-                            e4m3x4_to_f16x2_scaled(r1, e1, o1);
-                            e4m3x4_to_f16x2_scaled(r2, e2, o2);
-                            e4m3x4_to_f16x2_scaled(r3, e3, o3);
+                            codes_to_f16x2<CV>(r0, e0, o0);
+                            codes_to_f16x2<CV>(r1, e1, o1);
+                            codes_to_f16x2<CV>(r2, e2, o2);
+                            codes_to_f16x2<CV>(r3, e3, o3);
                             mma_f16_16816(o[2 * u0], pa[p], e0, e1);
                             mma_f16_16816(o[2 * u0 + 1], pa[p], o0, o1);
                             mma_f16_16816(o[2 * u1], pa[p], e2, e3);
@@ -528,6 +554,74 @@ __global__ void __launch_bounds__(256)
             e4m3x2_from_f32(__fdiv_rn(xv[4 * w + 2], vs), __fdiv_rn(xv[4 * w + 3], vs));
         kc[w] = k01 | (k23 << 16);
         vc[w] = v01 | (v23 << 16);
+    }
+    const long long block = slot / a.block_size;
+    const long long offset = slot - block * a.block_size;
+    const long long dst = ((block * a.num_kv_heads + h) * a.block_size + offset) * a.vecs_per_row + c;
+    a.k_cache[dst] = make_uint4(kc[0], kc[1], kc[2], kc[3]);
+    a.v_cache[dst] = make_uint4(vc[0], vc[1], vc[2], vc[3]);
+}
+
+// INT8 append: as the E4M3 append, each code the nearest integer of the
+// fp32 quotient x / scale[h] (IEEE division; ties to even by the
+// round-to-nearest-even conversion, which also turns NaN into 0), saturated
+// to [-127, 127].
+__device__ __forceinline__ uint32_t int8x4_from_f32(float x0, float x1, float x2, float x3) {
+    auto one = [](float x) -> uint32_t {
+        const int r = min(max(__float2int_rn(x), -127), 127);
+        return (uint32_t)(r & 0xff);
+    };
+    return one(x0) | (one(x1) << 8) | (one(x2) << 16) | (one(x3) << 24);
+}
+
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_int8_kernel(const __grid_constant__ ReshapeFp8Args a) {
+    const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (i >= a.total_vecs) return;
+    const long long t = i / a.vecs_per_token;
+    const int r = static_cast<int>(i - t * a.vecs_per_token);
+    const int h = r / a.vecs_per_row;
+    const int c = r - h * a.vecs_per_row;
+    const long long slot = __ldg(a.slot_mapping + t);
+    if (slot < 0) return;
+    if (slot >= a.num_slots) {
+        flag_error(PA_ERR_BAD_TABLE);
+        return;
+    }
+    const float ks = __ldg(a.k_scale + h), vs = __ldg(a.v_scale + h);
+    float xk[16], xv[16];
+    if (a.bf16_in) {
+        const uint4 *k4 = reinterpret_cast<const uint4 *>(a.key) + 2 * i;
+        const uint4 *v4 = reinterpret_cast<const uint4 *>(a.value) + 2 * i;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            const uint4 kk = __ldg(k4 + w), vv = __ldg(v4 + w);
+            const uint32_t kw[4] = {kk.x, kk.y, kk.z, kk.w}, vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                xk[8 * w + 2 * e] = bf16_lo(kw[e]);
+                xk[8 * w + 2 * e + 1] = bf16_hi(kw[e]);
+                xv[8 * w + 2 * e] = bf16_lo(vw[e]);
+                xv[8 * w + 2 * e + 1] = bf16_hi(vw[e]);
+            }
+        }
+    } else {
+        const float4 *k4 = reinterpret_cast<const float4 *>(a.key) + 4 * i;
+        const float4 *v4 = reinterpret_cast<const float4 *>(a.value) + 4 * i;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float4 kk = __ldg(k4 + w), vv = __ldg(v4 + w);
+            xk[4 * w] = kk.x; xk[4 * w + 1] = kk.y; xk[4 * w + 2] = kk.z; xk[4 * w + 3] = kk.w;
+            xv[4 * w] = vv.x; xv[4 * w + 1] = vv.y; xv[4 * w + 2] = vv.z; xv[4 * w + 3] = vv.w;
+        }
+    }
+    uint32_t kc[4], vc[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        kc[w] = int8x4_from_f32(__fdiv_rn(xk[4 * w], ks), __fdiv_rn(xk[4 * w + 1], ks),
+                                __fdiv_rn(xk[4 * w + 2], ks), __fdiv_rn(xk[4 * w + 3], ks));
+        vc[w] = int8x4_from_f32(__fdiv_rn(xv[4 * w], vs), __fdiv_rn(xv[4 * w + 1], vs),
+                                __fdiv_rn(xv[4 * w + 2], vs), __fdiv_rn(xv[4 * w + 3], vs));
     }
     const long long block = slot / a.block_size;
     const long long offset = slot - block * a.block_size;

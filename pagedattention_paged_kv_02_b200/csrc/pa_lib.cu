@@ -120,7 +120,7 @@ Pipe decode_pipe() {
 }
 
 // Launch shape of the FP8 split kernel: warps x stages x tokens per stage x
-// code conversion (decode_split_e4m3's CV);
+// code conversion (decode_split_q8's CV);
 // PA_DECODE_PIPE_FP8=<warps>x<stages>x<tokens>x<cv> (built: 4x2x32x0,
 // 4x2x32x2, 4x2x16x0, 4x3x32x0; default 4x2x32x0: on B200 the conversion
 // instruction beat the integer-pipe form, 0.62 vs 0.55 of the HBM peak on
@@ -217,12 +217,12 @@ bool encode_cache_map_u8(CUtensorMap *m, const void *cache, int NB, int H_kv, in
 }
 
 template <int NW, int NS, int CT, int CV>
-pa_status launch_decode_e4m3(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
+pa_status launch_decode_q8(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
                              dim3 grid, cudaStream_t st) {
     constexpr int STAGE = 2 * CT * 128;
     using L = DecodeSmem<NW, NS, STAGE, kHeadsBf16, 128>;
     const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
-    auto k = decode_split_e4m3<NW, NS, CT, CV>;
+    auto k = decode_split_q8<NW, NS, CT, CV>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
     k<<<grid, NW * 32, smem, st>>>(a, mk, mv);
     return launch_status();
@@ -440,11 +440,11 @@ pa_status pa_decode_sliding_window(void *out, const void *q, const void *k_cache
                        workspace_bytes_given, dtype, sliding_window, stream);
 }
 
-pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache,
-                                   void *v_cache, const int64_t *slot_mapping, int num_tokens,
-                                   int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                                   const float *k_scale, const float *v_scale, pa_dtype dtype,
-                                   cudaStream_t stream) {
+static pa_status reshape_q8_impl(const void *key, const void *value, void *k_cache,
+                                 void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                                 int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                 const float *k_scale, const float *v_scale, pa_dtype dtype,
+                                 bool int8, cudaStream_t stream) {
     if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
         return PA_ERR_INVALID_ARG;
     if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
@@ -473,17 +473,41 @@ pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_c
     a.bf16_in = dtype == PA_BF16;
     const long long blocks = (a.total_vecs + 255) / 256;
     if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-    reshape_and_cache_e4m3_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    if (int8)
+        reshape_and_cache_int8_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    else
+        reshape_and_cache_e4m3_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
     return launch_status();
 }
 
-pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
-                        const float *k_scale, const float *v_scale, const int32_t *block_tables,
-                        const int32_t *context_lens, int num_seqs, int num_q_heads,
-                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                        int max_blocks_per_seq, int max_context_len, float scale,
-                        int partition_size, void *workspace, size_t workspace_bytes_given,
-                        cudaStream_t stream) {
+pa_status pa_reshape_and_cache_fp8(const void *key, const void *value, void *k_cache,
+                                   void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                                   int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                   const float *k_scale, const float *v_scale, pa_dtype dtype,
+                                   cudaStream_t stream) {
+    return reshape_q8_impl(key, value, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
+                           head_dim, block_size, num_blocks, k_scale, v_scale, dtype, false,
+                           stream);
+}
+
+pa_status pa_reshape_and_cache_int8(const void *key, const void *value, void *k_cache,
+                                    void *v_cache, const int64_t *slot_mapping, int num_tokens,
+                                    int num_kv_heads, int head_dim, int block_size,
+                                    int num_blocks, const float *k_scale, const float *v_scale,
+                                    pa_dtype dtype, cudaStream_t stream) {
+    return reshape_q8_impl(key, value, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads,
+                           head_dim, block_size, num_blocks, k_scale, v_scale, dtype, true,
+                           stream);
+}
+
+static pa_status decode_q8_impl(void *out, const void *q, const void *k_cache,
+                                const void *v_cache, const float *k_scale, const float *v_scale,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                int block_size, int num_blocks, int max_blocks_per_seq,
+                                int max_context_len, float scale, int partition_size,
+                                void *workspace, size_t workspace_bytes_given, bool int8,
+                                cudaStream_t stream) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
         return PA_ERR_INVALID_ARG;
@@ -548,13 +572,43 @@ pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const voi
     auto is = [&](int w, int n, int c, int v) {
         return pp.nw == w && pp.ns == n && pp.ct == c && pp.cv == v;
     };
-    pa_status st = is(4, 2, 32, 2)   ? launch_decode_e4m3<4, 2, 32, 2>(a, mk, mv, grid, stream)
-                   : is(4, 2, 16, 0) ? launch_decode_e4m3<4, 2, 16, 0>(a, mk, mv, grid, stream)
-                   : is(4, 3, 32, 0) ? launch_decode_e4m3<4, 3, 32, 0>(a, mk, mv, grid, stream)
-                                     : launch_decode_e4m3<4, 2, 32, 0>(a, mk, mv, grid, stream);
+    pa_status st;
+    if (int8)
+        st = launch_decode_q8<4, 2, 32, 3>(a, mk, mv, grid, stream);
+    else
+        st = is(4, 2, 32, 2)   ? launch_decode_q8<4, 2, 32, 2>(a, mk, mv, grid, stream)
+             : is(4, 2, 16, 0) ? launch_decode_q8<4, 2, 16, 0>(a, mk, mv, grid, stream)
+             : is(4, 3, 32, 0) ? launch_decode_q8<4, 3, 32, 0>(a, mk, mv, grid, stream)
+                               : launch_decode_q8<4, 2, 32, 0>(a, mk, mv, grid, stream);
     if (st != PA_OK) return st;
     if (S1 > 1) st = launch_reduce<128, __nv_bfloat16>(a, stream);
     return st;
+}
+
+pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const float *k_scale, const float *v_scale, const int32_t *block_tables,
+                        const int32_t *context_lens, int num_seqs, int num_q_heads,
+                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                        int max_blocks_per_seq, int max_context_len, float scale,
+                        int partition_size, void *workspace, size_t workspace_bytes_given,
+                        cudaStream_t stream) {
+    return decode_q8_impl(out, q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                          context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                          block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+                          partition_size, workspace, workspace_bytes_given, false, stream);
+}
+
+pa_status pa_decode_int8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const float *k_scale, const float *v_scale, const int32_t *block_tables,
+                         const int32_t *context_lens, int num_seqs, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                         int max_blocks_per_seq, int max_context_len, float scale,
+                         int partition_size, void *workspace, size_t workspace_bytes_given,
+                         cudaStream_t stream) {
+    return decode_q8_impl(out, q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                          context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                          block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+                          partition_size, workspace, workspace_bytes_given, true, stream);
 }
 
 static pa_status prefill_impl(void *out, const void *q, const void *k_cache, const void *v_cache,

@@ -27,7 +27,7 @@ EXPORTS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_partit
            "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
            "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
            "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window",
-           "pa_prefill_chunk_sliding_window")
+           "pa_prefill_chunk_sliding_window", "pa_reshape_and_cache_int8", "pa_decode_int8")
 
 
 class PAError(RuntimeError):
@@ -62,8 +62,10 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_sliding_window.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,
                                                P, SZ, I, P]
         L.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, I, P]
+        L.pa_reshape_and_cache_int8.argtypes = L.pa_reshape_and_cache_fp8.argtypes
         L.pa_decode_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, SZ,
                                     P]
+        L.pa_decode_int8.argtypes = L.pa_decode_fp8.argtypes
         L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P]
         L.pa_swap_blocks.argtypes = [P, P, I, P, P, I, P, I, I, I, I, I, P]
         L.pa_check_tables.argtypes = [P, P, I, I, I, I, P, ctypes.POINTER(I), P]
@@ -74,7 +76,8 @@ def lib() -> ctypes.CDLL:
         for f in ("pa_reshape_and_cache", "pa_decode", "pa_decode_static_workspace",
                   "pa_prefill_chunk", "pa_check_tables", "pa_copy_blocks", "pa_swap_blocks",
                   "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window",
-                  "pa_prefill_chunk_sliding_window", "pa_device_error",
+                  "pa_prefill_chunk_sliding_window", "pa_reshape_and_cache_int8",
+                  "pa_decode_int8", "pa_device_error",
                   "pa_selftest_bounded_wait", "pa_decode_partition_tokens", "pa_version"):
             getattr(L, f).restype = I
         _lib = L
@@ -237,45 +240,73 @@ def pa_prefill_chunk_sliding_window(out, q, k_cache, v_cache, block_tables, cont
           _dt(q), _stream(stream))
 
 
-def _fp8_pool(k_cache, v_cache, k_scale, v_scale):
-    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
-        raise TypeError("FP8 caches are uint8 tensors of E4M3 codes")
+def _fp8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype=torch.uint8):
+    if k_cache.dtype != code_dtype or v_cache.dtype != code_dtype:
+        raise TypeError("FP8 caches are uint8 tensors of E4M3 codes, INT8 caches int8 tensors")
     H_kv = k_cache.shape[1]
     for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
         if t.dtype != torch.float32 or t.numel() != H_kv:
             raise ValueError(f"{n} must be float32 [num_kv_heads]")
 
 
-def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
-                             stream=None) -> None:
-    """Quantising append into E4M3 caches (codes of x / scale[h])."""
+def _reshape_q8(fn, code_dtype, key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                stream):
     _check_int(slot_mapping, torch.int64, "slot_mapping")
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale)
+    _fp8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype)
     NB, H_kv, bs, D = k_cache.shape
     T = slot_mapping.numel()
     if key.shape != (T, H_kv, D) or value.shape != (T, H_kv, D) or key.dtype != value.dtype:
         raise ValueError("key/value must be [num_tokens, num_kv_heads, head_dim], one dtype")
-    _call("pa_reshape_and_cache_fp8", _p(key), _p(value), _p(k_cache), _p(v_cache),
-          _p(slot_mapping), T, H_kv, D, bs, NB, _p(k_scale), _p(v_scale), _dt(key),
+    _call(fn, _p(key), _p(value), _p(k_cache), _p(v_cache), _p(slot_mapping), T, H_kv, D, bs, NB,
+          _p(k_scale), _p(v_scale), _dt(key), _stream(stream))
+
+
+def _decode_q8(fn, code_dtype, out, q, k_cache, v_cache, k_scale, v_scale, block_tables,
+               context_lens, max_context_len, scale, partition_size, workspace, stream):
+    _check_int(block_tables, torch.int32, "block_tables")
+    _check_int(context_lens, torch.int32, "context_lens")
+    _fp8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype)
+    B, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or q.dtype != torch.bfloat16 or out.dtype != q.dtype:
+        raise ValueError("q and out must be bf16 [B, H_q, head_dim]")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _call(fn, _p(out), _p(q), _p(k_cache), _p(v_cache), _p(k_scale), _p(v_scale),
+          _p(block_tables), _p(context_lens), B, H_q, H_kv, D, bs, NB, block_tables.shape[1],
+          int(max_context_len), float(scale), int(partition_size), _p(workspace), ws_bytes,
           _stream(stream))
+
+
+def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                             stream=None) -> None:
+    """Quantising append into E4M3 caches (codes of x / scale[h])."""
+    _reshape_q8("pa_reshape_and_cache_fp8", torch.uint8, key, value, k_cache, v_cache,
+                slot_mapping, k_scale, v_scale, stream)
+
+
+def pa_reshape_and_cache_int8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                              stream=None) -> None:
+    """Quantising append into INT8 caches (nearest integers of x / scale[h])."""
+    _reshape_q8("pa_reshape_and_cache_int8", torch.int8, key, value, k_cache, v_cache,
+                slot_mapping, k_scale, v_scale, stream)
 
 
 def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                   max_context_len: int, scale: float, partition_size: int = 0,
                   workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """Paged decode over E4M3 caches; q/out bf16 [B, H_q, 128]."""
-    _check_int(block_tables, torch.int32, "block_tables")
-    _check_int(context_lens, torch.int32, "context_lens")
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale)
-    B, H_q, D = q.shape
-    NB, H_kv, bs, D2 = k_cache.shape
-    if out.shape != q.shape or D2 != D or q.dtype != torch.bfloat16 or out.dtype != q.dtype:
-        raise ValueError("q and out must be bf16 [B, H_q, head_dim]")
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _call("pa_decode_fp8", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(k_scale), _p(v_scale),
-          _p(block_tables), _p(context_lens), B, H_q, H_kv, D, bs, NB, block_tables.shape[1],
-          int(max_context_len), float(scale), int(partition_size), _p(workspace), ws_bytes,
-          _stream(stream))
+    _decode_q8("pa_decode_fp8", torch.uint8, out, q, k_cache, v_cache, k_scale, v_scale,
+               block_tables, context_lens, max_context_len, scale, partition_size, workspace,
+               stream)
+
+
+def pa_decode_int8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                   max_context_len: int, scale: float, partition_size: int = 0,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Paged decode over INT8 caches; q/out bf16 [B, H_q, 128]."""
+    _decode_q8("pa_decode_int8", torch.int8, out, q, k_cache, v_cache, k_scale, v_scale,
+               block_tables, context_lens, max_context_len, scale, partition_size, workspace,
+               stream)
 
 
 def _addressable(t: torch.Tensor):
@@ -413,24 +444,28 @@ def prepare_prefill_chunk(out, q, k_cache, v_cache, block_tables, context_lens, 
 
 def prepare_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale,
                                   v_scale) -> Prepared:
+    """``pa_reshape_and_cache_fp8``, or ``pa_reshape_and_cache_int8`` for int8 caches."""
     _check_int(slot_mapping, torch.int64, "slot_mapping")
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale)
+    int8 = k_cache.dtype == torch.int8
+    _fp8_pool(k_cache, v_cache, k_scale, v_scale, torch.int8 if int8 else torch.uint8)
     NB, H_kv, bs, D = k_cache.shape
-    return Prepared("pa_reshape_and_cache_fp8", (_p(key), _p(value), _p(k_cache), _p(v_cache),
-                                                 _p(slot_mapping), slot_mapping.numel(), H_kv, D,
-                                                 bs, NB, _p(k_scale), _p(v_scale), _dt(key)))
+    return Prepared("pa_reshape_and_cache_int8" if int8 else "pa_reshape_and_cache_fp8",
+                    (_p(key), _p(value), _p(k_cache), _p(v_cache), _p(slot_mapping),
+                     slot_mapping.numel(), H_kv, D, bs, NB, _p(k_scale), _p(v_scale), _dt(key)))
 
 
 def prepare_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                        max_context_len: int, scale: float, partition_size: int = 0,
                        workspace: Optional[torch.Tensor] = None) -> Prepared:
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale)
+    """``pa_decode_fp8``, or ``pa_decode_int8`` for int8 caches."""
+    int8 = k_cache.dtype == torch.int8
+    _fp8_pool(k_cache, v_cache, k_scale, v_scale, torch.int8 if int8 else torch.uint8)
     B, H_q, D = q.shape
     NB, H_kv, bs, _ = k_cache.shape
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    return Prepared("pa_decode_fp8", (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(k_scale),
-                                      _p(v_scale), _p(block_tables), _p(context_lens), B, H_q,
-                                      H_kv, D, bs, NB, block_tables.shape[1], int(max_context_len),
-                                      float(scale), int(partition_size), _p(workspace),
-                                      ws_bytes))
+    return Prepared("pa_decode_int8" if int8 else "pa_decode_fp8",
+                    (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(k_scale), _p(v_scale),
+                     _p(block_tables), _p(context_lens), B, H_q, H_kv, D, bs, NB,
+                     block_tables.shape[1], int(max_context_len), float(scale),
+                     int(partition_size), _p(workspace), ws_bytes))
 

@@ -69,7 +69,7 @@ class Batch:
     prefill_context_lens: Optional[torch.Tensor] = None
     query_start_loc: Optional[torch.Tensor] = None
     partition_size: int = 0
-    k_scale: Optional[torch.Tensor] = None  # FP8 pools: float32 [H_kv] per-head scales
+    k_scale: Optional[torch.Tensor] = None  # 8-bit pools: float32 [H_kv] per-head scales
     v_scale: Optional[torch.Tensor] = None
     sliding_window: int = 0  # > 0: every query sees only its last sliding_window positions
 
@@ -99,6 +99,15 @@ class Batch:
     @property
     def fp8(self) -> bool:
         return self.k_cache.dtype == torch.uint8
+
+    @property
+    def int8(self) -> bool:
+        return self.k_cache.dtype == torch.int8
+
+    @property
+    def quantized(self) -> bool:
+        """The pool holds 8-bit codes (FP8 E4M3 or INT8) with per-head scales."""
+        return self.fp8 or self.int8
 
     @property
     def num_seqs(self) -> int:
@@ -359,6 +368,27 @@ def to_fp8(batch: Batch, k_amax: float = 4.0, v_amax: float = 4.0) -> Batch:
     return Batch(**kw)
 
 
+def to_int8(batch: Batch, k_amax: float = 4.0, v_amax: float = 4.0) -> Batch:
+    """A copy of a decode batch whose pool holds INT8 codes: each cached value
+    divided by its K/V head's scale (amax / 127) and rounded to the nearest
+    integer (torch.round: ties to even), clamped to [-127, 127]. NaN poison
+    becomes 0 (INT8 has no NaN). q and the step's new K/V rows keep their
+    type (the append quantises them)."""
+    H = batch.num_kv_heads
+    ks = torch.full((H,), k_amax / 127.0, dtype=torch.float32)
+    vs = torch.full((H,), v_amax / 127.0, dtype=torch.float32)
+
+    def enc(pool, sc):
+        x = pool.float() / sc[None, :, None, None]
+        x = torch.nan_to_num(x, nan=0.0).round().clamp(-127.0, 127.0)
+        return x.to(torch.int8)
+
+    kw = dict(batch.__dict__)
+    kw.update(k_cache=enc(batch.k_cache, ks), v_cache=enc(batch.v_cache, vs), k_scale=ks,
+              v_scale=vs, name=batch.name + "_int8")
+    return Batch(**kw)
+
+
 def llama7b_decode_fp8(seed: int = 0, num_blocks: int = 16384, block_size: int = 16) -> Batch:
     """The Llama-2-7B-shaped decode batch with an FP8 E4M3 pool."""
     return to_fp8(llama7b_decode(seed, num_blocks, block_size))
@@ -369,6 +399,16 @@ def gqa_decode_fp8(seed: int = 0, num_blocks: int = 32768, block_size: int = 16)
     return to_fp8(gqa_decode(seed, num_blocks, block_size))
 
 
+def llama7b_decode_int8(seed: int = 0, num_blocks: int = 16384, block_size: int = 16) -> Batch:
+    """The Llama-2-7B-shaped decode batch with an INT8 pool."""
+    return to_int8(llama7b_decode(seed, num_blocks, block_size))
+
+
+def gqa_decode_int8(seed: int = 0, num_blocks: int = 32768, block_size: int = 16) -> Batch:
+    """The GQA decode batch with an INT8 pool."""
+    return to_int8(gqa_decode(seed, num_blocks, block_size))
+
+
 WORKLOADS = {
     "tiny_fp32": tiny_fp32,
     "llama7b_decode": llama7b_decode,
@@ -377,4 +417,6 @@ WORKLOADS = {
     "mixed_prefill_decode": mixed_prefill_decode,
     "llama7b_decode_fp8": llama7b_decode_fp8,
     "gqa_decode_fp8": gqa_decode_fp8,
+    "llama7b_decode_int8": llama7b_decode_int8,
+    "gqa_decode_int8": gqa_decode_int8,
 }

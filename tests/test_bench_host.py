@@ -39,3 +39,35 @@ def test_reference_arm_with_window(capsys, monkeypatch):
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["config"]["sliding_window"] == 8
     assert line["value"] > 0
+
+
+def test_profiled_traffic_follows_the_source_digest(tmp_path, monkeypatch):
+    """The DRAM bytes of a committed ncu summary are reported only while the
+    kernel source still hashes to the digest recorded beside them."""
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "k.cuh"
+    src.write_text("kernel v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    digest = bench.source_digest(["k.cuh"])
+    (tmp_path / "profiles" / "p.md").write_text(
+        f"# summary\n\n- source-sha256: `{digest}`\n- dram-bytes-per-launch: `123456`\n")
+    assert bench.profiled_traffic("p.md", ["k.cuh"]) == 123456.0
+    assert bench.profiled_traffic("missing.md", ["k.cuh"]) is None
+    src.write_text("kernel v2\n")
+    assert bench.profiled_traffic("p.md", ["k.cuh"]) is None
+
+
+def test_committed_profiles_match_the_sources():
+    """Every committed decode/prefill summary carries a digest of the current
+    kernel sources (a stale summary would silently drop roofline.traffic)."""
+    import glob
+    import os
+    for path in glob.glob(os.path.join(bench.ROOT, "profiles", "*.md")):
+        name = os.path.basename(path)
+        if name.startswith("prefill_"):
+            files = bench.PREFILL_SOURCES
+        elif name.endswith(("_fp8.md", "_int8.md")):
+            files = bench.DECODE_FP8_SOURCES
+        else:
+            files = bench.DECODE_SOURCES
+        assert bench.profiled_traffic(name, files) is not None, f"{name} is stale"
