@@ -47,6 +47,7 @@ struct DecodeArgs {
     const float *k_scale;  // FP8 caches: per K/V head dequantisation scales
     const float *v_scale;
     int num_seqs, H_q, H_kv, group, bs, NB, MB, max_ctx, P, S_max, n_htiles;
+    int bs_shift;      // log2(bs): block sizes are powers of two
     int window;        // > 0: attend only the last `window` positions
     float scale_log2;  // scale * log2(e): scores are kept in the base-2 domain
     unsigned long long timeout_ns;
@@ -181,8 +182,8 @@ __global__ void __launch_bounds__(NW * 32)
     const int tok0 = base + s * a.P;
     const int tok1 = min(tok0 + a.P, ctx);
     const int n_chunks = (tok1 - tok0 + kChunk - 1) / kChunk;
-    const int lb0 = tok0 / a.bs;
-    const int n_tbl = (tok1 - 1) / a.bs - lb0 + 1;
+    const int lb0 = tok0 >> a.bs_shift;
+    const int n_tbl = ((tok1 - 1) >> a.bs_shift) - lb0 + 1;
 
     // table slice of this partition -> shared memory (ids checked once here)
     const int32_t *row = a.block_tables + (size_t)b * a.MB + lb0;
@@ -208,14 +209,14 @@ __global__ void __launch_bounds__(NW * 32)
         const int st = i % NS;
         const uint32_t bar = bar0 + st * 8;
         const int t = tok0 + (warp + i * NW) * kChunk;
-        const int id = tbl[t / a.bs - lb0];
+        const int id = tbl[(t >> a.bs_shift) - lb0];
         if (id < 0) {
             mbar_arrive(bar);  // nothing to load; the chunk is skipped
             return;
         }
         mbar_arrive_expect_tx(bar, STAGE);
         const uint32_t kdst = stage0 + st * STAGE;
-        const int off = t % a.bs;
+        const int off = t & (a.bs - 1);
 #pragma unroll
         for (int sub = 0; sub < D / 64; ++sub) {
             tma_load_4d(kdst + sub * SUBTILE, &tmk, bar, sub * 64, off, kvh, id);
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(NW * 32)
         }
         done = i + 1;
         const int t = tok0 + (warp + i * NW) * kChunk;
-        const int id = tbl[t / a.bs - lb0];
+        const int id = tbl[(t >> a.bs_shift) - lb0];
         if (id >= 0) {
             const int valid = min(kChunk, tok1 - t);
             const int first = max(0, lo - t);  // rows before the window start
@@ -424,8 +425,8 @@ __global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constan
     const int tok0 = base + s * a.P;
     const int tok1 = min(tok0 + a.P, ctx);
     const int n_chunks = (tok1 - tok0 + kChunk - 1) / kChunk;
-    const int lb0 = tok0 / a.bs;
-    const int n_tbl = (tok1 - 1) / a.bs - lb0 + 1;
+    const int lb0 = tok0 >> a.bs_shift;
+    const int n_tbl = ((tok1 - 1) >> a.bs_shift) - lb0 + 1;
 
     const int32_t *row = a.block_tables + (size_t)b * a.MB + lb0;
     for (int i = threadIdx.x; i < n_tbl; i += NW * 32) {
@@ -452,13 +453,13 @@ __global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constan
         const int st = i % NS;
         const uint32_t bar = bar0 + st * 8;
         const int t = tok0 + (warp + i * NW) * kChunk;
-        const int id = tbl[t / a.bs - lb0];
+        const int id = tbl[(t >> a.bs_shift) - lb0];
         if (id < 0) {
             mbar_arrive(bar);
             return;
         }
         mbar_arrive_expect_tx(bar, STAGE);
-        const size_t page = (((size_t)id * a.H_kv + kvh) * a.bs + (t % a.bs)) * D;
+        const size_t page = (((size_t)id * a.H_kv + kvh) * a.bs + (t & (a.bs - 1))) * D;
         bulk_load(stage0 + st * STAGE, kc + page, HALF, bar);
         bulk_load(stage0 + st * STAGE + HALF, vc + page, HALF, bar);
     };
@@ -493,7 +494,7 @@ __global__ void __launch_bounds__(NW * 32) decode_split_f32(const __grid_constan
         }
         done = i + 1;
         const int t = tok0 + (warp + i * NW) * kChunk;
-        const int id = tbl[t / a.bs - lb0];
+        const int id = tbl[(t >> a.bs_shift) - lb0];
         if (id >= 0) {
             const int valid = min(kChunk, tok1 - t);
             const int first = max(0, lo - t);

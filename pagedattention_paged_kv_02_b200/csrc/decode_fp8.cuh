@@ -156,8 +156,8 @@ __global__ void __launch_bounds__(NW * 32)
     const int tok0 = base + s * a.P;
     const int tok1 = min(tok0 + a.P, ctx);
     const int n_chunks = (tok1 - tok0 + CT - 1) / CT;
-    const int lb0 = tok0 / a.bs;
-    const int n_tbl = (tok1 - 1) / a.bs - lb0 + 1;
+    const int lb0 = tok0 >> a.bs_shift;
+    const int n_tbl = ((tok1 - 1) >> a.bs_shift) - lb0 + 1;
 
     const int32_t *row = a.block_tables + (size_t)b * a.MB + lb0;
     for (int i = threadIdx.x; i < n_tbl; i += NW * 32) {
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
         for (int p = 0; p < PIECES; ++p) {
             const int tp = t + p * kChunk;
-            ids[p] = tp < tok1 ? tbl[tp / a.bs - lb0] : -1;
+            ids[p] = tp < tok1 ? tbl[(tp >> a.bs_shift) - lb0] : -1;
             n += ids[p] >= 0;
         }
         if (n == 0) {
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
         for (int p = 0; p < PIECES; ++p) {
             if (ids[p] < 0) continue;
-            const int off = (t + p * kChunk) % a.bs;
+            const int off = (t + p * kChunk) & (a.bs - 1);
             tma_load_4d(kdst + p * kChunk * D, &tmk, bar, 0, off, kvh, ids[p]);
             tma_load_4d(kdst + HALF + p * kChunk * D, &tmv, bar, 0, off, kvh, ids[p]);
         }
@@ -262,7 +262,8 @@ __global__ void __launch_bounds__(NW * 32)
         int pok = 0;
 #pragma unroll
         for (int p = 0; p < PIECES; ++p)
-            if (t + p * kChunk < tok1 && tbl[(t + p * kChunk) / a.bs - lb0] >= 0) pok |= 1 << p;
+            if (t + p * kChunk < tok1 && tbl[((t + p * kChunk) >> a.bs_shift) - lb0] >= 0)
+                pok |= 1 << p;
         if (pok) {
             const int valid = min(CT, tok1 - t);
             const int first = max(0, lo - t);  // rows before the window start

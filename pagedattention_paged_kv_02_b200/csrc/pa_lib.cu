@@ -188,10 +188,11 @@ int prefill_poly() {
     return v;
 }
 
-template <int POLY, bool WIN>
+template <int D, int POLY, bool WIN>
 pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
-                            const CUtensorMap &mv, dim3 grid, size_t smem, cudaStream_t st) {
-    auto k = prefill_tc_kernel<POLY, WIN>;
+                            const CUtensorMap &mv, dim3 grid, cudaStream_t st) {
+    const size_t smem = 1024 + pf_smem_bytes(D);
+    auto k = prefill_tc_kernel<D, POLY, WIN>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
     // the kernel's register split must fit the registers it launches with,
     // or the warpgroups that grow would wait forever
@@ -373,6 +374,7 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
     a.H_kv = num_kv_heads;
     a.group = group;
     a.bs = block_size;
+    a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.NB = num_blocks;
     a.MB = max_blocks_per_seq;
     a.max_ctx = max_context_len;
@@ -555,6 +557,7 @@ static pa_status decode_q8_impl(void *out, const void *q, const void *k_cache,
     a.H_kv = num_kv_heads;
     a.group = group;
     a.bs = block_size;
+    a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.NB = num_blocks;
     a.MB = max_blocks_per_seq;
     a.max_ctx = max_context_len;
@@ -624,7 +627,7 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
         return PA_ERR_INVALID_ARG;
     if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
-    if (dtype != PA_BF16 || num_q_heads % num_kv_heads != 0 || head_dim != 128 ||
+    if (dtype != PA_BF16 || num_q_heads % num_kv_heads != 0 || !head_dim_ok(head_dim) ||
         !block_size_ok(block_size))
         return PA_ERR_UNSUPPORTED;
     if (num_chunks == 0 || max_query_len == 0 || num_query_tokens == 0) return PA_OK;
@@ -641,8 +644,10 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     if (!fn) return PA_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     {
-        cuuint64_t dims[3] = {128, (cuuint64_t)num_q_heads, (cuuint64_t)num_query_tokens};
-        cuuint64_t strides[2] = {128 * 2, (cuuint64_t)num_q_heads * 128 * 2};
+        cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads,
+                              (cuuint64_t)num_query_tokens};
+        cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2,
+                                 (cuuint64_t)num_q_heads * head_dim * 2};
         cuuint32_t box[3] = {64, 1, kPfRows};
         cuuint32_t estr[3] = {1, 1, 1};
         if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box,
@@ -650,8 +655,8 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return PA_ERR_CUDA;
     }
-    if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, block_size, 128, 16) ||
-        !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, block_size, 128, 16))
+    if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, block_size, head_dim, 16) ||
+        !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, block_size, head_dim, 16))
         return PA_ERR_CUDA;
 
     PrefillArgs a;
@@ -670,11 +675,13 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     a.window = window;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
-    const size_t smem = 1024 + kPfSmem;
     const dim3 grid((unsigned)qtiles, (unsigned)num_q_heads, (unsigned)num_chunks);
-    if (window > 0) return launch_prefill_tc<0, true>(a, mq, mk, mv, grid, smem, stream);
-    if (prefill_poly() == 4) return launch_prefill_tc<4, false>(a, mq, mk, mv, grid, smem, stream);
-    return launch_prefill_tc<0, false>(a, mq, mk, mv, grid, smem, stream);
+    if (head_dim == 64)
+        return window > 0 ? launch_prefill_tc<64, 0, true>(a, mq, mk, mv, grid, stream)
+                          : launch_prefill_tc<64, 0, false>(a, mq, mk, mv, grid, stream);
+    if (window > 0) return launch_prefill_tc<128, 0, true>(a, mq, mk, mv, grid, stream);
+    if (prefill_poly() == 4) return launch_prefill_tc<128, 4, false>(a, mq, mk, mv, grid, stream);
+    return launch_prefill_tc<128, 0, false>(a, mq, mk, mv, grid, stream);
 }
 
 pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,

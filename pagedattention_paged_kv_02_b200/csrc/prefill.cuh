@@ -59,9 +59,13 @@ constexpr int kPfThreads = 384;   // 2 softmax warpgroups + a control warpgroup
 constexpr int kPfCtlRegs = 56;
 constexpr int kPfSoftmaxRegs = 224;
 constexpr int kPfRegsNeeded = 128 * (2 * kPfSoftmaxRegs + kPfCtlRegs);
-constexpr int kPfTileBytes = kPfRows * 128 * 2;  // 128 x 128 bf16 = 32 KB
 constexpr int kPfTblMax = 4096;   // block-table entries staged in shared memory
-constexpr int kPfSmem = (kPfQTiles + 2 * kPfStages) * kPfTileBytes + 512 + kPfTblMax * 4;
+// A Q, K or V tile: 128 rows of head_dim bf16, as head_dim/64 halves of 128 x
+// 128 bytes (one 128-byte swizzle atom wide), each 16 KB.
+__host__ __device__ constexpr int pf_tile_bytes(int D) { return kPfRows * D * 2; }
+__host__ __device__ constexpr int pf_smem_bytes(int D) {
+    return (kPfQTiles + 2 * kPfStages) * pf_tile_bytes(D) + 512 + kPfTblMax * 4;
+}
 
 struct PrefillArgs {
     __nv_bfloat16 *out;
@@ -236,20 +240,24 @@ __device__ __forceinline__ float ex2_poly(float x) {
 // computed with ex2_poly instead of the special-function unit (0 = none).
 // WIN: the sliding-window build; without it the band logic folds away at
 // compile time and the causal kernel keeps its tighter code.
-template <int POLY, bool WIN>
+// D: head_dim, 64 or 128 (one or two 64-wide halves per row; the S tiles
+// and the P.V accumulators keep their TMEM columns, O using the first D).
+template <int D, int POLY, bool WIN>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    constexpr int TB = pf_tile_bytes(D);
+    constexpr int HALVES = D / 64;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
-    const uint32_t sQ = smem_u32(smem);                         // Q tile x at sQ + x*32K
-    const uint32_t sK = sQ + kPfQTiles * kPfTileBytes;          // K stage st at sK + st*32K
-    const uint32_t sV = sK + kPfStages * kPfTileBytes;          // V stage st at sV + st*32K
-    PfBars *bars = reinterpret_cast<PfBars *>(smem + (kPfQTiles + 2 * kPfStages) * kPfTileBytes);
-    int32_t *tbl = reinterpret_cast<int32_t *>(smem + (kPfQTiles + 2 * kPfStages) * kPfTileBytes +
-                                               512);
+    const uint32_t sQ = smem_u32(smem);            // Q tile x at sQ + x*TB
+    const uint32_t sK = sQ + kPfQTiles * TB;       // K stage st at sK + st*TB
+    const uint32_t sV = sK + kPfStages * TB;       // V stage st at sV + st*TB
+    PfBars *bars = reinterpret_cast<PfBars *>(smem + (kPfQTiles + 2 * kPfStages) * TB);
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + (kPfQTiles + 2 * kPfStages) * TB + 512);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tp = blockIdx.x, h = blockIdx.y;
@@ -338,11 +346,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // of a K or V tile (8 pieces of 16 tokens x 2 halves of 64 dims)
         // go out from 16 lanes at once. Lane 0 arms the barrier first with
         // the exact byte count of the pieces that exist.
-        const int s16 = lane >> 1, half = lane & 1;
+        const int s16 = lane / HALVES, half = lane % HALVES;
         auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j) {
             const int key = j * kPfKeys + s16 * 16;
             int id = -1;
-            if (lane < 16 && key < ctx && (!WIN || key + 15 >= chunk_lo)) {
+            if (lane < 8 * HALVES && key < ctx && (!WIN || key + 15 >= chunk_lo)) {
                 const int lb = key / a.bs;
                 if (lb - blk0 < kPfTblMax) {
                     id = tbl[lb - blk0];
@@ -362,11 +370,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             key % a.bs, kvh, id);
         };
         const int nq = rows1 > 0 ? 2 : 1;
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * kPfTileBytes);
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * TB);
         __syncwarp();
-        if (lane < 2 * nq) {
-            const int x = lane >> 1, hf = lane & 1;
-            tma_load_3d(sQ + x * kPfTileBytes + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64,
+        if (lane < HALVES * nq) {
+            const int x = lane / HALVES, hf = lane % HALVES;
+            tma_load_3d(sQ + x * TB + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64,
                         h, q0 + row0 + x * kPfRows);
         }
         int k_issued = 0, v_issued = 0;  // counted from jmin
@@ -375,11 +383,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const uint32_t use = (j - jmin) / kPfStages;
             if (use > 0 && !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
                 break;
-            issue(sK + st * kPfTileBytes, &tmk, &bars->k_full[st], j);
+            issue(sK + st * TB, &tmk, &bars->k_full[st], j);
             k_issued = j - jmin + 1;
             if (use > 0 && !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
                 break;
-            issue(sV + st * kPfTileBytes, &tmv, &bars->v_full[st], j);
+            issue(sV + st * TB, &tmv, &bars->v_full[st], j);
             v_issued = j - jmin + 1;
         }
         if (bars->abort && lane == 0) {  // let copies already in flight land
@@ -395,16 +403,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             constexpr uint32_t kIdQK = f16_idesc(128, 128, false);
-            constexpr uint32_t kIdPV = f16_idesc(128, 128, true);
+            constexpr uint32_t kIdPV = f16_idesc(128, D, true);
             auto issue_s = [&](int x, int j) -> bool {  // S_x = Q_x K_j^T
                 const int st = (j - jmin) % kPfStages;
                 if (!pf_wait(bars, &bars->k_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
                              false))
                     return false;
                 tc_fence_after();
-                const uint32_t q = sQ + x * kPfTileBytes, k = sK + st * kPfTileBytes;
+                const uint32_t q = sQ + x * TB, k = sK + st * TB;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
+                for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
                     mma_ss(tmem + x * 128, sw128_desc(q + koff, 16, 1024),
                            sw128_desc(k + koff, 16, 1024), kIdQK, ks > 0);
@@ -420,7 +428,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                              false))
                     return false;
                 tc_fence_after();
-                const uint32_t v = sV + st * kPfTileBytes;
+                const uint32_t v = sV + st * TB;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     mma_ts(tmem + 256 + x * 128, tmem + x * 128 + ks * 8,
@@ -534,7 +542,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 l *= corr;
                 m = m_new;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t v[32];
                     tmem_ld32(tO + cc * 32, v);
                     tmem_ld_wait();
@@ -599,10 +607,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     ok = false;
                     break;
                 }
-                const uint32_t vb = sV + st * kPfTileBytes;
+                const uint32_t vb = sV + st * TB;
                 const int nz = z0 + (kPfKeys - z1);  // rows [0, z0) and [z1, 128)
-                for (int e = r; e < nz * 16; e += 128) {
-                    const int zr = e / 16, u = e % 16;
+                for (int e = r; e < nz * (D / 8); e += 128) {  // 16-byte units of a row
+                    const int zr = e / (D / 8), u = e % (D / 8);
                     const int row = zr < z0 ? zr : z1 + (zr - z0);
                     const uint32_t addr = vb + (u / 8) * 16384 + row * 128 + (u % 8) * 16;
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
@@ -617,9 +625,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             pf_wait(bars, &bars->o_full[x], (j1 - j0 - 1) & 1, a.timeout_ns, true)) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + h) * 128;
+            __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + h) * D;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t v[32];
                 tmem_ld32(tO + cc * 32, v);
                 tmem_ld_wait();

@@ -130,7 +130,7 @@ def test_prefill_host_checks(L):
     assert len(base) == 19
     assert f(*base[:17], 0, None) == pa.PA_ERR_UNSUPPORTED  # fp32 has no tensor-core path
     b = list(base)
-    b[12] = 64
+    b[12] = 96  # head_dim 64 and 128 only
     assert f(*b) == pa.PA_ERR_UNSUPPORTED
     b = list(base)
     b[10], b[11] = 12, 8

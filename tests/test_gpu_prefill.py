@@ -59,18 +59,18 @@ CASES = [
 ]
 
 
-def mixed_chunks(cached, lens, Hq, Hkv, bs, seed):
+def mixed_chunks(cached, lens, Hq, Hkv, bs, seed, D=128):
     """Chunks of differing lengths: built one length at a time, then merged."""
     nb = sum(-(-(c + n) // bs) for c, n in zip(cached, lens)) + 8
     gen = torch.Generator().manual_seed(seed)
     from pagedattention_paged_kv_02_b200.workloads import SeqSpec, build_pool, Batch, _randn
     specs = [SeqSpec(c + n, n) for c, n in zip(cached, lens)]
-    k, v, tables, key, value, slots, poison = build_pool(specs, Hkv, 128, bs, nb,
+    k, v, tables, key, value, slots, poison = build_pool(specs, Hkv, D, bs, nb,
                                                          torch.bfloat16, 1.0, gen)
     qsl = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()), dtype=torch.int32)
-    q = _randn(gen, (int(qsl[-1]), Hq, 128), 1.0, torch.bfloat16)
+    q = _randn(gen, (int(qsl[-1]), Hq, D), 1.0, torch.bfloat16)
     return Batch(name="chunks", k_cache=k, v_cache=v, key=key, value=value, slot_mapping=slots,
-                 scale=128 ** -0.5, block_size=bs, poison_block=poison, prefill_q=q,
+                 scale=D ** -0.5, block_size=bs, poison_block=poison, prefill_q=q,
                  prefill_block_tables=tables,
                  prefill_context_lens=torch.tensor([s.ctx for s in specs], dtype=torch.int32),
                  query_start_loc=qsl)
@@ -84,6 +84,17 @@ def test_prefill_small(pa, case):
     k, v = oracle_after_append(batch)
     ref, _ = oracle_prefill(batch, k, v)
     assert_close(out, ref, f"prefill {case}")
+    assert pa.pa_device_error() == 0
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"h{c[1]}kv{c[2]}-bs{c[3]}-{max(c[0][1])}q")
+def test_prefill_head_dim_64(pa, case):
+    (cached, lens), Hq, Hkv, bs = case
+    batch = mixed_chunks(cached, lens, Hq, Hkv, bs, seed=sum(lens) + Hq + 64, D=64)
+    d, out = run_prefill(pa, batch)
+    k, v = oracle_after_append(batch)
+    ref, _ = oracle_prefill(batch, k, v)
+    assert_close(out, ref, f"prefill D64 {case}")
     assert pa.pa_device_error() == 0
 
 

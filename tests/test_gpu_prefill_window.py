@@ -75,6 +75,15 @@ def test_blocks_before_the_band_are_never_read(pa, window):
     assert_close(out, reference(batch, window), f"freed prefix, window {window}")
 
 
+@pytest.mark.parametrize("window", [1, 100, 129])
+def test_prefill_window_head_dim_64(pa, window):
+    (cached, lens), Hq, Hkv, bs = CASES[0]
+    batch = mixed_chunks(cached, lens, Hq, Hkv, bs, seed=97 + window, D=64)
+    _, out = run(pa, batch, window)
+    assert_close(out, reference(batch, window), f"prefill D64 window {window}")
+    assert pa.pa_device_error() == 0
+
+
 def test_window_covering_everything_is_plain_prefill(pa):
     (cached, lens), Hq, Hkv, bs = CASES[1]
     batch = mixed_chunks(cached, lens, Hq, Hkv, bs, seed=95)
