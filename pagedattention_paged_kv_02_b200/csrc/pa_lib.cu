@@ -297,15 +297,17 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache
     a.k_cache = static_cast<uint4 *>(k_cache);
     a.v_cache = static_cast<uint4 *>(v_cache);
     a.slot_mapping = slot_mapping;
-    a.vecs_per_row = head_dim * elem / 16;
-    a.vecs_per_token = num_kv_heads * a.vecs_per_row;
-    a.total_vecs = (long long)num_tokens * a.vecs_per_token;
+    const int vecs_per_row = head_dim * elem / 16;  // 8, 16 or 32: a power of two
+    if ((long long)num_kv_heads * vecs_per_row > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    a.num_tokens = num_tokens;
+    a.vecs_per_token = num_kv_heads * vecs_per_row;
+    a.row_shift = __builtin_ctz((unsigned)vecs_per_row);
+    a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.num_kv_heads = num_kv_heads;
-    a.block_size = block_size;
     a.num_slots = (long long)num_blocks * block_size;
-    const long long blocks = (a.total_vecs + 255) / 256;
-    if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-    reshape_and_cache_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    const dim3 grid((unsigned)((a.vecs_per_token + kScatterThreads - 1) / kScatterThreads),
+                    (unsigned)(num_tokens < 65535 ? num_tokens : 65535));
+    reshape_and_cache_kernel<<<grid, kScatterThreads, 0, stream>>>(a);
     return launch_status();
 }
 
@@ -466,19 +468,21 @@ static pa_status reshape_q8_impl(const void *key, const void *value, void *k_cac
     a.slot_mapping = slot_mapping;
     a.k_scale = k_scale;
     a.v_scale = v_scale;
-    a.vecs_per_row = head_dim / 16;
-    a.vecs_per_token = num_kv_heads * a.vecs_per_row;
-    a.total_vecs = (long long)num_tokens * a.vecs_per_token;
+    const int vecs_per_row = head_dim / 16;  // 4 or 8: a power of two
+    if ((long long)num_kv_heads * vecs_per_row > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    a.num_tokens = num_tokens;
+    a.vecs_per_token = num_kv_heads * vecs_per_row;
+    a.row_shift = __builtin_ctz((unsigned)vecs_per_row);
+    a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.num_kv_heads = num_kv_heads;
-    a.block_size = block_size;
     a.num_slots = (long long)num_blocks * block_size;
     a.bf16_in = dtype == PA_BF16;
-    const long long blocks = (a.total_vecs + 255) / 256;
-    if (blocks > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)((a.vecs_per_token + kScatterThreads - 1) / kScatterThreads),
+                    (unsigned)(num_tokens < 65535 ? num_tokens : 65535));
     if (int8)
-        reshape_and_cache_int8_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+        reshape_and_cache_int8_kernel<<<grid, kScatterThreads, 0, stream>>>(a);
     else
-        reshape_and_cache_e4m3_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+        reshape_and_cache_e4m3_kernel<<<grid, kScatterThreads, 0, stream>>>(a);
     return launch_status();
 }
 
