@@ -240,7 +240,7 @@ def pa_prefill_chunk_sliding_window(out, q, k_cache, v_cache, block_tables, cont
           _dt(q), _stream(stream))
 
 
-def _fp8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype=torch.uint8):
+def _q8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype=torch.uint8):
     if k_cache.dtype != code_dtype or v_cache.dtype != code_dtype:
         raise TypeError("FP8 caches are uint8 tensors of E4M3 codes, INT8 caches int8 tensors")
     H_kv = k_cache.shape[1]
@@ -252,7 +252,7 @@ def _fp8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype=torch.uint8):
 def _reshape_q8(fn, code_dtype, key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
                 stream):
     _check_int(slot_mapping, torch.int64, "slot_mapping")
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype)
+    _q8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype)
     NB, H_kv, bs, D = k_cache.shape
     T = slot_mapping.numel()
     if key.shape != (T, H_kv, D) or value.shape != (T, H_kv, D) or key.dtype != value.dtype:
@@ -265,7 +265,7 @@ def _decode_q8(fn, code_dtype, out, q, k_cache, v_cache, k_scale, v_scale, block
                context_lens, max_context_len, scale, partition_size, workspace, stream):
     _check_int(block_tables, torch.int32, "block_tables")
     _check_int(context_lens, torch.int32, "context_lens")
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype)
+    _q8_pool(k_cache, v_cache, k_scale, v_scale, code_dtype)
     B, H_q, D = q.shape
     NB, H_kv, bs, D2 = k_cache.shape
     if out.shape != q.shape or D2 != D or q.dtype != torch.bfloat16 or out.dtype != q.dtype:
@@ -447,7 +447,7 @@ def prepare_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_
     """``pa_reshape_and_cache_fp8``, or ``pa_reshape_and_cache_int8`` for int8 caches."""
     _check_int(slot_mapping, torch.int64, "slot_mapping")
     int8 = k_cache.dtype == torch.int8
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale, torch.int8 if int8 else torch.uint8)
+    _q8_pool(k_cache, v_cache, k_scale, v_scale, torch.int8 if int8 else torch.uint8)
     NB, H_kv, bs, D = k_cache.shape
     return Prepared("pa_reshape_and_cache_int8" if int8 else "pa_reshape_and_cache_fp8",
                     (_p(key), _p(value), _p(k_cache), _p(v_cache), _p(slot_mapping),
@@ -459,7 +459,7 @@ def prepare_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables,
                        workspace: Optional[torch.Tensor] = None) -> Prepared:
     """``pa_decode_fp8``, or ``pa_decode_int8`` for int8 caches."""
     int8 = k_cache.dtype == torch.int8
-    _fp8_pool(k_cache, v_cache, k_scale, v_scale, torch.int8 if int8 else torch.uint8)
+    _q8_pool(k_cache, v_cache, k_scale, v_scale, torch.int8 if int8 else torch.uint8)
     B, H_q, D = q.shape
     NB, H_kv, bs, _ = k_cache.shape
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
