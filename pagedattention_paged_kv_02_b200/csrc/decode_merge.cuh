@@ -47,7 +47,10 @@ __global__ void __launch_bounds__(256) decode_reduce_warp(const __grid_constant_
     wait_for_primary_grid();
     const float *lse = a.part_lse + (size_t)bh * a.S_max;
     const float *po = a.part_o + (size_t)bh * a.S_max * D + lane * VEC;
-    float M = lane < n ? __ldcg(lse + lane) : -INFINITY;
+    // lane s holds lse_s: one load for all of them, then shuffles (no second
+    // round trip before the partials' loads, which are independent)
+    const float my_lse = lane < n ? __ldcg(lse + lane) : -INFINITY;
+    float M = my_lse;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float acc[VEC];
@@ -55,8 +58,9 @@ __global__ void __launch_bounds__(256) decode_reduce_warp(const __grid_constant_
     for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
     float W = 0.f;
     if (M != -INFINITY) {
+#pragma unroll 4
         for (int s = 0; s < n; ++s) {
-            const float w = exp2f(__ldcg(lse + s) - M);
+            const float w = exp2f(__shfl_sync(0xffffffffu, my_lse, s) - M);
             W += w;
             if constexpr (VEC == 4) {
                 const float4 x = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)s * D));
