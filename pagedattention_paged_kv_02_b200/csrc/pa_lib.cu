@@ -677,6 +677,7 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     a.NB = num_blocks;
     a.MB = max_blocks_per_seq;
     a.window = window;
+    a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
     const dim3 grid((unsigned)qtiles, (unsigned)num_q_heads, (unsigned)num_chunks);

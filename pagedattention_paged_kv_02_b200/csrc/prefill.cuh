@@ -74,6 +74,7 @@ struct PrefillArgs {
     const int32_t *qsl;
     int n_chunks, total_q, H_q, H_kv, group, bs, NB, MB;
     int window;  // > 0: query at position p sees keys p-window+1 .. p only
+    int bs_shift;  // log2(bs)
     float scale_log2;
     unsigned long long timeout_ns;
 };
@@ -351,7 +352,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int key = j * kPfKeys + s16 * 16;
             int id = -1;
             if (lane < 8 * HALVES && key < ctx && (!WIN || key + 15 >= chunk_lo)) {
-                const int lb = key / a.bs;
+                const int lb = key >> a.bs_shift;
                 if (lb - blk0 < kPfTblMax) {
                     id = tbl[lb - blk0];
                 } else {
@@ -367,7 +368,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             __syncwarp();
             if (id >= 0)
                 tma_load_4d(dst + half * 16384 + s16 * 2048, map, smem_u32(bar), half * 64,
-                            key % a.bs, kvh, id);
+                            key & (a.bs - 1), kvh, id);
         };
         const int nq = rows1 > 0 ? 2 : 1;
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * TB);
