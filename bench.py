@@ -344,15 +344,15 @@ class Runner:
                                             self.host.sliding_window)
         return c
 
-    def step(self, ev=None, calls=None):
+    def step(self, ev=None, calls=None, stream=None):
         """One pass; ``ev`` (start, end) events bracket the dominant call."""
         c = calls or self._calls
-        c["reshape"]()
+        c["reshape"](stream)
         for name in ("prefill", "decode"):
             if name in c:
                 if ev is not None and name == self.dominant:
                     ev[0].record()
-                c[name]()
+                c[name](stream)
                 if ev is not None and name == self.dominant:
                     ev[1].record()
 
@@ -388,10 +388,27 @@ def run_ours(args, rank, world):
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
-    # the step, back to back, timed as a whole (no events between steps)
+    # the step, back to back, timed as a whole (no events between steps):
+    # its launches captured once in a CUDA graph and replayed (launch-bound
+    # steps such as the tiny batch run 3x faster), or issued one by one with
+    # --eager; the calls marshal nothing per step either way
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                r.step(stream=side)
+        torch.cuda.current_stream().wait_stream(side)
+        graph.replay()
+        torch.cuda.synchronize()
     t0.record()
     for i in range(K):
-        r.step()
+        if graph is not None:
+            graph.replay()
+        else:
+            r.step()
     t1.record()
     torch.cuda.synchronize()
     # the same K steps again, events around the dominant call of each, for
@@ -528,7 +545,7 @@ def run_ours(args, rank, world):
             "dtype": ("e4m3 KV / bf16 q" if batch.fp8 else "int8 KV / bf16 q" if batch.int8 else
                       "bf16" if batch.dtype.itemsize == 2 else "f32"),
             "data": "synthetic (seeded; one batch per rank)",
-            "config": workload_config(batch, args.workload, world, r),
+            "config": {**workload_config(batch, args.workload, world, r), **_graph_note(args)},
             "tokens_per_s": round(tok_total / (ms * 1e-3), 1),
             "frac_of_hbm_peak": round(value / world / hbm, 4),
             "frac_of_nominal_8tbs": round(value / world / 8000.0, 4),
@@ -577,6 +594,10 @@ def workload_config(batch, name, world, r=None):
     if batch.sliding_window > 0:
         c["sliding_window"] = batch.sliding_window
     return c
+
+
+def _graph_note(args):
+    return {"launch": "cuda_graph_replay" if getattr(args, "graph", False) else "eager"}
 
 
 # --------------------------------------------------------------------------
@@ -770,6 +791,9 @@ def main(argv=None):
     ap.add_argument("--window", type=int, default=0,
                     help="sliding window: each query sees only its last W positions "
                          "(0: the whole context); not for the FP8 workloads")
+    ap.add_argument("--eager", dest="graph", action="store_false",
+                    help="time the step as individual launches instead of replays of one "
+                         "CUDA graph capture of it")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     args = ap.parse_args(argv)
