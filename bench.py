@@ -115,6 +115,24 @@ def decode_bytes(batch) -> float:
     return float(kv + qo + tbl + 4 * batch.num_seqs)
 
 
+def decode_unique_bytes(batch) -> float:
+    """K/V bytes of the distinct cached tokens the decode sequences read:
+    sequences that share prefix blocks count them once (what HBM must
+    deliver at least once; the logical bytes count every reader)."""
+    import torch
+    if batch.q is None or batch.num_seqs == 0:
+        return 0.0
+    bs = batch.block_size
+    used = {}
+    tables = batch.block_tables.tolist()
+    for b, ctx in enumerate(batch.context_lens.tolist()):
+        for lb in range(-(-ctx // bs)):
+            blk = tables[b][lb]
+            used[blk] = max(used.get(blk, 0), min(bs, ctx - lb * bs))
+    e = batch.k_cache.element_size()
+    return float(2 * sum(used.values()) * batch.num_kv_heads * batch.head_dim * e)
+
+
 def reshape_bytes(batch) -> float:
     """Algorithmic bytes of the cache scatter: read and write K and V rows of
     every non-padding token, plus the slots."""
@@ -560,6 +578,10 @@ def run_ours(args, rank, world):
         }
         if r.dominant != "decode":
             line["prefill_tflops"] = round(pflops * world / (ms * 1e-3) / 1e12, 1)
+            # the decode part of the mixed step reads shared prefix blocks
+            # through many tables: logical bytes (value) and distinct bytes
+            line["decode_bytes_per_step"] = {"logical": dbytes,
+                                             "unique_kv": decode_unique_bytes(batch)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(batch, args.cpu_seconds)
     if world > 1:

@@ -2,6 +2,8 @@
 without a sliding window, and the reference arm (the oracle) with a window."""
 import json
 
+import torch
+
 import bench
 from pagedattention_paged_kv_02_b200 import workloads as W
 
@@ -71,3 +73,17 @@ def test_committed_profiles_match_the_sources():
         else:
             files = bench.DECODE_SOURCES
         assert bench.profiled_traffic(name, files) is not None, f"{name} is stale"
+
+
+def test_unique_bytes_count_shared_prefix_blocks_once():
+    """Without sharing, the distinct K/V bytes are the logical K/V bytes; the
+    mixed batch's 24 beam groups share a 64-block prefix, read 8 times each."""
+    b = W.llama7b_decode()
+    ctx = b.context_lens.to(torch.int64)
+    kv = int((2 * ctx * b.num_kv_heads * b.head_dim * b.k_cache.element_size()).sum())
+    assert bench.decode_unique_bytes(b) == kv
+    m = W.mixed_prefill_decode()
+    per_token = 2 * m.num_kv_heads * m.head_dim * m.k_cache.element_size()
+    logical = int(m.context_lens.to(torch.int64).sum()) * per_token
+    shared = 24 * 7 * 1024 * per_token  # 7 of each group's 8 readers of its prefix
+    assert bench.decode_unique_bytes(m) == logical - shared
