@@ -641,8 +641,7 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
         return PA_ERR_INVALID_ARG;
     const long long qtiles = (max_query_len + kPfRows * kPfQTiles - 1) / (kPfRows * kPfQTiles);
-    if (num_q_heads > 65535 || num_chunks > 65535 || qtiles > 0x7fffffffLL)
-        return PA_ERR_UNSUPPORTED;
+    if (qtiles > 65535 || num_chunks > 65535) return PA_ERR_UNSUPPORTED;
 
     EncodeTiledFn fn = encode_fn();
     if (!fn) return PA_ERR_CUDA;
@@ -680,7 +679,7 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
-    const dim3 grid((unsigned)qtiles, (unsigned)num_q_heads, (unsigned)num_chunks);
+    const dim3 grid((unsigned)num_q_heads, (unsigned)qtiles, (unsigned)num_chunks);
     if (head_dim == 64)
         return window > 0 ? launch_prefill_tc<64, 0, true>(a, mq, mk, mv, grid, stream)
                           : launch_prefill_tc<64, 0, false>(a, mq, mk, mv, grid, stream);

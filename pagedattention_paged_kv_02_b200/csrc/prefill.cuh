@@ -261,8 +261,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int32_t *tbl = reinterpret_cast<int32_t *>(smem + (kPfQTiles + 2 * kPfStages) * TB + 512);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tp = blockIdx.x, h = blockIdx.y;
-    const int c = a.n_chunks - 1 - (int)blockIdx.z;  // later (longer) chunks first
+    // CTAs start in order of decreasing work (the scheduler hands them out
+    // in launch order): the last chunk first, within it the last query-tile
+    // pair first, every query head of one pair before the next pair
+    const int h = blockIdx.x;
+    const int tp = (int)gridDim.y - 1 - (int)blockIdx.y;
+    const int c = a.n_chunks - 1 - (int)blockIdx.z;
     const int q0 = a.qsl[c];
     const int C = a.qsl[c + 1] - q0;
     const int row0 = tp * kPfRows * kPfQTiles;  // first query of this CTA within the chunk
@@ -292,7 +296,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int jmin = jlo0, jmax = max(jhi0, jhi1);  // K/V tiles this CTA streams
     const int kvh = h / a.group;
 
-    if (threadIdx.x == 0) {
+    const int nq = rows1 > 0 ? 2 : 1;  // Q tiles with rows
+    if (warp == 8) {
+      if (lane == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
         for (int st = 0; st < kPfStages; ++st) {
             mbar_init(smem_u32(&bars->k_full[st]), 1);
@@ -308,6 +314,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_init(smem_u32(&bars->fin), 1);
         bars->abort = 0;
         fence_mbar_init();
+      }
+      __syncwarp();
+      // the Q tiles need no table: their copy overlaps the table staging below
+      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * TB);
+      __syncwarp();
+      if (lane < HALVES * nq) {
+          const int x = lane / HALVES, hf = lane % HALVES;
+          tma_load_3d(sQ + x * TB + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64, h,
+                      q0 + row0 + x * kPfRows);
+      }
     }
     if (warp == 9) {
         tmem_alloc(smem_u32(&bars->tmem_base), 512);
@@ -370,14 +386,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 tma_load_4d(dst + half * 16384 + s16 * 2048, map, smem_u32(bar), half * 64,
                             key & (a.bs - 1), kvh, id);
         };
-        const int nq = rows1 > 0 ? 2 : 1;
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars->q_full), nq * TB);
-        __syncwarp();
-        if (lane < HALVES * nq) {
-            const int x = lane / HALVES, hf = lane % HALVES;
-            tma_load_3d(sQ + x * TB + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64,
-                        h, q0 + row0 + x * kPfRows);
-        }
         int k_issued = 0, v_issued = 0;  // counted from jmin
         for (int j = jmin; j < jmax; ++j) {
             const int st = (j - jmin) % kPfStages;
