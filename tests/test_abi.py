@@ -144,6 +144,14 @@ def test_prefill_host_checks(L):
     b = list(base)
     b[7] = 0
     assert f(*b) == pa.PA_OK
+    # the grid is (query head, tile pair, chunk): at most 65535 pairs of 256 queries and
+    # 65535 chunks; any number of query heads
+    b = list(base)
+    b[8], b[9] = 65536 * 256, 65536 * 256
+    assert f(*b) == pa.PA_ERR_UNSUPPORTED
+    b = list(base)
+    b[7] = 65536
+    assert f(*b) == pa.PA_ERR_UNSUPPORTED
 
 
 def test_prefill_window_host_checks(L):
