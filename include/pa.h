@@ -241,8 +241,9 @@ PA_API pa_status pa_decode_sliding_window(void *out, const void *q, const void *
  *                     chunk reaching past it, or with context_lens[c] < C_c,
  *                     is skipped and recorded as PA_ERR_BAD_TABLE.
  *   max_query_len     host-side upper bound of every C_c.
- * bf16 with head_dim 64 or 128 (the tcgen05 tensor-core path); anything else
- * returns PA_ERR_UNSUPPORTED. */
+ * bf16 with head_dim 64 or 128 (the tcgen05 tensor-core path), at most
+ * 65535 chunks and max_query_len at most 65535 * 256; anything else returns
+ * PA_ERR_UNSUPPORTED. */
 PA_API pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
                            const int32_t *block_tables, const int32_t *context_lens,
                            const int32_t *query_start_loc, int num_chunks, int num_query_tokens,
