@@ -134,11 +134,13 @@ def decode_unique_bytes(batch) -> float:
 
 
 def reshape_bytes(batch) -> float:
-    """Algorithmic bytes of the cache scatter: read and write K and V rows of
-    every non-padding token, plus the slots."""
-    e = batch.k_cache.element_size()
+    """Algorithmic bytes of the cache scatter: read the K and V rows of every
+    non-padding token (input element size), write them into the cache (cache
+    element size: 1 for the 8-bit pools), plus the slots."""
     T = int((batch.slot_mapping >= 0).sum())
-    return float(2 * 2 * T * batch.num_kv_heads * batch.head_dim * e + 8 * batch.slot_mapping.numel())
+    rows = 2 * T * batch.num_kv_heads * batch.head_dim  # K and V elements
+    return float(rows * (batch.key.element_size() + batch.k_cache.element_size()) +
+                 8 * batch.slot_mapping.numel())
 
 
 def prefill_flops(batch) -> float:
@@ -362,10 +364,15 @@ class Runner:
                                             self.host.sliding_window)
         return c
 
-    def step(self, ev=None, calls=None, stream=None):
-        """One pass; ``ev`` (start, end) events bracket the dominant call."""
+    def step(self, ev=None, calls=None, stream=None, rev=None):
+        """One pass; ``ev`` (start, end) events bracket the dominant call,
+        ``rev`` the cache scatter."""
         c = calls or self._calls
+        if rev is not None:
+            rev[0].record()
         c["reshape"](stream)
+        if rev is not None:
+            rev[1].record()
         for name in ("prefill", "decode"):
             if name in c:
                 if ev is not None and name == self.dominant:
@@ -433,14 +440,17 @@ def run_ours(args, rank, world):
     # its roofline
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
+    revs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(K)]
     for i in range(K):
-        r.step(evs[i])
+        r.step(evs[i], rev=revs[i])
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier(world)
     ms_local = t0.elapsed_time(t1) / K
     dom_all = sorted(a.elapsed_time(b) for a, b in evs)
     dom_ms = statistics.fmean(dom_all)
+    rs_ms = statistics.fmean(a.elapsed_time(b) for a, b in revs)
     pct = lambda q: dom_all[min(len(dom_all) - 1, int(q * len(dom_all)))]
 
     units = dbytes if r.dominant == "decode" else pflops
@@ -576,6 +586,14 @@ def run_ours(args, rank, world):
             "dominant_call_ms": {"mean": round(dom_ms, 5), "p10": round(pct(0.1), 5),
                                  "p50": round(pct(0.5), 5), "p90": round(pct(0.9), 5)},
         }
+        # the cache scatter against HBM: its algorithmic bytes over its own
+        # event-timed duration (the same pass as the dominant call's)
+        line["roofline_reshape"] = {
+            "bound": "hbm", "achieved": round(rbytes / (rs_ms * 1e-3) / 1e9, 1), "peak": hbm,
+            "unit": "GB/s", "frac": round(rbytes / (rs_ms * 1e-3) / 1e9 / hbm, 4),
+            "peak_basis": f"{basis} hbm_gbs", "kernel": "pa_reshape_and_cache",
+            "alg_bytes_per_launch": rbytes, "ms": round(rs_ms, 5),
+            "traffic": profiled_traffic(f"reshape_{args.workload}.md", RESHAPE_SOURCES)}
         if r.dominant != "decode":
             line["prefill_tflops"] = round(pflops * world / (ms * 1e-3) / 1e12, 1)
             # the decode part of the mixed step reads shared prefix blocks
@@ -596,6 +614,8 @@ DECODE_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/decode.cuh",
 PREFILL_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/prefill.cuh",
                    "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
 DECODE_FP8_SOURCES = DECODE_SOURCES + ["pagedattention_paged_kv_02_b200/csrc/decode_fp8.cuh"]
+RESHAPE_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/reshape_and_cache.cuh",
+                   "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
 
 
 def workload_config(batch, name, world, r=None):

@@ -199,13 +199,20 @@ PA_API pa_status pa_decode_int8(void *out, const void *q, const void *k_cache, c
  * the library, which every GPU that loads the library keeps until exit.
  *   - A request whose workspace (pa_decode_workspace_size) exceeds 16 MiB is
  *     refused with PA_ERR_WORKSPACE before anything is launched.
- *   - The first call on a device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *   - Set-up: the first call in a CUDA context (per device; again after
+ *     cudaDeviceReset) looks up the array's device address with that device
+ *     current. With lazy module loading, CUDA's default, that first call --
+ *     or the first launch of any libpa kernel on the device, whichever comes
+ *     first -- also loads the library's device code and so reserves the
+ *     16 MiB, which allocates and can synchronise. A call with num_seqs = 0
+ *     does this set-up and launches nothing: make it at start-up, before
+ *     any stream capture.
  *   - All calls share the one array: two calls whose kernels overlap on the
  *     GPU (different streams, no ordering between them) race and may return
  *     wrong results. Calls ordered on one stream are safe; nothing needs to
  *     be cleared between them.
- *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call). */
+ *   - After set-up, allocates nothing (no cudaMalloc, cudaFree or allocating
+ *     library call). */
 PA_API pa_status pa_decode_static_workspace(void *out, const void *q, const void *k_cache,
                                             const void *v_cache, const int32_t *block_tables,
                                             const int32_t *context_lens, int num_seqs,
@@ -238,9 +245,14 @@ PA_API pa_status pa_decode_sliding_window(void *out, const void *q, const void *
  * sits at position p = context_lens[c] - C_c + i and attends positions 0..p:
  *   out[r][h] = sum_{j<=p} softmax_j(scale * q[r][h] . K_j) V_j,  r = qsl[c]+i.
  *   num_query_tokens  rows of q and out (query_start_loc[num_chunks]); a
- *                     chunk reaching past it, or with context_lens[c] < C_c,
- *                     is skipped and recorded as PA_ERR_BAD_TABLE.
- *   max_query_len     host-side upper bound of every C_c.
+ *                     chunk reaching past it, with C_c < 0 (decreasing
+ *                     query_start_loc), with context_lens[c] < C_c or above
+ *                     max_blocks_per_seq*block_size is skipped and recorded
+ *                     as PA_ERR_BAD_TABLE.
+ *   max_query_len     host-side upper bound of every C_c. The launch covers
+ *                     max_query_len rounded up to a multiple of 256 rows per
+ *                     chunk; the rows of a longer chunk past that are left
+ *                     unwritten and the chunk is recorded as PA_ERR_BAD_TABLE.
  * bf16 with head_dim 64 or 128 (the tcgen05 tensor-core path), at most
  * 65535 chunks and max_query_len at most 65535 * 256; anything else returns
  * PA_ERR_UNSUPPORTED. */

@@ -52,28 +52,12 @@ __device__ __forceinline__ void e4m3x4_to_f16x2_hw(uint32_t w, uint32_t &lo, uin
         : "r"(w));
 }
 
-
 // 2^x on the special-function unit, subnormal results flushed to zero (a
 // softmax weight below 2^-126 of the row's largest does not register).
 __device__ __forceinline__ float ex2_fast(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// Four E4M3 codes w = [c0 c1 c2 c3] (c0 the low byte) -> the f16 pairs
-// {c0, c2} (even) and {c1, c3} (odd), each half equal to its code's value
-// times 2^-8, on the integer pipe: the code's sign goes to bit 15 and its
-// seven magnitude bits to bits 13..7, so the 4-bit exponent field becomes the
-// low four bits of f16's 5-bit field (biases 7 and 15: a factor 2^-8) and the
-// 3-bit mantissa the top of f16's; subnormal codes become f16 subnormals with
-// the same factor. Exact for every finite code; the two NaN codes (0x7f,
-// 0xff), which the quantising append never writes, come out finite (+-480
-// once the 2^8 is put back).
-__device__ __forceinline__ void e4m3x4_to_f16x2_scaled(uint32_t w, uint32_t &even,
-                                                       uint32_t &odd) {
-    odd = (w & 0x80008000u) | ((w >> 1) & 0x3F803F80u);
-    even = ((w << 8) & 0x80008000u) | ((w << 7) & 0x3F803F80u);
 }
 
 // Four INT8 codes w = [c0 c1 c2 c3] (c0 the low byte) -> the f16 pairs
@@ -87,16 +71,6 @@ __device__ __forceinline__ void int8x4_to_f16x2(uint32_t w, uint32_t &even, uint
     const uint32_t o = __byte_perm(u, 0x64646464u, 0x4341);  // [c1', 0x64, c3', 0x64]
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(even) : "r"(e), "r"(0x64806480u));
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(odd) : "r"(o), "r"(0x64806480u));
-}
-
-// The even/odd f16 pairs of a word of four codes, for the integer-pipe forms
-// of decode_split_q8 (CV 1, 2: E4M3 times 2^-8; CV 3: INT8).
-template <int CV>
-__device__ __forceinline__ void codes_to_f16x2(uint32_t w, uint32_t &even, uint32_t &odd) {
-    if constexpr (CV == 3)
-        int8x4_to_f16x2(w, even, odd);
-    else
-        e4m3x4_to_f16x2_scaled(w, even, odd);
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -115,15 +89,10 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
 // CT: tokens per pipeline stage (16 or 32). A 32-token stage is two
 // 16-token page pieces (each inside one physical block, so each has its own
 // table lookup); it halves the softmax and hand-off work per byte.
-// CV: the code format and where codes become f16. E4M3: 0 = the conversion
-// instruction for K and V; 1 = K on the integer pipe
-// (e4m3x4_to_f16x2_scaled), V by instruction; 2 = both on the integer pipe
-// (the 2^-8 of the integer form folds into the scales). The conversion
-// instruction shares a narrow pipe with the exponentials, but the E4M3
-// integer form costs 3.5 instructions per pair and measured slower on B200,
-// so 0 is the E4M3 default. INT8: 3 = both on the integer and FMA pipes
-// (int8x4_to_f16x2, 2.5 instructions per pair).
-template <int NW, int NS, int CT, int CV>
+// INT8: the code format. E4M3 codes become f16 through the conversion
+// instruction; INT8 codes on the integer and FMA pipes (int8x4_to_f16x2,
+// 2.5 instructions per pair).
+template <int NW, int NS, int CT, bool INT8>
 __global__ void __launch_bounds__(NW * 32)
     decode_split_q8(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -211,8 +180,8 @@ __global__ void __launch_bounds__(NW * 32)
         for (int i = 0; i < NS && i < my_n; ++i) issue(i);
     }
 
-    const float sl2 = a.scale_log2 * __ldg(a.k_scale + kvh) * (CV == 1 || CV == 2 ? 256.f : 1.f);
-    const float vsc = __ldg(a.v_scale + kvh) * (CV == 2 ? 256.f : 1.f);
+    const float sl2 = a.scale_log2 * __ldg(a.k_scale + kvh);
+    const float vsc = __ldg(a.v_scale + kvh);
 
     // Q fragments in f16, dims permuted to match the K fragments: slot
     // 2c+j (j = 0,1) of k-step ks holds dim 16ks+4c+j, slot 2c+8+j holds
@@ -232,7 +201,7 @@ __global__ void __launch_bounds__(NW * 32)
                 uint2 v = make_uint2(0u, 0u);
                 if (qr < nh)
                     v = __ldg(reinterpret_cast<const uint2 *>(qb + qr * D + ks * 16 + 4 * tig));
-                if (CV >= 1) {
+                if (INT8) {
                     qa[ks][hr] = pack_f16x2(bf16_lo(v.x), bf16_lo(v.y));      // dims +0, +2
                     qa[ks][hr + 2] = pack_f16x2(bf16_hi(v.x), bf16_hi(v.y));  // dims +1, +3
                 } else {
@@ -301,12 +270,12 @@ __global__ void __launch_bounds__(NW * 32)
                         const int u = kp * 2 + (mi >> 1);
                         uint32_t r0, r1, r2, r3;
                         ldsm_x4(kb + p * kChunk * D + sw128(r, u), r0, r1, r2, r3);
-                        if constexpr (CV >= 1) {
+                        if constexpr (INT8) {
                             uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
-                            codes_to_f16x2<CV>(r0, e0, o0);
-                            codes_to_f16x2<CV>(r1, e1, o1);
-                            codes_to_f16x2<CV>(r2, e2, o2);
-                            codes_to_f16x2<CV>(r3, e3, o3);
+                            int8x4_to_f16x2(r0, e0, o0);
+                            int8x4_to_f16x2(r1, e1, o1);
+                            int8x4_to_f16x2(r2, e2, o2);
+                            int8x4_to_f16x2(r3, e3, o3);
                             mma_f16_16816(sc[2 * p], qa[2 * kp], e0, o0);
                             mma_f16_16816(sc[2 * p + 1], qa[2 * kp], e1, o1);
                             mma_f16_16816(sc[2 * p], qa[2 * kp + 1], e2, o2);
@@ -410,13 +379,13 @@ __global__ void __launch_bounds__(NW * 32)
                         uint32_t r0, r1, r2, r3;
                         ldsm_x4_t(vb + p * kChunk * D + sw128(r, u), r0, r1, r2, r3);
                         const int u0 = up * 2, u1 = up * 2 + 1;
-                        if constexpr (CV >= 2) {
+                        if constexpr (INT8) {
                             // even codes of a word: dim 2g, odd codes: dim 2g+1
                             uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
-                            codes_to_f16x2<CV>(r0, e0, o0);
-                            codes_to_f16x2<CV>(r1, e1, o1);
-                            codes_to_f16x2<CV>(r2, e2, o2);
-                            codes_to_f16x2<CV>(r3, e3, o3);
+                            int8x4_to_f16x2(r0, e0, o0);
+                            int8x4_to_f16x2(r1, e1, o1);
+                            int8x4_to_f16x2(r2, e2, o2);
+                            int8x4_to_f16x2(r3, e3, o3);
                             mma_f16_16816(o[2 * u0], pa[p], e0, e1);
                             mma_f16_16816(o[2 * u0 + 1], pa[p], o0, o1);
                             mma_f16_16816(o[2 * u1], pa[p], e2, e3);

@@ -101,45 +101,12 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 // ------------------------------------------------------------- decode
-// Launch shape of the split kernel: warps per CTA and pipeline stages per
-// warp. PA_DECODE_PIPE=<warps>x<stages> selects another built shape.
-struct Pipe {
-    int nw, ns;
-};
-
-Pipe decode_pipe() {
-    static Pipe p = [] {
-        Pipe r{4, 2};
-        if (const char *e = std::getenv("PA_DECODE_PIPE")) {
-            int w = 0, s = 0;
-            if (sscanf(e, "%dx%d", &w, &s) == 2) r = Pipe{w, s};
-        }
-        return r;
-    }();
-    return p;
-}
-
-// Launch shape of the FP8 split kernel: warps x stages x tokens per stage x
-// code conversion (decode_split_q8's CV);
-// PA_DECODE_PIPE_FP8=<warps>x<stages>x<tokens>x<cv> (built: 4x2x32x0,
-// 4x2x32x2, 4x2x16x0, 4x3x32x0; default 4x2x32x0: on B200 the conversion
-// instruction beat the integer-pipe form, 0.62 vs 0.55 of the HBM peak on
-// the Llama-7B batch).
-struct PipeFp8 {
-    int nw, ns, ct, cv;
-};
-
-PipeFp8 decode_pipe_fp8() {
-    static PipeFp8 p = [] {
-        PipeFp8 r{4, 2, 32, 0};
-        if (const char *e = std::getenv("PA_DECODE_PIPE_FP8")) {
-            int w = 0, s = 0, c = 0, v = 0;
-            if (sscanf(e, "%dx%dx%dx%d", &w, &s, &c, &v) == 4) r = PipeFp8{w, s, c, v};
-        }
-        return r;
-    }();
-    return p;
-}
+// Launch shapes (measured on B200 in sweeps of warps x stages): the bf16
+// and fp32 split kernels run 4 warps with 2-deep per-warp TMA rings; the
+// 8-bit kernel 4 warps x 2 stages of 32 tokens.
+constexpr int kDecodeWarps = 4;
+constexpr int kDecodeStages = 2;
+constexpr int kQ8Tokens = 32;
 
 template <int D, int NW, int NS>
 pa_status launch_decode_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
@@ -164,35 +131,11 @@ pa_status launch_decode_f32(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
     return launch_status();
 }
 
-template <int D>
-pa_status dispatch_bf16(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
-                        dim3 grid, cudaStream_t st) {
-    const Pipe p = decode_pipe();
-    if (p.nw == 2 && p.ns == 2) return launch_decode_bf16<D, 2, 2>(a, mk, mv, grid, st);
-    if (p.nw == 2 && p.ns == 3) return launch_decode_bf16<D, 2, 3>(a, mk, mv, grid, st);
-    if (p.nw == 2 && p.ns == 4) return launch_decode_bf16<D, 2, 4>(a, mk, mv, grid, st);
-    if (p.nw == 4 && p.ns == 1) return launch_decode_bf16<D, 4, 1>(a, mk, mv, grid, st);
-    if (p.nw == 4 && p.ns == 3) return launch_decode_bf16<D, 4, 3>(a, mk, mv, grid, st);
-    return launch_decode_bf16<D, 4, 2>(a, mk, mv, grid, st);
-}
-
-// PA_PREFILL_POLY=4 computes every 4th pair of softmax exponentials in full
-// prefill tiles on the FMA pipe instead of the special-function unit. Off by
-// default: on B200 the softmax is limited by instruction issue, not by the
-// special-function unit, and the extra instructions cost more than they save.
-int prefill_poly() {
-    static int v = [] {
-        const char *e = std::getenv("PA_PREFILL_POLY");
-        return (e && std::atoi(e) == 4) ? 4 : 0;
-    }();
-    return v;
-}
-
-template <int D, int POLY, bool WIN>
+template <int D, bool WIN>
 pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                             const CUtensorMap &mv, dim3 grid, cudaStream_t st) {
     const size_t smem = 1024 + pf_smem_bytes(D);
-    auto k = prefill_tc_kernel<D, POLY, WIN>;
+    auto k = prefill_tc_kernel<D, WIN>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
     // the kernel's register split must fit the registers it launches with,
     // or the warpgroups that grow would wait forever
@@ -217,13 +160,13 @@ bool encode_cache_map_u8(CUtensorMap *m, const void *cache, int NB, int H_kv, in
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NW, int NS, int CT, int CV>
+template <int NW, int NS, int CT, bool INT8>
 pa_status launch_decode_q8(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
                              dim3 grid, cudaStream_t st) {
     constexpr int STAGE = 2 * CT * 128;
     using L = DecodeSmem<NW, NS, STAGE, kHeadsBf16, 128>;
     const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
-    auto k = decode_split_q8<NW, NS, CT, CV>;
+    auto k = decode_split_q8<NW, NS, CT, INT8>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
     k<<<grid, NW * 32, smem, st>>>(a, mk, mv);
     return launch_status();
@@ -396,16 +339,17 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
                               kChunk) ||
             !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, block_size, head_dim, kChunk))
             return PA_ERR_CUDA;
-        st = head_dim == 128 ? dispatch_bf16<128>(a, mk, mv, grid, stream)
-                             : dispatch_bf16<64>(a, mk, mv, grid, stream);
+        st = head_dim == 128
+                 ? launch_decode_bf16<128, kDecodeWarps, kDecodeStages>(a, mk, mv, grid, stream)
+                 : launch_decode_bf16<64, kDecodeWarps, kDecodeStages>(a, mk, mv, grid, stream);
         if (st != PA_OK) return st;
         if (S1 > 1) {
             st = head_dim == 128 ? launch_reduce<128, __nv_bfloat16>(a, stream)
                                  : launch_reduce<64, __nv_bfloat16>(a, stream);
         }
     } else {
-        st = head_dim == 128 ? launch_decode_f32<128, 4, 2>(a, grid, stream)
-                             : launch_decode_f32<64, 4, 2>(a, grid, stream);
+        st = head_dim == 128 ? launch_decode_f32<128, kDecodeWarps, kDecodeStages>(a, grid, stream)
+                             : launch_decode_f32<64, kDecodeWarps, kDecodeStages>(a, grid, stream);
         if (st != PA_OK) return st;
         if (S1 > 1) {
             st = head_dim == 128 ? launch_reduce<128, float>(a, stream)
@@ -575,21 +519,11 @@ static pa_status decode_q8_impl(void *out, const void *q, const void *k_cache,
         !encode_cache_map_u8(&mv, v_cache, num_blocks, num_kv_heads, block_size))
         return PA_ERR_CUDA;
     const dim3 grid((unsigned)S1, (unsigned)gy, (unsigned)num_seqs);
-    const PipeFp8 pp = decode_pipe_fp8();
-    auto is = [&](int w, int n, int c, int v) {
-        return pp.nw == w && pp.ns == n && pp.ct == c && pp.cv == v;
-    };
-    pa_status st;
-    if (int8)
-        st = launch_decode_q8<4, 2, 32, 3>(a, mk, mv, grid, stream);
-    else
-        st = is(4, 2, 32, 2)   ? launch_decode_q8<4, 2, 32, 2>(a, mk, mv, grid, stream)
-             : is(4, 2, 16, 0) ? launch_decode_q8<4, 2, 16, 0>(a, mk, mv, grid, stream)
-             : is(4, 3, 32, 0) ? launch_decode_q8<4, 3, 32, 0>(a, mk, mv, grid, stream)
-                               : launch_decode_q8<4, 2, 32, 0>(a, mk, mv, grid, stream);
+    const pa_status st =
+        int8 ? launch_decode_q8<kDecodeWarps, kDecodeStages, kQ8Tokens, true>(a, mk, mv, grid, stream)
+             : launch_decode_q8<kDecodeWarps, kDecodeStages, kQ8Tokens, false>(a, mk, mv, grid, stream);
     if (st != PA_OK) return st;
-    if (S1 > 1) st = launch_reduce<128, __nv_bfloat16>(a, stream);
-    return st;
+    return S1 > 1 ? launch_reduce<128, __nv_bfloat16>(a, stream) : PA_OK;
 }
 
 pa_status pa_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -681,11 +615,10 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     a.timeout_ns = kWaitTimeoutNs;
     const dim3 grid((unsigned)num_q_heads, (unsigned)qtiles, (unsigned)num_chunks);
     if (head_dim == 64)
-        return window > 0 ? launch_prefill_tc<64, 0, true>(a, mq, mk, mv, grid, stream)
-                          : launch_prefill_tc<64, 0, false>(a, mq, mk, mv, grid, stream);
-    if (window > 0) return launch_prefill_tc<128, 0, true>(a, mq, mk, mv, grid, stream);
-    if (prefill_poly() == 4) return launch_prefill_tc<128, 4, false>(a, mq, mk, mv, grid, stream);
-    return launch_prefill_tc<128, 0, false>(a, mq, mk, mv, grid, stream);
+        return window > 0 ? launch_prefill_tc<64, true>(a, mq, mk, mv, grid, stream)
+                          : launch_prefill_tc<64, false>(a, mq, mk, mv, grid, stream);
+    return window > 0 ? launch_prefill_tc<128, true>(a, mq, mk, mv, grid, stream)
+                      : launch_prefill_tc<128, false>(a, mq, mk, mv, grid, stream);
 }
 
 pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -861,8 +794,10 @@ pa_status pa_selftest_bounded_wait(long long timeout_ns, cudaStream_t stream) {
 // Its scratch is a file-scope device array compiled into the library, so
 // every GPU that loads the library holds these 16 MiB until the process
 // exits. In host code the array's name is only a host-side stand-in; the
-// device address is looked up with cudaGetSymbolAddress the first time the
-// entry point runs on a device (with that device current) and cached.
+// device address is looked up with cudaGetSymbolAddress, with the device
+// current, the first time the entry point runs in a CUDA context, and cached
+// under that context's unique id: after cudaDeviceReset the next call runs in
+// a new context and looks the address up again.
 namespace {
 
 constexpr size_t kStaticWorkspaceBytes = size_t(16) << 20;  // 16 MiB per device
@@ -872,17 +807,51 @@ __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes
 constexpr int kMaxDevices = 64;
 std::mutex g_static_ws_mutex;
 void *g_static_ws_ptr[kMaxDevices] = {};
+unsigned long long g_static_ws_ctx[kMaxDevices] = {};  // context id of each cached address
+
+// Unique id (cuCtxGetId, never reused within the process) of the calling
+// thread's current context, 0 when there is none or the lookup fails. The
+// driver entry points are fetched through the runtime so that the library
+// does not link libcuda directly.
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr, *q = nullptr;
+        cudaDriverEntryPointQueryResult r1, r2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r1) ==
+                cudaSuccess &&
+            r1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &q, cudaEnableDefault, &r2) == cudaSuccess &&
+            r2 == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+            get_id = reinterpret_cast<GetIdFn>(q);
+        }
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 // Device address of g_static_workspace on the current device, looked up once
-// per device; nullptr if the lookup fails.
+// per CUDA context; nullptr if the lookup fails.
 void *static_workspace_address() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-    if (!g_static_ws_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_static_ws_ptr[dev] || ctx == 0 || ctx != g_static_ws_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) return nullptr;
         g_static_ws_ptr[dev] = p;
+        // the lookup makes the device's primary context current if no
+        // context was: key the address on the context it was found in
+        g_static_ws_ctx[dev] = current_context_id();
     }
     return g_static_ws_ptr[dev];
 }

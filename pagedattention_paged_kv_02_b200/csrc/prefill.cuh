@@ -221,29 +221,11 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, to take part of the softmax's exponentials off the
-// special-function unit. Cody-Waite style range reduction: x = n + f with
-// n = round(x) (adding 1.5*2^23 leaves n in the low mantissa bits) and
-// |f| <= 1/2; 2^f by a cubic 1 + c1 f + c2 f^2 + c3 f^3 whose coefficients
-// were fitted for minimum maximum relative error on [-1/2, 1/2] (1.02e-4,
-// about 2^-13, exact at f = 0: below the bf16 rounding of P); 2^n is added
-// to the exponent field. Inputs below -125 give 2^-125.
-__device__ __forceinline__ float ex2_poly(float x) {
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;
-    const float n = t - 12582912.f;
-    const float f = x - n;
-    const float p = fmaf(fmaf(fmaf(0.05500824f, f, 0.24220951f), f, 0.69328284f), f, 1.f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// POLY: every POLY-th pair of exponentials in a full (unmasked) tile is
-// computed with ex2_poly instead of the special-function unit (0 = none).
 // WIN: the sliding-window build; without it the band logic folds away at
 // compile time and the causal kernel keeps its tighter code.
 // D: head_dim, 64 or 128 (one or two 64-wide halves per row; the S tiles
 // and the P.V accumulators keep their TMEM columns, O using the first D).
-template <int D, int POLY, bool WIN>
+template <int D, bool WIN>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
@@ -269,13 +251,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int c = a.n_chunks - 1 - (int)blockIdx.z;
     const int q0 = a.qsl[c];
     const int C = a.qsl[c + 1] - q0;
-    const int row0 = tp * kPfRows * kPfQTiles;  // first query of this CTA within the chunk
-    if (row0 >= C) return;
     const int ctx = a.context_lens[c];
+    // the chunk is checked before any CTA leaves for lack of rows, so that a
+    // malformed chunk is recorded even when it has no rows at all
     if (q0 < 0 || C < 0 || q0 + C > a.total_q || ctx < C || (long long)ctx > (long long)a.MB * a.bs) {
         if (threadIdx.x == 0) flag_error(PA_ERR_BAD_TABLE);
         return;
     }
+    // rows past the grid's reach (a chunk longer than max_query_len rounded
+    // up to the CTA's rows) would be left unwritten: recorded once per chunk
+    if (C > (int)gridDim.y * kPfRows * kPfQTiles && blockIdx.x == 0 && blockIdx.y == 0 &&
+        threadIdx.x == 0)
+        flag_error(PA_ERR_BAD_TABLE);
+    const int row0 = tp * kPfRows * kPfQTiles;  // first query of this CTA within the chunk
+    if (row0 >= C) return;
     const int cached = ctx - C;
     // Rows of each Q tile (a Q tile past the chunk has none) and the K/V
     // tiles [jlo_x, jhi_x) it needs: up to its last row's position, from its
@@ -585,14 +574,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const float2 t = __ffma2_rn(
                         make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2v,
                         nmv);
-                    float p0, p1;
-                    if (POLY > 0 && e % (POLY > 0 ? POLY : 1) == POLY - 1) {
-                        p0 = ex2_poly(t.x);
-                        p1 = ex2_poly(t.y);
-                    } else {
-                        p0 = ex2_approx(t.x);
-                        p1 = ex2_approx(t.y);
-                    }
+                    const float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
                     acc2[e & 1] = __fadd2_rn(acc2[e & 1], make_float2(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
                 }

@@ -179,6 +179,8 @@ def pa_decode_sliding_window(out, q, k_cache, v_cache, block_tables, context_len
     NB, H_kv, bs, D2 = k_cache.shape
     if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
         raise ValueError("out must match q; caches must share head_dim")
+    if not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("q and caches must share one dtype")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _call("pa_decode_sliding_window", _p(out), _p(q), _p(k_cache), _p(v_cache),
           _p(block_tables), _p(context_lens), B, H_q, H_kv, D, bs, NB, block_tables.shape[1],
@@ -413,6 +415,8 @@ def prepare_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_con
     NB, H_kv, bs, D2 = k_cache.shape
     if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
         raise ValueError("out must match q; caches must share head_dim")
+    if not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("q and caches must share one dtype")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     head = (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens), B,
             H_q, H_kv, D, bs, NB, block_tables.shape[1], int(max_context_len), float(scale))

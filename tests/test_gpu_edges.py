@@ -84,3 +84,41 @@ def test_prefill_edge_chunks(pa, cached, lens):
     if ref.numel():
         assert_close(out, ref, f"prefill edge {cached} {lens}")
     assert pa.pa_device_error() == 0
+
+
+def test_prefill_chunk_longer_than_max_query_len(pa):
+    """A chunk of 300 queries launched with max_query_len 200: the grid covers
+    256 rows of it (200 rounded up to the CTA's 256). Rows 0..255 are
+    computed as usual, rows 256..299 are left as they were (NaN poison) and
+    the chunk is recorded as PA_ERR_BAD_TABLE."""
+    batch = mixed_chunks([40], [300], 8, 2, 16, seed=104)
+    d = batch.to(DEV)
+    pa.pa_reshape_and_cache(d.key, d.value, d.k_cache, d.v_cache, d.slot_mapping)
+    out = torch.full_like(d.prefill_q, float("nan"))
+    pa.pa_prefill_chunk(out, d.prefill_q, d.k_cache, d.v_cache, d.prefill_block_tables,
+                        d.prefill_context_lens, d.query_start_loc, 200, batch.scale)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == pa.PA_ERR_BAD_TABLE
+    got = out.cpu()
+    assert torch.isnan(got[256:].float()).all(), "rows past the launch were written"
+    k, v = oracle_after_append(batch)
+    ref, _ = oracle_prefill(batch, k, v)
+    assert_close(got[:256], ref[:256], "covered rows of the over-long chunk")
+
+
+def test_prefill_decreasing_query_start_loc_is_recorded(pa):
+    """query_start_loc going backwards (C < 0) is a malformed chunk: skipped
+    and recorded, whatever its row count; the well-formed chunk beside it is
+    still computed."""
+    batch = mixed_chunks([10, 20], [64, 64], 8, 2, 16, seed=105)
+    d = batch.to(DEV)
+    pa.pa_reshape_and_cache(d.key, d.value, d.k_cache, d.v_cache, d.slot_mapping)
+    qsl = torch.tensor([0, 64, 32], dtype=torch.int32, device=DEV)  # chunk 1: C = -32
+    out = torch.full_like(d.prefill_q, float("nan"))
+    pa.pa_prefill_chunk(out, d.prefill_q, d.k_cache, d.v_cache, d.prefill_block_tables,
+                        d.prefill_context_lens, qsl, 64, batch.scale)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == pa.PA_ERR_BAD_TABLE
+    k, v = oracle_after_append(batch)
+    ref, _ = oracle_prefill(batch, k, v)
+    assert_close(out.cpu()[:64], ref[:64], "well-formed chunk beside a malformed one")

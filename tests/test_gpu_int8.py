@@ -96,7 +96,8 @@ def test_int8_workload_full(pa, name):
     b = W.WORKLOADS[name]()
     d, out = gpu_step_int8(pa, b)
     k, v = oracle_after_append_int8(b)
-    assert torch.equal(d.k_cache.cpu(), k), "quantising append not bit-exact"
+    assert torch.equal(d.k_cache.cpu(), k), "quantising append not bit-exact (K)"
+    assert torch.equal(d.v_cache.cpu(), v), "quantising append not bit-exact (V)"
     ref, _ = oracle.decode_int8(b.q, k, v, b.k_scale, b.v_scale, b.block_tables, b.context_lens,
                                 b.scale)
     assert_close(out, ref, name)
