@@ -291,13 +291,15 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
-def make_batch(name: str, seed: int, num_blocks=None, block_size=None):
+def make_batch(name: str, seed: int, num_blocks=None, block_size=None, head_dim=None):
     from pagedattention_paged_kv_02_b200 import workloads as W
     kw = {}
     if num_blocks:
         kw["num_blocks"] = num_blocks
     if block_size:
         kw["block_size"] = block_size
+    if head_dim:
+        kw["head_dim"] = head_dim
     return W.WORKLOADS[name](seed=seed, **kw)
 
 
@@ -315,9 +317,17 @@ class Runner:
         self.max_ctx = batch.max_context_len  # host-side bound, computed once
         self.ws = None
         self.S = 0
+        # sequences sharing prefix blocks go through the prefix-aware decode
+        self.shared = (d.decode_group_start is not None and not batch.quantized and
+                       batch.sliding_window == 0 and batch.dtype == torch.bfloat16)
         if d.q is not None and d.num_seqs:
             B, H_q, D = d.q.shape
-            n = pa.pa_decode_workspace_size(B, H_q, D, d.max_context_len, self.part)
+            if self.shared:
+                n = pa.pa_decode_shared_prefix_workspace_size(
+                    B, H_q, d.num_kv_heads, D, d.decode_prefix_lens.numel(),
+                    batch.max_group_size, batch.max_prefix_len, d.max_context_len, self.part)
+            else:
+                n = pa.pa_decode_workspace_size(B, H_q, D, d.max_context_len, self.part)
             self.ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
             P = pa.pa_decode_partition_tokens(d.max_context_len, self.part)
             self.S = -(-d.max_context_len // P)
@@ -330,7 +340,9 @@ class Runner:
 
     def launches_per_step(self) -> int:
         n = 1  # reshape_and_cache
-        if self.d.q is not None and self.d.num_seqs:
+        if self.d.q is not None and self.d.num_seqs and self.shared:
+            n += 3 if self.host.max_prefix_len > 0 else 2  # prefix, tails, merge
+        elif self.d.q is not None and self.d.num_seqs:
             n += 1 + (1 if self.S > 1 else 0)
         if self.d.prefill_q is not None:
             n += 1
@@ -357,6 +369,12 @@ class Runner:
                                                 d.k_cache, d.v_cache, d.k_scale, d.v_scale,
                                                 d.block_tables, d.context_lens, self.max_ctx,
                                                 d.scale, self.part, self.ws)
+        elif d.q is not None and d.num_seqs and self.shared:
+            c["decode"] = pa.prepare_decode_shared_prefix(
+                out if out is not None else self.out, d.q, d.k_cache, d.v_cache, d.block_tables,
+                d.context_lens, d.decode_group_start, d.decode_prefix_lens,
+                self.host.max_group_size, self.host.max_prefix_len, self.max_ctx, d.scale,
+                self.part, self.ws)
         elif d.q is not None and d.num_seqs:
             c["decode"] = pa.prepare_decode(out if out is not None else self.out, d.q, d.k_cache,
                                             d.v_cache, d.block_tables, d.context_lens,
@@ -364,22 +382,17 @@ class Runner:
                                             self.host.sliding_window)
         return c
 
-    def step(self, ev=None, calls=None, stream=None, rev=None):
-        """One pass; ``ev`` (start, end) events bracket the dominant call,
-        ``rev`` the cache scatter."""
+    def step(self, ev=None, calls=None, stream=None):
+        """One pass; ``ev`` maps a call's name ("reshape", "prefill",
+        "decode") to (start, end) events recorded around it."""
         c = calls or self._calls
-        if rev is not None:
-            rev[0].record()
-        c["reshape"](stream)
-        if rev is not None:
-            rev[1].record()
-        for name in ("prefill", "decode"):
+        for name in ("reshape", "prefill", "decode"):
             if name in c:
-                if ev is not None and name == self.dominant:
-                    ev[0].record()
+                if ev is not None and name in ev:
+                    ev[name][0].record()
                 c[name](stream)
-                if ev is not None and name == self.dominant:
-                    ev[1].record()
+                if ev is not None and name in ev:
+                    ev[name][1].record()
 
     @property
     def dominant(self):
@@ -392,7 +405,7 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     dist = init_dist(world, "nccl")
     batch = make_batch(args.workload, seed=rank, num_blocks=args.num_blocks,
-                       block_size=args.block_size)
+                       block_size=args.block_size, head_dim=args.head_dim)
     if args.partition is not None:
         batch.partition_size = args.partition
     batch.sliding_window = args.window
@@ -438,19 +451,29 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     # the same K steps again, events around the dominant call of each, for
     # its roofline
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
-    revs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(K)]
+    pair = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    evs = [{n: pair() for n in r._calls} for _ in range(K)]
     for i in range(K):
-        r.step(evs[i], rev=revs[i])
+        r.step(evs[i])
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier(world)
     ms_local = t0.elapsed_time(t1) / K
-    dom_all = sorted(a.elapsed_time(b) for a, b in evs)
+    call_ms = lambda n: [e[n][0].elapsed_time(e[n][1]) for e in evs]
+    dom_all = sorted(call_ms(r.dominant))
     dom_ms = statistics.fmean(dom_all)
-    rs_ms = statistics.fmean(a.elapsed_time(b) for a, b in revs)
+    dec_ms = statistics.fmean(call_ms("decode")) if "decode" in r._calls else None
+    # the scatter is a few microseconds: events around one launch measure
+    # mostly the launch itself, so its duration is taken over a burst of
+    # back-to-back launches (re-appending the same rows is idempotent)
+    burst = 50
+    b0, b1 = pair()
+    b0.record()
+    for _ in range(burst):
+        r._calls["reshape"]()
+    b1.record()
+    torch.cuda.synchronize()
+    rs_ms = b0.elapsed_time(b1) / burst
     pct = lambda q: dom_all[min(len(dom_all) - 1, int(q * len(dom_all)))]
 
     units = dbytes if r.dominant == "decode" else pflops
@@ -466,6 +489,8 @@ def run_ours(args, rank, world):
     names = ["key", "value", "slot_mapping"]
     if batch.q is not None:
         names += ["q", "block_tables", "context_lens"]
+        if r.shared:
+            names += ["decode_group_start", "decode_prefix_lens"]
     if batch.prefill_q is not None:
         names += ["prefill_q", "prefill_block_tables", "prefill_context_lens", "query_start_loc"]
     # the step's inputs packed into one pinned buffer (one upload per step)
@@ -498,41 +523,75 @@ def run_ours(args, rank, world):
         out_hs.append(torch.empty(out_shape, dtype=out_dtype, pin_memory=True))
         bcalls.append(r.calls(d=dd, out=outs[-1], pout=pouts[-1]))
     d2h = out_hs[0].numel() * out_hs[0].element_size()
-    comp = torch.cuda.current_stream()
     up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()  # uploads never queue behind downloads
     up_done = [torch.cuda.Event() for _ in range(2)]
     used = [torch.cuda.Event() for _ in range(2)]
     down_done = [torch.cuda.Event() for _ in range(2)]
-    for e in used + down_done:
-        e.record(comp)
 
-    def e2e_step(i):
-        k = i % 2
-        up_s.wait_event(used[k])          # buffer k's previous step is done with it
-        with torch.cuda.stream(up_s):
-            d_flats[k].copy_(h_flat, non_blocking=True)
-        up_done[k].record(up_s)
-        comp.wait_event(up_done[k])
-        comp.wait_event(down_done[k])     # its previous result has been read back
-        r.step(calls=bcalls[k])
-        used[k].record(comp)
-        down_s.wait_event(used[k])
-        with torch.cuda.stream(down_s):
-            out_hs[k].copy_(outs[k] if outs[k] is not None else pouts[k], non_blocking=True)
-        down_done[k].record(down_s)
+    def e2e_steps(n, comp):
+        """n steps on stream comp, alternating the two staging buffers: step
+        i's upload waits for step i-2's compute (same buffer), its compute for
+        its upload and for step i-2's download. The first two steps of a run
+        fork from comp's position."""
+        up_s.wait_stream(comp)
+        down_s.wait_stream(comp)
+        for i in range(n):
+            k = i % 2
+            if i >= 2:
+                up_s.wait_event(used[k])      # buffer k's previous step is done with it
+            with torch.cuda.stream(up_s):
+                d_flats[k].copy_(h_flat, non_blocking=True)
+            up_done[k].record(up_s)
+            comp.wait_event(up_done[k])
+            if i >= 2:
+                comp.wait_event(down_done[k])  # its previous result has been read back
+            r.step(calls=bcalls[k], stream=comp)
+            used[k].record(comp)
+            down_s.wait_event(used[k])
+            with torch.cuda.stream(down_s):
+                out_hs[k].copy_(outs[k] if outs[k] is not None else pouts[k], non_blocking=True)
+            down_done[k].record(down_s)
+        comp.wait_stream(up_s)
+        comp.wait_stream(down_s)
 
-    for i in range(max(3, args.warmup // 4)):
-        e2e_step(i)
+    # the steps, uploads and downloads included, captured as CUDA graphs of
+    # up to 8 steps (the host issue cost of a step's dozen stream operations
+    # would otherwise exceed a short step's device time); replays of one
+    # graph serialise on the stream, so consecutive graphs do not overlap
+    comp = torch.cuda.current_stream()
+    e2e_graphs = {}
+    if args.graph:
+        side = torch.cuda.Stream()
+        for n in sorted({min(8, K), K % min(8, K)} - {0}):
+            g = torch.cuda.CUDAGraph()
+            side.wait_stream(comp)
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(g, stream=side):
+                    e2e_steps(n, side)
+            comp.wait_stream(side)
+            e2e_graphs[n] = g
+        torch.cuda.synchronize()
+
+    def e2e_run(n_steps):
+        if not e2e_graphs:
+            e2e_steps(n_steps, comp)
+            return
+        g_len = max(e2e_graphs)
+        for _ in range(n_steps // g_len):
+            e2e_graphs[g_len].replay()
+        if n_steps % g_len:
+            e2e_graphs[n_steps % g_len].replay()
+
+    if e2e_graphs:  # warm-up: every captured graph once
+        for g in e2e_graphs.values():
+            g.replay()
+    else:
+        e2e_run(max(3, args.warmup // 4))
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(comp)
-    up_s.wait_event(e0)
-    down_s.wait_event(e0)
-    for i in range(K):
-        e2e_step(i)
-    comp.wait_stream(up_s)
-    comp.wait_stream(down_s)
+    e2e_run(K)
     e1.record(comp)
     torch.cuda.synchronize()
     barrier(world)
@@ -598,8 +657,19 @@ def run_ours(args, rank, world):
             line["prefill_tflops"] = round(pflops * world / (ms * 1e-3) / 1e12, 1)
             # the decode part of the mixed step reads shared prefix blocks
             # through many tables: logical bytes (value) and distinct bytes
-            line["decode_bytes_per_step"] = {"logical": dbytes,
-                                             "unique_kv": decode_unique_bytes(batch)}
+            ubytes = decode_unique_bytes(batch)
+            line["decode_bytes_per_step"] = {"logical": dbytes, "unique_kv": ubytes}
+            if dec_ms:
+                # its roofline on the bytes HBM must deliver at least once
+                line["roofline_decode"] = {
+                    "bound": "hbm", "achieved": round(ubytes / (dec_ms * 1e-3) / 1e9, 1),
+                    "peak": hbm, "unit": "GB/s",
+                    "frac": round(ubytes / (dec_ms * 1e-3) / 1e9 / hbm, 4),
+                    "peak_basis": f"{basis} hbm_gbs", "basis": "distinct K/V bytes",
+                    "kernel": ("pa_decode_shared_prefix (prefix + tails + merge)" if r.shared
+                               else "pa_decode (decode_split + merge)"),
+                    "ms": round(dec_ms, 5), "logical_bytes_GBps": round(
+                        dbytes / (dec_ms * 1e-3) / 1e9, 1)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(batch, args.cpu_seconds)
     if world > 1:
@@ -828,6 +898,9 @@ def main(argv=None):
                     help="decode KV partition tokens (0 automatic, <0 no split)")
     ap.add_argument("--block-size", type=int, default=None, choices=[16, 32, 64],
                     help="block size override for the decode workloads (pool bytes kept)")
+    ap.add_argument("--head-dim", type=int, default=None, choices=[64, 128],
+                    help="head_dim override for llama7b_decode, gqa_decode and "
+                         "mixed_prefill_decode")
     ap.add_argument("--num-blocks", type=int, default=None,
                     help="physical pool size override (a smaller pool for profiler captures)")
     ap.add_argument("--window", type=int, default=0,
@@ -841,6 +914,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.head_dim and args.workload not in ("llama7b_decode", "gqa_decode",
+                                               "mixed_prefill_decode"):
+        ap.error("--head-dim applies to llama7b_decode, gqa_decode and mixed_prefill_decode")
     if args.window < 0 or (args.window and args.workload.endswith(("_fp8", "_int8"))):
         ap.error("--window takes W > 0 and a bf16/fp32 workload")
     rank, local, world = rank_env()

@@ -137,6 +137,57 @@ PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const 
                     int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
                     cudaStream_t stream);
 
+/* Paged decode for batches whose sequences share prefix blocks, reading
+ * each shared block once for all its readers: page "字节跳动 AI Infra (2)",
+ * question "vLLM与PagedAttention的原理" (beams of one request share prefix
+ * blocks, B1 and B3 in its example; a partially filled shared block is
+ * copied on write, B6'), with the split of each sequence's attention into a
+ * prefix part and a private part merged by log-sum-exp (same page,
+ * algorithm-level table, FlashDecoding row). The result is pa_decode's:
+ *   out[b][h] = sum_{j < context_lens[b]} softmax_j(scale * q[b][h] . K_j) V_j.
+ *   group_start   int32 [num_groups + 1], device: sequences are listed group
+ *                 by group; group g is [group_start[g], group_start[g+1]).
+ *                 The groups partition [0, num_seqs) (group_start[0] = 0,
+ *                 group_start[num_groups] = num_seqs, non-decreasing); a
+ *                 sequence that shares nothing is a group of one.
+ *   prefix_lens   int32 [num_groups], device: group g's sequences hold the
+ *                 same K/V at positions [0, prefix_lens[g]) -- shared
+ *                 physical blocks, or copies of them. Those positions are
+ *                 read once per KV head through the table of the group's
+ *                 first sequence, for all of its sequences. The length used
+ *                 is min(prefix_lens[g], every member's context_len), and it
+ *                 need not be a multiple of block_size.
+ *   max_group_size, max_prefix_len   host-side bounds of the group sizes and
+ *                 prefix lengths. A malformed group, a group larger than
+ *                 max_group_size or a prefix longer than max_prefix_len is
+ *                 recorded as PA_ERR_BAD_TABLE (the outputs of that group's
+ *                 sequences are then unspecified).
+ *   partition_size   KV tokens per split of both the prefix and the tails
+ *                 (multiple of 16, <= 16384); 0 = automatic; < 0 = one
+ *                 partition each.
+ *   workspace     >= pa_decode_shared_prefix_workspace_size(...) bytes,
+ *                 256-byte aligned, always needed (the two passes always
+ *                 leave partials).
+ * bf16 only (fp32 returns PA_ERR_UNSUPPORTED); other arguments, limits and
+ * errors as for pa_decode. Three launches on `stream`: the prefix pass, the
+ * private-tail pass (which may start while the prefix pass runs) and the
+ * log-sum-exp merge. */
+PA_API size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads,
+                                                     int num_kv_heads, int head_dim,
+                                                     int num_groups, int max_group_size,
+                                                     int max_prefix_len, int max_context_len,
+                                                     int partition_size);
+PA_API pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
+                                         const void *v_cache, const int32_t *block_tables,
+                                         const int32_t *context_lens, const int32_t *group_start,
+                                         const int32_t *prefix_lens, int num_groups,
+                                         int max_group_size, int max_prefix_len, int num_seqs,
+                                         int num_q_heads, int num_kv_heads, int head_dim,
+                                         int block_size, int num_blocks, int max_blocks_per_seq,
+                                         int max_context_len, float scale, int partition_size,
+                                         void *workspace, size_t workspace_bytes,
+                                         pa_dtype dtype, cudaStream_t stream);
+
 /* FP8 KV cache (E4M3 codes, one byte per element, one dequantisation scale
  * per K/V head for K and one for V): page "字节跳动 AI Infra (2)", optimisation
  * table, KV quantisation row, and page "LLM推理优化", section 1.3 (store K/V
@@ -250,11 +301,11 @@ PA_API pa_status pa_decode_sliding_window(void *out, const void *q, const void *
  *                     max_blocks_per_seq*block_size is skipped and recorded
  *                     as PA_ERR_BAD_TABLE.
  *   max_query_len     host-side upper bound of every C_c. The launch covers
- *                     max_query_len rounded up to a multiple of 256 rows per
+ *                     max_query_len rounded up to a multiple of 128 rows per
  *                     chunk; the rows of a longer chunk past that are left
  *                     unwritten and the chunk is recorded as PA_ERR_BAD_TABLE.
  * bf16 with head_dim 64 or 128 (the tcgen05 tensor-core path), at most
- * 65535 chunks and max_query_len at most 65535 * 256; anything else returns
+ * 65535 chunks and max_query_len at most 65535 * 128; anything else returns
  * PA_ERR_UNSUPPORTED. */
 PA_API pa_status pa_prefill_chunk(void *out, const void *q, const void *k_cache, const void *v_cache,
                            const int32_t *block_tables, const int32_t *context_lens,

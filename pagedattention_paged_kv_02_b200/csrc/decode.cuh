@@ -51,6 +51,14 @@ struct DecodeArgs {
     int window;        // > 0: attend only the last `window` positions
     float scale_log2;  // scale * log2(e): scores are kept in the base-2 domain
     unsigned long long timeout_ns;
+    // shared-prefix decode (decode_prefix.cuh): sequences [group_start[g],
+    // group_start[g+1]) share their first prefix_lens[g] positions
+    const int32_t *group_start;
+    const int32_t *prefix_lens;
+    int num_groups, max_group, max_prefix;
+    int P_prefix;      // tokens per prefix partition
+    int S_prefix;      // partial slots [0, S_prefix) hold prefix partitions,
+                       // [S_prefix, S_max) the private tails' partitions
 };
 
 // First attended position of a sequence of ctx tokens (the sliding window's
@@ -75,11 +83,59 @@ __device__ __forceinline__ int clamped_ctx(const DecodeArgs &a, int b, bool repo
     return ctx;
 }
 
+// A shared-prefix group as the kernels use it: its first sequence, its
+// member count (capped at the host bound max_group) and its effective shared
+// length L = min(prefix_lens[g], every member's context), clamped to
+// [0, max_prefix]. Every warp computes it on its own (a lane per member, then
+// a warp minimum). False for a malformed group: bounds outside
+// [0, num_seqs], decreasing, or not starting at 0 / ending at num_seqs for
+// the first / last group (the groups must partition the batch).
+struct PrefixGroup {
+    int first, n, L;
+};
+
+__device__ __forceinline__ bool prefix_group(const DecodeArgs &a, int g, PrefixGroup &pg,
+                                             bool report) {
+    const int g0 = __ldg(a.group_start + g), g1 = __ldg(a.group_start + g + 1);
+    if (g0 < 0 || g1 < g0 || g1 > a.num_seqs || (g == 0 && g0 != 0) ||
+        (g == a.num_groups - 1 && g1 != a.num_seqs)) {
+        if (report) flag_error(PA_ERR_BAD_TABLE);
+        return false;
+    }
+    int L = __ldg(a.prefix_lens + g);
+    if (L < 0 || L > a.max_prefix || g1 - g0 > a.max_group) {
+        if (report) flag_error(PA_ERR_BAD_TABLE);
+        L = L < 0 ? 0 : min(L, a.max_prefix);
+    }
+    const int lane = threadIdx.x & 31;
+    for (int i = lane; i < g1 - g0; i += 32) L = min(L, clamped_ctx(a, g0 + i, false));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L = min(L, __shfl_xor_sync(0xffffffffu, L, o));
+    pg.first = g0;
+    pg.n = min(g1 - g0, a.max_group);
+    pg.L = L;
+    return true;
+}
+
+// lse = -inf for `nh` rows (query heads h0.. of sequence b) at partial slot
+// `slot`: a partition with nothing to attend, skipped by the merge.
+__device__ __forceinline__ void write_empty_slot(const DecodeArgs &a, int b, int h0, int nh,
+                                                 int slot) {
+    for (int r = threadIdx.x; r < nh; r += blockDim.x)
+        a.part_lse[((size_t)b * a.H_q + h0 + r) * a.S_max + slot] = -INFINITY;
+}
+
 // Programmatic dependent launch: a split CTA lets the merge kernel queued
 // behind it (decode_merge.cuh) be scheduled as soon as every split CTA has
 // started; its CTAs then fill the SMs the split grid's tail leaves idle.
 __device__ __forceinline__ void allow_dependent_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits for the grid this one depends on to complete, with its writes
+// visible (a no-op when launched without the dependency).
+__device__ __forceinline__ void wait_for_primary_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // Shared-memory plan of a split CTA: the stage ring (reused after the main
@@ -145,7 +201,12 @@ __device__ __forceinline__ void write_zero_rows(const DecodeArgs &a, int b, int 
 }
 
 // ------------------------------------------------------------------ bf16
-template <int D, int NW, int NS>
+// SHARED: the private-tail pass of the shared-prefix decode. The grid is
+// (member x tail partition, KV head [x head tile], group); sequence b of
+// group g attends positions [L, ctx_b) here (L = the group's shared length,
+// decode_prefix.cuh attends [0, L)) and always leaves partials, in slots
+// S_prefix + s, with lse = -inf for a partition that has nothing to attend.
+template <int D, int NW, int NS, bool SHARED = false>
 __global__ void __launch_bounds__(NW * 32)
     decode_split_bf16(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -164,20 +225,43 @@ __global__ void __launch_bounds__(NW * 32)
     int32_t *tbl = reinterpret_cast<int32_t *>(smem + L::kTable);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int s = blockIdx.x;
     const int kvh = blockIdx.y / a.n_htiles, ht = blockIdx.y - kvh * a.n_htiles;
-    const int b = blockIdx.z;
     const int h0 = kvh * a.group + ht * HT;
     const int nh = min(HT, a.group - ht * HT);
 
     allow_dependent_launch();
-    const int ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
-    const int lo = window_lo(a, ctx), base = span_base(a, ctx);
-    const int n_splits = (ctx - base + a.P - 1) / a.P;
-    if (s >= (n_splits > 0 ? n_splits : 1)) return;
-    if (ctx == 0) {
-        write_zero_rows<D, __nv_bfloat16>(a, b, h0, nh);
-        return;
+    int s, b, ctx, lo, base, n_splits;
+    if constexpr (SHARED) {
+        const int St = a.S_max - a.S_prefix;
+        const int member = blockIdx.x / St;
+        s = blockIdx.x - member * St;
+        PrefixGroup pg;
+        if (!prefix_group(a, blockIdx.z, pg, false) || member >= pg.n) {
+            wait_for_primary_grid();
+            return;
+        }
+        b = pg.first + member;
+        ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+        lo = pg.L;
+        base = lo & ~(kChunk - 1);
+        n_splits = ctx > lo ? (ctx - base + a.P - 1) / a.P : 0;
+        if (s >= n_splits) {
+            write_empty_slot(a, b, h0, nh, a.S_prefix + s);
+            wait_for_primary_grid();
+            return;
+        }
+    } else {
+        s = blockIdx.x;
+        b = blockIdx.z;
+        ctx = clamped_ctx(a, b, s == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+        lo = window_lo(a, ctx);
+        base = span_base(a, ctx);
+        n_splits = (ctx - base + a.P - 1) / a.P;
+        if (s >= (n_splits > 0 ? n_splits : 1)) return;
+        if (ctx == 0) {
+            write_zero_rows<D, __nv_bfloat16>(a, b, h0, nh);
+            return;
+        }
     }
     const int tok0 = base + s * a.P;
     const int tok1 = min(tok0 + a.P, ctx);
@@ -388,7 +472,15 @@ __global__ void __launch_bounds__(NW * 32)
             make_float2(o[dt][2], o[dt][3]);
     }
     __syncthreads();
-    decode_epilogue<D, NW, HT, __nv_bfloat16>(a, red_o, red_m, red_l, b, h0, nh, s, n_splits);
+    if constexpr (SHARED) {  // always a partial, after the prefix slots
+        decode_epilogue<D, NW, HT, __nv_bfloat16>(a, red_o, red_m, red_l, b, h0, nh,
+                                                  a.S_prefix + s, 2);
+        // the tail pass may start while the prefix pass runs (programmatic
+        // dependent launch); it completes only after the prefix pass has, so
+        // that the merge behind it sees both passes' partials
+        wait_for_primary_grid();
+    } else
+        decode_epilogue<D, NW, HT, __nv_bfloat16>(a, red_o, red_m, red_l, b, h0, nh, s, n_splits);
 }
 
 // ------------------------------------------------------------------ fp32

@@ -18,12 +18,6 @@
 
 namespace pa {
 
-// Waits for the grid this one depends on to complete, with its writes
-// visible (a no-op when launched without the dependency).
-__device__ __forceinline__ void wait_for_primary_grid() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
 // ------------------------------------------------------------- LSE merge
 // out = sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M), M = max_s lse_s, for
 // every (sequence, query head) with more than one partition.
@@ -32,18 +26,26 @@ __device__ __forceinline__ void wait_for_primary_grid() {
 // (sequence, head), eight per CTA, each lane owning D/32 dimensions and
 // walking the partitions in order; heads with one partition cost a warp a
 // length read.
+//
+// SHARED (the shared-prefix decode): every one of the S_max slots of every
+// (sequence, head) was written -- prefix partitions, then the private tail's
+// -- and a slot with lse = -inf (nothing attended) has no partial output:
+// its weight is zero and its output is never read.
 constexpr int kWarpMergeMax = 16;
 
-template <int D, typename OutT>
+template <int D, typename OutT, bool SHARED = false>
 __global__ void __launch_bounds__(256) decode_reduce_warp(const __grid_constant__ DecodeArgs a) {
     constexpr int VEC = D / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x * 8 + warp;
     if (bh >= a.num_seqs * a.H_q) return;
     const int b = bh / a.H_q;
-    const int ctx = clamped_ctx(a, b, false);
-    const int n = (ctx - span_base(a, ctx) + a.P - 1) / a.P;
-    if (n <= 1) return;
+    int n = a.S_max;
+    if constexpr (!SHARED) {
+        const int ctx = clamped_ctx(a, b, false);
+        n = (ctx - span_base(a, ctx) + a.P - 1) / a.P;
+        if (n <= 1) return;
+    }
     wait_for_primary_grid();
     const float *lse = a.part_lse + (size_t)bh * a.S_max;
     const float *po = a.part_o + (size_t)bh * a.S_max * D + lane * VEC;
@@ -60,7 +62,9 @@ __global__ void __launch_bounds__(256) decode_reduce_warp(const __grid_constant_
     if (M != -INFINITY) {
 #pragma unroll 4
         for (int s = 0; s < n; ++s) {
-            const float w = exp2f(__shfl_sync(0xffffffffu, my_lse, s) - M);
+            const float ls = __shfl_sync(0xffffffffu, my_lse, s);
+            if (SHARED && ls == -INFINITY) continue;  // an empty slot
+            const float w = exp2f(ls - M);
             W += w;
             if constexpr (VEC == 4) {
                 const float4 x = __ldcg(reinterpret_cast<const float4 *>(po + (size_t)s * D));
@@ -84,15 +88,18 @@ __global__ void __launch_bounds__(256) decode_reduce_warp(const __grid_constant_
 // warps taking every 16th partition, four partitions' loads in flight per
 // warp (a long context has hundreds of partials per head and only a few
 // heads, so the merge is latency-bound unless many loads are outstanding).
-template <int D, typename OutT>
+template <int D, typename OutT, bool SHARED = false>
 __global__ void __launch_bounds__(512) decode_reduce(const __grid_constant__ DecodeArgs a) {
     constexpr int NWR = 16;
     constexpr int VEC = D / 32;
     const int bh = blockIdx.x;
     const int b = bh / a.H_q;
-    const int ctx = clamped_ctx(a, b, false);
-    const int n = (ctx - span_base(a, ctx) + a.P - 1) / a.P;
-    if (n <= 1) return;
+    int n = a.S_max;
+    if constexpr (!SHARED) {
+        const int ctx = clamped_ctx(a, b, false);
+        n = (ctx - span_base(a, ctx) + a.P - 1) / a.P;
+        if (n <= 1) return;
+    }
     wait_for_primary_grid();
     const float *lse = a.part_lse + (size_t)bh * a.S_max;
     const float *po = a.part_o + (size_t)bh * a.S_max * D;
@@ -118,7 +125,9 @@ __global__ void __launch_bounds__(512) decode_reduce(const __grid_constant__ Dec
     if (M != -INFINITY) {
 #pragma unroll 4
         for (int s = warp; s < n; s += NWR) {
-            const float w = exp2f(__ldcg(lse + s) - M);
+            const float ls = __ldcg(lse + s);
+            if (SHARED && ls == -INFINITY) continue;  // an empty slot
+            const float w = exp2f(ls - M);
             W += w;
             const float *src = po + (size_t)s * D + lane * VEC;
             if constexpr (VEC == 4) {

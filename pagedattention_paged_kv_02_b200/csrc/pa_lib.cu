@@ -19,6 +19,7 @@
 #include "reshape_and_cache.cuh"
 #include "decode.cuh"
 #include "decode_merge.cuh"
+#include "decode_prefix.cuh"
 #include "decode_fp8.cuh"
 #include "prefill.cuh"
 #include "blocks.cuh"
@@ -131,9 +132,22 @@ pa_status launch_decode_f32(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
     return launch_status();
 }
 
+#ifndef PA_PREFILL_1Q
+#define PA_PREFILL_1Q 0
+#endif
+
+// query rows one prefill CTA covers
+constexpr int kPrefillCtaRows = PA_PREFILL_1Q ? kPfRows : kPfRows * kPfQTiles;
+
 template <int D, bool WIN>
 pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                             const CUtensorMap &mv, dim3 grid, cudaStream_t st) {
+#if PA_PREFILL_1Q
+    const size_t smem = 1024 + pf1_smem_bytes(D);
+    auto k = prefill_1q_kernel<D, WIN>;
+    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
+    k<<<grid, kP1Threads, smem, st>>>(a, mq, mk, mv);
+#else
     const size_t smem = 1024 + pf_smem_bytes(D);
     auto k = prefill_tc_kernel<D, WIN>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
@@ -143,6 +157,7 @@ pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const C
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return PA_ERR_CUDA;
     if ((long long)fa.numRegs * kPfThreads < kPfRegsNeeded) return PA_ERR_UNSUPPORTED;
     k<<<grid, kPfThreads, smem, st>>>(a, mq, mk, mv);
+#endif
     return launch_status();
 }
 
@@ -175,7 +190,7 @@ pa_status launch_decode_q8(const DecodeArgs &a, const CUtensorMap &mk, const CUt
 // The LSE merge behind a split launch, as a programmatic dependent launch
 // (its CTAs may start while the split grid's last CTAs run; they wait for
 // that grid's completion before reading partials).
-template <int D, typename OutT>
+template <int D, typename OutT, bool SHARED = false>
 pa_status launch_reduce(const DecodeArgs &a, cudaStream_t st) {
     const long long heads = (long long)a.num_seqs * a.H_q;
     cudaLaunchConfig_t cfg = {};
@@ -189,14 +204,94 @@ pa_status launch_reduce(const DecodeArgs &a, cudaStream_t st) {
     if (a.S_max <= kWarpMergeMax) {
         cfg.gridDim = dim3((unsigned)((heads + 7) / 8));
         cfg.blockDim = dim3(256);
-        if (cudaLaunchKernelEx(&cfg, decode_reduce_warp<D, OutT>, a) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, decode_reduce_warp<D, OutT, SHARED>, a) != cudaSuccess)
             return PA_ERR_CUDA;
     } else {
         cfg.gridDim = dim3((unsigned)heads);
         cfg.blockDim = dim3(512);
-        if (cudaLaunchKernelEx(&cfg, decode_reduce<D, OutT>, a) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, decode_reduce<D, OutT, SHARED>, a) != cudaSuccess)
             return PA_ERR_CUDA;
     }
+    return launch_status();
+}
+
+// ------------------------------------------------------ shared-prefix decode
+// Partition sizes and slot counts of the shared-prefix decode.
+struct SharedPlan {
+    int Pp, Pt;  // tokens per prefix / tail partition
+    int Sp, St;  // partial slots of the prefix / tail passes
+    int MT, row_tiles;
+};
+
+int round16(int n) { return ((n > 0 ? n : 1) + kChunk - 1) / kChunk * kChunk; }
+
+// false if partition_size cannot be met. Automatic: a tail in one partition
+// up to 2048 tokens, else 1024-token partitions; prefix partitions of 512
+// tokens, 256 when that leaves fewer than two CTAs per SM of a B200.
+bool shared_plan(int max_ctx, int max_prefix, int max_group, int group, int H_kv, int num_groups,
+                 int partition_size, SharedPlan &p) {
+    const int rows = max_group * group;
+    p.MT = rows <= 16 ? 1 : rows <= 32 ? 2 : 4;
+    p.row_tiles = (rows + p.MT * 16 - 1) / (p.MT * 16);
+    if (partition_size > 0) {
+        if (partition_size % kChunk != 0 || partition_size > kMaxPartition) return false;
+        p.Pp = p.Pt = partition_size;
+    } else if (partition_size < 0) {
+        p.Pt = round16(max_ctx);
+        p.Pp = round16(max_prefix);
+        if (p.Pt > kMaxPartition || p.Pp > kMaxPartition) return false;
+    } else {
+        p.Pt = max_ctx <= 2048 ? round16(max_ctx) : 1024;
+        p.Pp = 512;
+        const long long ctas = (long long)((max_prefix + 511) / 512) * H_kv * p.row_tiles * num_groups;
+        if (ctas < 2 * 148) p.Pp = 256;
+        if (max_prefix < p.Pp) p.Pp = round16(max_prefix);
+    }
+    p.Sp = (max_prefix + p.Pp - 1) / p.Pp;
+    p.St = (max_ctx + p.Pt - 1) / p.Pt;
+    if (p.St < 1) p.St = 1;
+    return true;
+}
+
+size_t shared_workspace_bytes(int B, int H_q, int D, const SharedPlan &p) {
+    const size_t S = (size_t)p.Sp + p.St;
+    const size_t o = (size_t)B * H_q * S * D * sizeof(float);
+    const size_t l = (size_t)B * H_q * S * sizeof(float);
+    return (o + 255) / 256 * 256 + (l + 255) / 256 * 256;
+}
+
+template <int D, int MT>
+pa_status launch_prefix(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv,
+                        dim3 grid, cudaStream_t st) {
+    using L = PrefixSmem<D, MT>;
+    const size_t smem = 1024 + L::kTable + ((size_t)a.P_prefix / a.bs + 2) * 4;
+    auto k = decode_prefix_bf16<D, MT>;
+    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
+    k<<<grid, kPrefixWarps * 32, smem, st>>>(a, mk, mv);
+    return launch_status();
+}
+
+// The tail pass, as a programmatic dependent of the prefix pass when there
+// is one (it reads nothing the prefix pass writes; it only finishes after it).
+template <int D>
+pa_status launch_tail(const DecodeArgs &a, const CUtensorMap &mk, const CUtensorMap &mv, dim3 grid,
+                      bool dependent, cudaStream_t st) {
+    constexpr int STAGE = 2 * kChunk * D * 2;
+    using L = DecodeSmem<kDecodeWarps, kDecodeStages, STAGE, kHeadsBf16, D>;
+    const size_t smem = 1024 + L::kTable + ((size_t)a.P / a.bs + 2) * 4;
+    auto k = decode_split_bf16<D, kDecodeWarps, kDecodeStages, true>;
+    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    cfg.stream = st;
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kDecodeWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    if (cudaLaunchKernelEx(&cfg, k, a, mk, mv) != cudaSuccess) return PA_ERR_CUDA;
     return launch_status();
 }
 
@@ -302,6 +397,7 @@ static pa_status decode_impl(void *out, const void *q, const void *k_cache, cons
     if (gy > 65535 || num_seqs > 65535 || S > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
 
     DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
     a.out = out;
     a.q = q;
     a.k_cache = k_cache;
@@ -485,6 +581,7 @@ static pa_status decode_q8_impl(void *out, const void *q, const void *k_cache,
     const long long gy = (long long)num_kv_heads * n_htiles;
     if (gy > 65535 || num_seqs > 65535 || S > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
     DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
     a.out = out;
     a.q = q;
     a.k_cache = k_cache;
@@ -574,7 +671,7 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
         return PA_ERR_INVALID_ARG;
-    const long long qtiles = (max_query_len + kPfRows * kPfQTiles - 1) / (kPfRows * kPfQTiles);
+    const long long qtiles = (max_query_len + kPrefillCtaRows - 1) / kPrefillCtaRows;
     if (qtiles > 65535 || num_chunks > 65535) return PA_ERR_UNSUPPORTED;
 
     EncodeTiledFn fn = encode_fn();
@@ -702,6 +799,133 @@ pa_status pa_swap_blocks(const void *src_k, const void *src_v, int src_blocks, v
                          cudaStream_t stream) {
     return launch_copy_blocks(src_k, src_v, src_blocks, dst_k, dst_v, dst_blocks, block_mapping,
                               num_pairs, num_kv_heads, head_dim, block_size, dtype, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+size_t pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                              int head_dim, int num_groups, int max_group_size,
+                                              int max_prefix_len, int max_context_len,
+                                              int partition_size) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        num_q_heads % num_kv_heads != 0 || num_groups < 0 || max_group_size <= 0 ||
+        max_prefix_len < 0 || max_context_len < 0)
+        return 0;
+    SharedPlan p;
+    if (!shared_plan(max_context_len, max_prefix_len, max_group_size,
+                     num_q_heads / num_kv_heads, num_kv_heads, num_groups, partition_size, p))
+        return 0;
+    return shared_workspace_bytes(num_seqs, num_q_heads, head_dim, p);
+}
+
+pa_status pa_decode_shared_prefix(void *out, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *block_tables,
+                                  const int32_t *context_lens, const int32_t *group_start,
+                                  const int32_t *prefix_lens, int num_groups, int max_group_size,
+                                  int max_prefix_len, int num_seqs, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                  int max_blocks_per_seq, int max_context_len, float scale,
+                                  int partition_size, void *workspace, size_t workspace_bytes_given,
+                                  pa_dtype dtype, cudaStream_t stream) {
+    if (num_seqs < 0 || num_groups < 0 || max_group_size <= 0 || max_prefix_len < 0 ||
+        num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (dtype != PA_BF16 || num_q_heads % num_kv_heads != 0 || !head_dim_ok(head_dim) ||
+        !block_size_ok(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if ((long long)max_context_len > (long long)max_blocks_per_seq * block_size ||
+        max_prefix_len > max_context_len)
+        return PA_ERR_INVALID_ARG;
+    if ((num_seqs == 0) != (num_groups == 0)) return PA_ERR_INVALID_ARG;
+    const int group = num_q_heads / num_kv_heads;
+    SharedPlan plan;
+    if (!shared_plan(max_context_len, max_prefix_len, max_group_size, group, num_kv_heads,
+                     num_groups, partition_size, plan))
+        return partition_size > 0 ? PA_ERR_INVALID_ARG : PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !group_start ||
+        !prefix_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(group_start, 4) ||
+        !aligned(prefix_lens, 4))
+        return PA_ERR_INVALID_ARG;
+    const size_t need = shared_workspace_bytes(num_seqs, num_q_heads, head_dim, plan);
+    if (!workspace || workspace_bytes_given < need || !aligned(workspace, 256))
+        return PA_ERR_WORKSPACE;
+    const int n_htiles = (group + kHeadsBf16 - 1) / kHeadsBf16;
+    const long long S = (long long)plan.Sp + plan.St;
+    const long long tail_x = (long long)max_group_size * plan.St;
+    if (num_groups > 65535 || (long long)num_kv_heads * plan.row_tiles > 65535 ||
+        (long long)num_kv_heads * n_htiles > 65535 || tail_x > 0x7fffffffLL || S > 0x7fffffffLL)
+        return PA_ERR_UNSUPPORTED;
+
+    DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.part_o = static_cast<float *>(workspace);
+    a.part_lse = reinterpret_cast<float *>(
+        static_cast<char *>(workspace) +
+        ((size_t)num_seqs * num_q_heads * S * head_dim * 4 + 255) / 256 * 256);
+    a.num_seqs = num_seqs;
+    a.H_q = num_q_heads;
+    a.H_kv = num_kv_heads;
+    a.group = group;
+    a.bs = block_size;
+    a.bs_shift = __builtin_ctz((unsigned)block_size);
+    a.NB = num_blocks;
+    a.MB = max_blocks_per_seq;
+    a.max_ctx = max_context_len;
+    a.P = plan.Pt;
+    a.S_max = (int)S;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.timeout_ns = kWaitTimeoutNs;
+    a.window = 0;
+    a.group_start = group_start;
+    a.prefix_lens = prefix_lens;
+    a.num_groups = num_groups;
+    a.max_group = max_group_size;
+    a.max_prefix = max_prefix_len;
+    a.P_prefix = plan.Pp;
+    a.S_prefix = plan.Sp;
+
+    CUtensorMap mk, mv;
+    if (!encode_cache_map(&mk, k_cache, num_blocks, num_kv_heads, block_size, head_dim, kChunk) ||
+        !encode_cache_map(&mv, v_cache, num_blocks, num_kv_heads, block_size, head_dim, kChunk))
+        return PA_ERR_CUDA;
+    pa_status st = PA_OK;
+    if (plan.Sp > 0) {
+        DecodeArgs ap = a;
+        ap.n_htiles = plan.row_tiles;  // row tiles of (member, head) rows
+        const dim3 grid((unsigned)plan.Sp, (unsigned)(num_kv_heads * plan.row_tiles),
+                        (unsigned)num_groups);
+        if (head_dim == 128)
+            st = plan.MT == 1   ? launch_prefix<128, 1>(ap, mk, mv, grid, stream)
+                 : plan.MT == 2 ? launch_prefix<128, 2>(ap, mk, mv, grid, stream)
+                                : launch_prefix<128, 4>(ap, mk, mv, grid, stream);
+        else
+            st = plan.MT == 1   ? launch_prefix<64, 1>(ap, mk, mv, grid, stream)
+                 : plan.MT == 2 ? launch_prefix<64, 2>(ap, mk, mv, grid, stream)
+                                : launch_prefix<64, 4>(ap, mk, mv, grid, stream);
+        if (st != PA_OK) return st;
+    }
+    a.n_htiles = n_htiles;
+    const dim3 tgrid((unsigned)tail_x, (unsigned)(num_kv_heads * n_htiles), (unsigned)num_groups);
+    st = head_dim == 128 ? launch_tail<128>(a, mk, mv, tgrid, plan.Sp > 0, stream)
+                         : launch_tail<64>(a, mk, mv, tgrid, plan.Sp > 0, stream);
+    if (st != PA_OK) return st;
+    return head_dim == 128 ? launch_reduce<128, __nv_bfloat16, true>(a, stream)
+                           : launch_reduce<64, __nv_bfloat16, true>(a, stream);
 }
 
 }  // extern "C"

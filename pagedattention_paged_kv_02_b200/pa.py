@@ -27,7 +27,8 @@ EXPORTS = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_partit
            "pa_selftest_bounded_wait", "pa_status_string", "pa_version",
            "pa_decode_static_workspace", "pa_copy_blocks", "pa_swap_blocks",
            "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window",
-           "pa_prefill_chunk_sliding_window", "pa_reshape_and_cache_int8", "pa_decode_int8")
+           "pa_prefill_chunk_sliding_window", "pa_reshape_and_cache_int8", "pa_decode_int8",
+           "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size")
 
 
 class PAError(RuntimeError):
@@ -66,6 +67,10 @@ def lib() -> ctypes.CDLL:
         L.pa_decode_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, SZ,
                                     P]
         L.pa_decode_int8.argtypes = L.pa_decode_fp8.argtypes
+        L.pa_decode_shared_prefix.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                              I, I, I, F, I, P, SZ, I, P]
+        L.pa_decode_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I]
+        L.pa_decode_shared_prefix_workspace_size.restype = SZ
         L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I, P]
         L.pa_swap_blocks.argtypes = [P, P, I, P, P, I, P, I, I, I, I, I, P]
         L.pa_check_tables.argtypes = [P, P, I, I, I, I, P, ctypes.POINTER(I), P]
@@ -77,7 +82,7 @@ def lib() -> ctypes.CDLL:
                   "pa_prefill_chunk", "pa_check_tables", "pa_copy_blocks", "pa_swap_blocks",
                   "pa_reshape_and_cache_fp8", "pa_decode_fp8", "pa_decode_sliding_window",
                   "pa_prefill_chunk_sliding_window", "pa_reshape_and_cache_int8",
-                  "pa_decode_int8", "pa_device_error",
+                  "pa_decode_int8", "pa_decode_shared_prefix", "pa_device_error",
                   "pa_selftest_bounded_wait", "pa_decode_partition_tokens", "pa_version"):
             getattr(L, f).restype = I
         _lib = L
@@ -166,6 +171,57 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
     _call("pa_decode", _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
           _p(context_lens), B, H_q, H_kv, D, bs, NB, MB, int(max_context_len), float(scale),
           int(partition_size), _p(workspace), ws_bytes, _dt(q), _stream(stream))
+
+
+def pa_decode_shared_prefix_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                                           head_dim: int, num_groups: int, max_group_size: int,
+                                           max_prefix_len: int, max_context_len: int,
+                                           partition_size: int = 0) -> int:
+    """Bytes of workspace ``pa_decode_shared_prefix`` needs (0: invalid arguments)."""
+    return int(lib().pa_decode_shared_prefix_workspace_size(
+        int(num_seqs), int(num_q_heads), int(num_kv_heads), int(head_dim), int(num_groups),
+        int(max_group_size), int(max_prefix_len), int(max_context_len), int(partition_size)))
+
+
+def prepare_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens,
+                                 group_start, prefix_lens, max_group_size: int,
+                                 max_prefix_len: int, max_context_len: int, scale: float,
+                                 partition_size: int = 0,
+                                 workspace: Optional[torch.Tensor] = None) -> "Prepared":
+    """``pa_decode_shared_prefix``: sequences listed group by group (group g =
+    ``[group_start[g], group_start[g+1])``) sharing their first
+    ``prefix_lens[g]`` positions."""
+    for t, n in ((block_tables, "block_tables"), (context_lens, "context_lens"),
+                 (group_start, "group_start"), (prefix_lens, "prefix_lens")):
+        _check_int(t, torch.int32, n)
+    B, H_q, D = q.shape
+    NB, H_kv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or out.dtype != q.dtype:
+        raise ValueError("out must match q; caches must share head_dim")
+    if not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise TypeError("q and caches must share one dtype")
+    G = prefix_lens.numel()
+    if group_start.numel() != G + 1:
+        raise ValueError("group_start must have num_groups + 1 entries")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return Prepared("pa_decode_shared_prefix",
+                    (_p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables),
+                     _p(context_lens), _p(group_start), _p(prefix_lens), G, int(max_group_size),
+                     int(max_prefix_len), B, H_q, H_kv, D, bs, NB, block_tables.shape[1],
+                     int(max_context_len), float(scale), int(partition_size), _p(workspace),
+                     ws_bytes, _dt(q)))
+
+
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                            prefix_lens, max_group_size: int, max_prefix_len: int,
+                            max_context_len: int, scale: float, partition_size: int = 0,
+                            workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Paged decode reading each group's shared prefix once for all its
+    sequences; same result as :func:`pa_decode`. ``workspace``: at least
+    :func:`pa_decode_shared_prefix_workspace_size` bytes."""
+    prepare_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens,
+                                 group_start, prefix_lens, max_group_size, max_prefix_len,
+                                 max_context_len, scale, partition_size, workspace)(stream)
 
 
 def pa_decode_sliding_window(out, q, k_cache, v_cache, block_tables, context_lens,

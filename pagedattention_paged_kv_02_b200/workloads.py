@@ -72,6 +72,14 @@ class Batch:
     k_scale: Optional[torch.Tensor] = None  # 8-bit pools: float32 [H_kv] per-head scales
     v_scale: Optional[torch.Tensor] = None
     sliding_window: int = 0  # > 0: every query sees only its last sliding_window positions
+    # shared prefixes of the decode sequences, as the engine's block manager
+    # knows them: group g = sequences [decode_group_start[g],
+    # decode_group_start[g+1]) sharing their first decode_prefix_lens[g]
+    # positions (int32; None when the batch has no groups)
+    decode_group_start: Optional[torch.Tensor] = None
+    decode_prefix_lens: Optional[torch.Tensor] = None
+    max_group_size: int = 0
+    max_prefix_len: int = 0
 
     @property
     def num_blocks(self) -> int:
@@ -237,6 +245,29 @@ def build_pool(specs: Sequence[SeqSpec], num_kv_heads: int, head_dim: int, block
     return k_cache, v_cache, tables, key, value, slot_mapping, poison
 
 
+def prefix_groups(groups: Sequence[int], prefix: int):
+    """The group structure of a list of per-sequence group ids (-1: shares
+    nothing): (group_start int32 [G+1], prefix_lens int32 [G], largest group,
+    longest prefix). Sharing sequences must be listed group by group; each
+    non-sharing sequence is a group of one with prefix 0."""
+    starts, lens = [0], []
+    for i, g in enumerate(groups):
+        if i > 0 and g >= 0 and g == groups[i - 1]:
+            continue  # same group as the previous sequence
+        if g >= 0 and g in groups[:i]:
+            raise ValueError("sequences of a group must be consecutive")
+        if i > 0:
+            starts.append(i)
+        lens.append(prefix if g >= 0 else 0)
+    if groups:
+        starts.append(len(groups))
+    else:
+        starts = [0]
+    sizes = [b - a for a, b in zip(starts[:-1], starts[1:])]
+    return (torch.tensor(starts, dtype=torch.int32), torch.tensor(lens, dtype=torch.int32),
+            max(sizes + [1]), max(lens + [0]))
+
+
 def decode_batch(context_lens: Sequence[int], num_q_heads: int, num_kv_heads: int,
                  head_dim: int, block_size: int, num_blocks: int, dtype=torch.bfloat16,
                  std: float = 1.0, seed: int = 0, scale: Optional[float] = None,
@@ -254,11 +285,16 @@ def decode_batch(context_lens: Sequence[int], num_q_heads: int, num_kv_heads: in
         specs, num_kv_heads, head_dim, block_size, num_blocks, dtype, std, gen,
         max_blocks_per_seq)
     q = _randn(gen, (len(specs), num_q_heads, head_dim), std, dtype)
+    grp = {}
+    if groups is not None:
+        gs, pl, mg, mp = prefix_groups([int(x) for x in groups], prefix)
+        grp = dict(decode_group_start=gs, decode_prefix_lens=pl, max_group_size=mg,
+                   max_prefix_len=mp)
     return Batch(name=name, k_cache=k, v_cache=v, key=key, value=value, slot_mapping=slots,
                  scale=scale if scale is not None else 1.0 / math.sqrt(head_dim),
                  block_size=block_size, poison_block=poison, q=q, block_tables=tables,
                  context_lens=torch.tensor([int(c) for c in context_lens], dtype=torch.int32),
-                 partition_size=partition_size)
+                 partition_size=partition_size, **grp)
 
 
 def mixed_batch(cached: Sequence[int], chunk: int, decode_ctx: Sequence[int],
@@ -280,13 +316,18 @@ def mixed_batch(cached: Sequence[int], chunk: int, decode_ctx: Sequence[int],
     mb_d = max(1, max(_ceil_div(s.ctx, block_size) for s in dec)) if dec else 1
     pq = _randn(gen, (n_pre * chunk, num_q_heads, head_dim), std, dtype)
     dq = _randn(gen, (len(dec), num_q_heads, head_dim), std, dtype)
+    grp = {}
+    if decode_groups is not None:
+        gs, pl, mg, mp = prefix_groups([int(x) for x in decode_groups], prefix)
+        grp = dict(decode_group_start=gs, decode_prefix_lens=pl, max_group_size=mg,
+                   max_prefix_len=mp)
     return Batch(name=name, k_cache=k, v_cache=v, key=key, value=value, slot_mapping=slots,
                  scale=1.0 / math.sqrt(head_dim), block_size=block_size, poison_block=poison,
                  q=dq, block_tables=tables[n_pre:, :mb_d].contiguous(),
                  context_lens=torch.tensor([s.ctx for s in dec], dtype=torch.int32),
                  prefill_q=pq, prefill_block_tables=tables[:n_pre, :mb_p].contiguous(),
                  prefill_context_lens=torch.tensor([s.ctx for s in pre], dtype=torch.int32),
-                 query_start_loc=torch.arange(0, n_pre + 1, dtype=torch.int32) * chunk)
+                 query_start_loc=torch.arange(0, n_pre + 1, dtype=torch.int32) * chunk, **grp)
 
 
 # ---------------------------------------------------------------------------
@@ -299,19 +340,22 @@ def tiny_fp32(seed: int = 0) -> Batch:
                         scale=1.0 / 8.0, name="tiny_fp32_b4_d64")
 
 
-def llama7b_decode(seed: int = 0, num_blocks: int = 16384, block_size: int = 16) -> Batch:
+def llama7b_decode(seed: int = 0, num_blocks: int = 16384, block_size: int = 16,
+                   head_dim: int = 128) -> Batch:
     """Llama-2-7B-shaped decode: 64 sequences with lengths uniform in
     [128, 2048], 32/32 heads, head_dim 128, 16-token blocks, 16384-block pool,
-    bf16, N(0,1)."""
+    bf16, N(0,1). Other block sizes and head_dim 64 keep the lengths (and,
+    for block sizes, the pool's bytes)."""
     gen = torch.Generator().manual_seed(seed + 7919)
     lens = torch.randint(128, 2049, (64,), generator=gen).tolist()
     nb, mb = num_blocks * 16 // block_size, 2048 // block_size  # same pool bytes
-    return decode_batch(lens, 32, 32, 128, block_size, nb, torch.bfloat16, 1.0, seed,
+    return decode_batch(lens, 32, 32, head_dim, block_size, nb, torch.bfloat16, 1.0, seed,
                         max_blocks_per_seq=mb,
-                        name=f"llama7b_decode_b64_h32_d128_bs{block_size}")
+                        name=f"llama7b_decode_b64_h32_d{head_dim}_bs{block_size}")
 
 
-def gqa_decode(seed: int = 0, num_blocks: int = 32768, block_size: int = 16) -> Batch:
+def gqa_decode(seed: int = 0, num_blocks: int = 32768, block_size: int = 16,
+               head_dim: int = 128) -> Batch:
     """GQA decode: 128 sequences, lengths log-normal with median 1024 and
     sigma 0.75 (natural-log scale) clipped to [16, 4096], 64 q / 8 kv heads,
     head_dim 128, 16-token blocks, 32768-block pool, bf16, N(0,1)."""
@@ -319,9 +363,9 @@ def gqa_decode(seed: int = 0, num_blocks: int = 32768, block_size: int = 16) -> 
     z = torch.randn(128, generator=gen, dtype=torch.float64)
     lens = torch.exp(math.log(1024.0) + 0.75 * z).round().clamp(16, 4096).to(torch.int64).tolist()
     nb, mb = num_blocks * 16 // block_size, 4096 // block_size  # same pool bytes
-    return decode_batch(lens, 64, 8, 128, block_size, nb, torch.bfloat16, 1.0, seed,
+    return decode_batch(lens, 64, 8, head_dim, block_size, nb, torch.bfloat16, 1.0, seed,
                         max_blocks_per_seq=mb,
-                        name=f"gqa_decode_b128_h64kv8_d128_bs{block_size}")
+                        name=f"gqa_decode_b128_h64kv8_d{head_dim}_bs{block_size}")
 
 
 def long_context_decode(seed: int = 0, num_blocks: int = 8192) -> Batch:
@@ -333,7 +377,7 @@ def long_context_decode(seed: int = 0, num_blocks: int = 8192) -> Batch:
                         name="long_ctx_decode_b4_h32kv8_d128_bs64_p512")
 
 
-def mixed_prefill_decode(seed: int = 0, num_blocks: int = 16384) -> Batch:
+def mixed_prefill_decode(seed: int = 0, num_blocks: int = 16384, head_dim: int = 128) -> Batch:
     """8 prefill chunks of 512 query tokens after round(i*4096/7) cached tokens
     (i = 0..7), plus 192 decode sequences in 24 groups of 8 beams sharing a
     1024-token prefix (64 shared blocks) with private tails uniform in
@@ -343,8 +387,9 @@ def mixed_prefill_decode(seed: int = 0, num_blocks: int = 16384) -> Batch:
     tails = torch.randint(64, 513, (192,), generator=gen).tolist()
     ctx = [1024 + t for t in tails]
     groups = [b // 8 for b in range(192)]
-    return mixed_batch(cached, 512, ctx, groups, 1024, 32, 8, 128, 16, num_blocks, torch.bfloat16,
-                       1.0, seed, name="mixed_prefill8x512_decode192_h32kv8_d128_bs16")
+    return mixed_batch(cached, 512, ctx, groups, 1024, 32, 8, head_dim, 16, num_blocks,
+                       torch.bfloat16, 1.0, seed,
+                       name=f"mixed_prefill8x512_decode192_h32kv8_d{head_dim}_bs16")
 
 
 def to_fp8(batch: Batch, k_amax: float = 4.0, v_amax: float = 4.0) -> Batch:

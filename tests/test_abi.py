@@ -144,10 +144,10 @@ def test_prefill_host_checks(L):
     b = list(base)
     b[7] = 0
     assert f(*b) == pa.PA_OK
-    # the grid is (query head, tile pair, chunk): at most 65535 pairs of 256 queries and
-    # 65535 chunks; any number of query heads
+    # the grid is (query head, query tile, chunk): at most 65535 tiles of 128 queries
+    # and 65535 chunks; any number of query heads
     b = list(base)
-    b[8], b[9] = 65536 * 256, 65536 * 256
+    b[8], b[9] = 65535 * 128 + 1, 65535 * 128 + 1
     assert f(*b) == pa.PA_ERR_UNSUPPORTED
     b = list(base)
     b[7] = 65536
@@ -188,3 +188,62 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(pa, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         pa.lib()
+
+
+def test_shared_prefix_workspace_arithmetic(L):
+    """Slots: prefix partitions then tail partitions per (sequence, head)."""
+    from pagedattention_paged_kv_02_b200 import pa
+    f = pa.pa_decode_shared_prefix_workspace_size
+
+    def ws(B, Hq, D, S):
+        o = B * Hq * S * D * 4
+        return (o + 255) // 256 * 256 + (B * Hq * S * 4 + 255) // 256 * 256
+
+    # explicit 256-token partitions: 1024-token prefix -> 4 slots, 1536-token
+    # contexts -> 6 tail slots
+    assert f(192, 32, 8, 128, 24, 8, 1024, 1536, 256) == ws(192, 32, 128, 10)
+    # never split: one prefix slot and one tail slot
+    assert f(192, 32, 8, 128, 24, 8, 1024, 1536, -1) == ws(192, 32, 128, 2)
+    # automatic: 24 groups x 8 KV heads x 1 row tile x 2 partitions of 512
+    # -> 384 prefix CTAs (>= 2 per SM), tails in one partition up to 2048
+    assert f(192, 32, 8, 128, 24, 8, 1024, 1536, 0) == ws(192, 32, 128, 3)
+    # few groups: 256-token prefix partitions
+    assert f(16, 32, 8, 128, 2, 8, 1024, 1536, 0) == ws(16, 32, 128, 5)
+    # no prefix at all: tail slots only
+    assert f(8, 8, 8, 64, 8, 1, 0, 100, 0) == ws(8, 8, 64, 1)
+    # invalid: odd partition, heads not grouped, prefix bound above context bound
+    assert f(8, 8, 8, 128, 8, 1, 64, 100, 24) == 0
+    assert f(8, 6, 4, 128, 8, 1, 64, 100, 0) == 0
+    assert f(8, 8, 8, 128, 8, 0, 64, 100, 0) == 0
+
+
+def _shared(L, **kw):
+    args = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, tables=FAKE, lens=FAKE, gs=FAKE, pl=FAKE,
+                G=2, maxg=4, maxp=64, B=8, Hq=8, Hkv=2, D=128, bs=16, NB=64, MB=8, max_ctx=128,
+                scale=0.1, part=0, ws=None, ws_bytes=0, dtype=1)
+    args.update(kw)
+    a = args
+    return L.pa_decode_shared_prefix(a["out"], a["q"], a["k"], a["v"], a["tables"], a["lens"],
+                                     a["gs"], a["pl"], a["G"], a["maxg"], a["maxp"], a["B"],
+                                     a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"], a["MB"],
+                                     a["max_ctx"], a["scale"], a["part"], a["ws"], a["ws_bytes"],
+                                     a["dtype"], None)
+
+
+def test_shared_prefix_host_checks(L):
+    from pagedattention_paged_kv_02_b200 import pa
+    assert _shared(L, dtype=0) == pa.PA_ERR_UNSUPPORTED     # fp32: not offered
+    assert _shared(L, D=96) == pa.PA_ERR_UNSUPPORTED
+    assert _shared(L, Hq=6, Hkv=4) == pa.PA_ERR_UNSUPPORTED
+    assert _shared(L, gs=None) == pa.PA_ERR_INVALID_ARG
+    assert _shared(L, pl=ctypes.c_void_p(0x10002)) == pa.PA_ERR_INVALID_ARG
+    assert _shared(L, maxg=0) == pa.PA_ERR_INVALID_ARG
+    assert _shared(L, maxp=129) == pa.PA_ERR_INVALID_ARG   # prefix bound above the context bound
+    assert _shared(L, G=0) == pa.PA_ERR_INVALID_ARG        # sequences but no groups
+    assert _shared(L, part=24) == pa.PA_ERR_INVALID_ARG
+    # the workspace is always needed: both passes leave partials
+    assert _shared(L) == pa.PA_ERR_WORKSPACE
+    need = pa.pa_decode_shared_prefix_workspace_size(8, 8, 2, 128, 2, 4, 64, 128, 0)
+    assert _shared(L, ws=FAKE, ws_bytes=need - 1) == pa.PA_ERR_WORKSPACE
+    assert _shared(L, ws=ctypes.c_void_p(0x10010), ws_bytes=need) == pa.PA_ERR_WORKSPACE
+    assert _shared(L, B=0, G=0) == pa.PA_OK

@@ -88,9 +88,9 @@ def test_prefill_edge_chunks(pa, cached, lens):
 
 def test_prefill_chunk_longer_than_max_query_len(pa):
     """A chunk of 300 queries launched with max_query_len 200: the grid covers
-    256 rows of it (200 rounded up to the CTA's 256). Rows 0..255 are
-    computed as usual, rows 256..299 are left as they were (NaN poison) and
-    the chunk is recorded as PA_ERR_BAD_TABLE."""
+    256 rows of it (200 rounded up to a multiple of the CTA's 128). Rows
+    0..255 are computed as usual, rows 256..299 are left as they were (NaN
+    poison) and the chunk is recorded as PA_ERR_BAD_TABLE."""
     batch = mixed_chunks([40], [300], 8, 2, 16, seed=104)
     d = batch.to(DEV)
     pa.pa_reshape_and_cache(d.key, d.value, d.k_cache, d.v_cache, d.slot_mapping)
