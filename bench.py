@@ -399,6 +399,49 @@ class Runner:
         return "prefill" if self.d.prefill_q is not None else "decode"
 
 
+def scatter_burst_ms(r, batch, dev, pair, burst=16):
+    """Mean duration of one cache scatter of the step's size, over `burst`
+    launches replayed from a CUDA graph, each with its own key/value rows
+    and its own slots in a scratch pool (the pool is the step's shape, so
+    the slots spread over the same bytes)."""
+    import torch
+    pa = r.pa
+    T = batch.slot_mapping.numel()
+    NB, H, bs, D = batch.k_cache.shape
+    kc = torch.empty_like(r.d.k_cache)
+    vc = torch.empty_like(r.d.v_cache)
+    g = torch.Generator(device=dev).manual_seed(1234)
+    n_slots = NB * bs
+    per = min(T, n_slots // burst)
+    perm = torch.randperm(n_slots, generator=g, device=dev)
+    calls = []
+    for i in range(burst):
+        key = torch.randn(per, H, D, generator=g, device=dev).to(batch.key.dtype)
+        val = torch.randn(per, H, D, generator=g, device=dev).to(batch.key.dtype)
+        slots = perm[i * per:(i + 1) * per].to(torch.int64).contiguous()
+        if batch.k_scale is not None:
+            c = pa.prepare_reshape_and_cache_fp8(key, val, kc, vc, slots, r.d.k_scale, r.d.v_scale)
+        else:
+            c = pa.prepare_reshape_and_cache(key, val, kc, vc, slots)
+        calls.append((c, key, val, slots))
+    bg = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(bg, stream=side):
+            for c, *_ in calls:
+                c(side)
+    torch.cuda.current_stream().wait_stream(side)
+    bg.replay()
+    b0, b1 = pair()
+    b0.record()
+    bg.replay()
+    b1.record()
+    torch.cuda.synchronize()
+    # scaled to the step's token count when a launch moved fewer
+    return b0.elapsed_time(b1) / burst * (T / per)
+
+
 def run_ours(args, rank, world):
     import torch
     dev = torch.device("cuda:0")
@@ -465,15 +508,11 @@ def run_ours(args, rank, world):
     dec_ms = statistics.fmean(call_ms("decode")) if "decode" in r._calls else None
     # the scatter is a few microseconds: events around one launch measure
     # mostly the launch itself, so its duration is taken over a burst of
-    # back-to-back launches (re-appending the same rows is idempotent)
-    burst = 50
-    b0, b1 = pair()
-    b0.record()
-    for _ in range(burst):
-        r._calls["reshape"]()
-    b1.record()
-    torch.cuda.synchronize()
-    rs_ms = b0.elapsed_time(b1) / burst
+    # back-to-back launches replayed from one CUDA graph. Each launch of the
+    # burst moves its own rows (fresh inputs, distinct slots of a scratch
+    # pool of the same shape), so that neither the rows read nor the lines
+    # written are still in L2 from the launch before.
+    rs_ms = scatter_burst_ms(r, batch, dev, pair)
     pct = lambda q: dom_all[min(len(dom_all) - 1, int(q * len(dom_all)))]
 
     units = dbytes if r.dominant == "decode" else pflops
@@ -669,7 +708,9 @@ def run_ours(args, rank, world):
                     "kernel": ("pa_decode_shared_prefix (prefix + tails + merge)" if r.shared
                                else "pa_decode (decode_split + merge)"),
                     "ms": round(dec_ms, 5), "logical_bytes_GBps": round(
-                        dbytes / (dec_ms * 1e-3) / 1e9, 1)}
+                        dbytes / (dec_ms * 1e-3) / 1e9, 1),
+                    "traffic": (profiled_traffic(f"decode_shared_prefix_{args.workload}.md",
+                                                 SHARED_DECODE_SOURCES) if r.shared else None)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(batch, args.cpu_seconds)
     if world > 1:
@@ -686,6 +727,10 @@ PREFILL_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/prefill.cuh",
 DECODE_FP8_SOURCES = DECODE_SOURCES + ["pagedattention_paged_kv_02_b200/csrc/decode_fp8.cuh"]
 RESHAPE_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/reshape_and_cache.cuh",
                    "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
+SHARED_DECODE_SOURCES = ["pagedattention_paged_kv_02_b200/csrc/decode.cuh",
+                         "pagedattention_paged_kv_02_b200/csrc/decode_prefix.cuh",
+                         "pagedattention_paged_kv_02_b200/csrc/decode_merge.cuh",
+                         "pagedattention_paged_kv_02_b200/csrc/pa_device.cuh"]
 
 
 def workload_config(batch, name, world, r=None):

@@ -343,8 +343,9 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache
     a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.num_kv_heads = num_kv_heads;
     a.num_slots = (long long)num_blocks * block_size;
+    const long long groups = (num_tokens + kScatterTokens - 1) / kScatterTokens;
     const dim3 grid((unsigned)((a.vecs_per_token + kScatterThreads - 1) / kScatterThreads),
-                    (unsigned)(num_tokens < 65535 ? num_tokens : 65535));
+                    (unsigned)(groups < 65535 ? groups : 65535));
     reshape_and_cache_kernel<<<grid, kScatterThreads, 0, stream>>>(a);
     return launch_status();
 }

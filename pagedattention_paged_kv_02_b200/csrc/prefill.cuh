@@ -60,6 +60,12 @@ constexpr int kPfCtlRegs = 56;
 constexpr int kPfSoftmaxRegs = 224;
 constexpr int kPfRegsNeeded = 128 * (2 * kPfSoftmaxRegs + kPfCtlRegs);
 constexpr int kPfTblMax = 4096;   // block-table entries staged in shared memory
+#ifndef PA_PREFILL_POLY_EVERY
+#define PA_PREFILL_POLY_EVERY 0
+#endif
+// every kPfPolyEvery-th pair of exponentials of an unmasked tile on the FMA
+// pipe (ex2_poly2), the rest on the special-function unit; 0: none
+constexpr int kPfPolyEvery = PA_PREFILL_POLY_EVERY;
 // A Q, K or V tile: 128 rows of head_dim bf16, as head_dim/64 halves of 128 x
 // 128 bytes (one 128-byte swizzle atom wide), each 16 KB.
 __host__ __device__ constexpr int pf_tile_bytes(int D) { return kPfRows * D * 2; }
@@ -215,10 +221,45 @@ __device__ __forceinline__ bool pf_wait(PfBars *bars, uint64_t *bar, uint32_t pa
     return ok;
 }
 
+// Two non-negative finite fp32 values -> a bf16 pair (lo in the low half),
+// rounded to nearest on the integer pipe: half a bf16 ulp added to the fp32
+// bits, the upper halves kept (a tie, low half exactly 0x8000, rounds away
+// from zero instead of to even). The softmax's conversion instruction would
+// otherwise share the special-function pipe with its exponentials.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
+#if !defined(PA_PREFILL_PACK_CVT) || PA_PREFILL_PACK_CVT
+    return pack_bf16x2(lo, hi);
+#else
+    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+#endif
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for a pair of values on the FMA pipe (packed f32x2), so that part of
+// the softmax's exponentials leave the special-function pipe. Cody-Waite
+// style: x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low
+// mantissa bits) and |f| <= 1/2; 2^f by a cubic whose coefficients were
+// fitted for minimum maximum relative error on [-1/2, 1/2] (1.02e-4, exact at
+// f = 0: below the bf16 rounding of the weights); 2^n is added to the
+// exponent field. Inputs below -125 give 2^-125.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 t = __fadd2_rn(x, magic);
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(0.05500824f, 0.05500824f), f,
+                          make_float2(0.24220951f, 0.24220951f));
+    p = __ffma2_rn(p, f, make_float2(0.69328284f, 0.69328284f));
+    p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // WIN: the sliding-window build; without it the band logic folds away at
@@ -345,7 +386,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
     if (warp >= 8) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfCtlRegs));
-      if (warp == 8) {
+#ifndef PA_PREFILL_SPLIT_KV
+#define PA_PREFILL_SPLIT_KV 0
+#endif
+      // K and V streamed by warps 8 and 10 (SPLIT_KV), or both by warp 8
+      if (warp == 8 || (PA_PREFILL_SPLIT_KV && warp == 10)) {
+        const bool do_k = warp == 8, do_v = !PA_PREFILL_SPLIT_KV || warp == 10;
         // ------------------------------------------------------------ TMA
         // One box per lane: a thread issuing tensor copies back to back is
         // slow (each issue takes a while to be accepted), so the 16 boxes
@@ -379,17 +425,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int j = jmin; j < jmax; ++j) {
             const int st = (j - jmin) % kPfStages;
             const uint32_t use = (j - jmin) / kPfStages;
-            if (use > 0 && !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
-                break;
-            issue(sK + st * TB, &tmk, &bars->k_full[st], j);
-            k_issued = j - jmin + 1;
-            if (use > 0 && !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
-                break;
-            issue(sV + st * TB, &tmv, &bars->v_full[st], j);
-            v_issued = j - jmin + 1;
+            if (do_k) {
+                if (use > 0 &&
+                    !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
+                    break;
+                issue(sK + st * TB, &tmk, &bars->k_full[st], j);
+                k_issued = j - jmin + 1;
+            }
+            if (do_v) {
+                if (use > 0 &&
+                    !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
+                    break;
+                issue(sV + st * TB, &tmv, &bars->v_full[st], j);
+                v_issued = j - jmin + 1;
+            }
         }
         if (bars->abort && lane == 0) {  // let copies already in flight land
-            mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
+            if (do_k) mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
             for (int j = max(0, k_issued - kPfStages); j < k_issued; ++j)
                 mbar_wait(smem_u32(&bars->k_full[j % kPfStages]), (j / kPfStages) & 1,
                           a.timeout_ns);
@@ -561,7 +613,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const float p1 = k0 + 1 <= pos && (!WIN || k0 + 1 >= lo)
                                          ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m)) : 0.f;
                     ls[e & 3] += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    pk[e] = pack_bf16x2_int(p0, p1);
                 }
             } else {
                 // scale and shift as one packed f32x2 FMA per key pair, the
@@ -574,9 +626,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const float2 t = __ffma2_rn(
                         make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2v,
                         nmv);
-                    const float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
+                    float p0, p1;
+                    if (kPfPolyEvery > 0 && e % (kPfPolyEvery > 0 ? kPfPolyEvery : 1) == 0) {
+                        const float2 pp = ex2_poly2(t);
+                        p0 = pp.x;
+                        p1 = pp.y;
+                    } else {
+                        p0 = ex2_approx(t.x);
+                        p1 = ex2_approx(t.y);
+                    }
                     acc2[e & 1] = __fadd2_rn(acc2[e & 1], make_float2(p0, p1));
-                    pk[e] = pack_bf16x2(p0, p1);
+                    pk[e] = pack_bf16x2_int(p0, p1);
                 }
                 ls[0] = acc2[0].x;
                 ls[1] = acc2[0].y;
@@ -662,11 +722,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 // buffer, any completion the softmax can ask for is within one phase of the
 // barrier (S(u) landing implies P.V(u-2) completed), so the softmax waits on
 // it only when it must rescale O, and in the epilogue.
-constexpr int kP1Threads = 192;  // softmax warpgroup, TMA warp, MMA warp
+constexpr int kP1Threads = 224;  // softmax warpgroup, K warp, MMA warp, V warp
+// ring depths: a K tile is freed when its S completes and is needed two
+// tiles ahead of the softmax, a V tile when its P.V completes; K and V are
+// streamed by warps of their own, so neither load waits behind the other
+constexpr int kP1KStages = 3;
+constexpr int kP1VStages = 2;
 
 struct Pf1Bars {
     uint64_t q_full;
-    uint64_t k_full[kPfStages], k_free[kPfStages], v_full[kPfStages], v_free[kPfStages];
+    uint64_t k_full[kP1KStages], k_free[kP1KStages], v_full[kP1VStages], v_free[kP1VStages];
     uint64_t s_full[2], p_full[2], o_full[2];
     uint64_t fin;
     uint32_t tmem_base;
@@ -675,7 +740,7 @@ struct Pf1Bars {
 static_assert(sizeof(Pf1Bars) <= 512, "barriers fit their slot");
 
 __host__ __device__ constexpr int pf1_smem_bytes(int D) {
-    return (1 + 2 * kPfStages) * pf_tile_bytes(D) + 512 + kPfTblMax * 4;
+    return (1 + kP1KStages + kP1VStages) * pf_tile_bytes(D) + 512 + kPfTblMax * 4;
 }
 
 __device__ __forceinline__ bool pf1_wait(Pf1Bars *bars, uint64_t *bar, uint32_t parity,
@@ -700,11 +765,12 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
+    constexpr int KS = kP1KStages, VS = kP1VStages;
     const uint32_t sQ = smem_u32(smem);            // the Q tile
     const uint32_t sK = sQ + TB;                   // K stage st at sK + st*TB
-    const uint32_t sV = sK + kPfStages * TB;       // V stage st at sV + st*TB
-    Pf1Bars *bars = reinterpret_cast<Pf1Bars *>(smem + (1 + 2 * kPfStages) * TB);
-    int32_t *tbl = reinterpret_cast<int32_t *>(smem + (1 + 2 * kPfStages) * TB + 512);
+    const uint32_t sV = sK + KS * TB;              // V stage st at sV + st*TB
+    Pf1Bars *bars = reinterpret_cast<Pf1Bars *>(smem + (1 + KS + VS) * TB);
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + (1 + KS + VS) * TB + 512);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // CTAs start in order of decreasing work: the last chunk first, within it
@@ -743,9 +809,11 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     if (warp == 4) {
       if (lane == 0) {
         mbar_init(smem_u32(&bars->q_full), 1);
-        for (int st = 0; st < kPfStages; ++st) {
+        for (int st = 0; st < KS; ++st) {
             mbar_init(smem_u32(&bars->k_full[st]), 1);
             mbar_init(smem_u32(&bars->k_free[st]), 1);
+        }
+        for (int st = 0; st < VS; ++st) {
             mbar_init(smem_u32(&bars->v_full[st]), 1);
             mbar_init(smem_u32(&bars->v_free[st]), 1);
         }
@@ -792,12 +860,23 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ TMA
-        // one 16-token x 64-dim box per lane (16 lanes per K or V tile);
-        // lane 0 arms the barrier with the bytes of the pieces that exist
+    if (warp == 4 || warp == 6) {
+        // ----------------------------------------------------- TMA (K, V)
+        // warp 4 streams K, warp 6 V, each into its own ring; one 16-token
+        // x 64-dim box per lane (16 lanes per tile); lane 0 arms the
+        // barrier with the bytes of the pieces that exist
+        const bool is_k = warp == 4;
+        const int NSt = is_k ? KS : VS;
+        const CUtensorMap *map = is_k ? &tmk : &tmv;
+        uint64_t *full = is_k ? bars->k_full : bars->v_full;
+        uint64_t *freeb = is_k ? bars->k_free : bars->v_free;
+        const uint32_t ring = is_k ? sK : sV;
         const int s16 = lane / HALVES, half = lane % HALVES;
-        auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j) {
+        int issued = 0;  // tiles issued, counted from jlo
+        for (int j = jlo; j < jhi; ++j) {
+            const int st = (j - jlo) % NSt;
+            const uint32_t use = (j - jlo) / NSt;
+            if (use > 0 && !pf1_wait(bars, &freeb[st], (use - 1) & 1, a.timeout_ns, true)) break;
             const int key = j * kPfKeys + s16 * 16;
             int id = -1;
             if (lane < 8 * HALVES && key < ctx && (!WIN || key + 15 >= chunk_lo)) {
@@ -813,33 +892,17 @@ __global__ void __launch_bounds__(kP1Threads, 1)
                 }
             }
             const int n = __popc(__ballot_sync(0xffffffffu, id >= 0));
-            if (lane == 0) mbar_arrive_expect_tx(smem_u32(bar), n * 2048);
+            if (lane == 0) mbar_arrive_expect_tx(smem_u32(&full[st]), n * 2048);
             __syncwarp();
             if (id >= 0)
-                tma_load_4d(dst + half * 16384 + s16 * 2048, map, smem_u32(bar), half * 64,
-                            key & (a.bs - 1), kvh, id);
-        };
-        int k_issued = 0, v_issued = 0;  // counted from jlo
-        for (int j = jlo; j < jhi; ++j) {
-            const int st = (j - jlo) % kPfStages;
-            const uint32_t use = (j - jlo) / kPfStages;
-            if (use > 0 && !pf1_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
-                break;
-            issue(sK + st * TB, &tmk, &bars->k_full[st], j);
-            k_issued = j - jlo + 1;
-            if (use > 0 && !pf1_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
-                break;
-            issue(sV + st * TB, &tmv, &bars->v_full[st], j);
-            v_issued = j - jlo + 1;
+                tma_load_4d(ring + st * TB + half * 16384 + s16 * 2048, map, smem_u32(&full[st]),
+                            half * 64, key & (a.bs - 1), kvh, id);
+            issued = j - jlo + 1;
         }
         if (bars->abort && lane == 0) {  // let copies already in flight land
-            mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
-            for (int j = max(0, k_issued - kPfStages); j < k_issued; ++j)
-                mbar_wait(smem_u32(&bars->k_full[j % kPfStages]), (j / kPfStages) & 1,
-                          a.timeout_ns);
-            for (int j = max(0, v_issued - kPfStages); j < v_issued; ++j)
-                mbar_wait(smem_u32(&bars->v_full[j % kPfStages]), (j / kPfStages) & 1,
-                          a.timeout_ns);
+            if (is_k) mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
+            for (int j = max(0, issued - NSt); j < issued; ++j)
+                mbar_wait(smem_u32(&full[j % NSt]), (j / NSt) & 1, a.timeout_ns);
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA
@@ -847,9 +910,8 @@ __global__ void __launch_bounds__(kP1Threads, 1)
             constexpr uint32_t kIdQK = f16_idesc(128, kPfKeys, false);
             constexpr uint32_t kIdPV = f16_idesc(128, D, true);
             auto issue_s = [&](int u) -> bool {  // S(u) = Q K(u)^T into buffer (u - jlo) & 1
-                const int st = (u - jlo) % kPfStages;
-                if (!pf1_wait(bars, &bars->k_full[st], ((u - jlo) / kPfStages) & 1, a.timeout_ns,
-                              false))
+                const int st = (u - jlo) % KS;
+                if (!pf1_wait(bars, &bars->k_full[st], ((u - jlo) / KS) & 1, a.timeout_ns, false))
                     return false;
                 tc_fence_after();
                 const uint32_t k = sK + st * TB;
@@ -865,11 +927,10 @@ __global__ void __launch_bounds__(kP1Threads, 1)
                 return true;
             };
             auto issue_pv = [&](int u) -> bool {  // O += P(u) V(u)
-                const int st = (u - jlo) % kPfStages, b = (u - jlo) & 1;
+                const int st = (u - jlo) % VS, b = (u - jlo) & 1;
                 if (!pf1_wait(bars, &bars->p_full[b], ((u - jlo) >> 1) & 1, a.timeout_ns, false))
                     return false;
-                if (!pf1_wait(bars, &bars->v_full[st], ((u - jlo) / kPfStages) & 1, a.timeout_ns,
-                              false))
+                if (!pf1_wait(bars, &bars->v_full[st], ((u - jlo) / VS) & 1, a.timeout_ns, false))
                     return false;
                 tc_fence_after();
                 const uint32_t v = sV + st * TB;
@@ -982,7 +1043,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
                     const float p1 = k0 + 1 <= pos && (!WIN || k0 + 1 >= lo)
                                          ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m)) : 0.f;
                     ls[e & 3] += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
+                    pk[e] = pack_bf16x2_int(p0, p1);
                 }
             } else {
                 // scale and shift as one packed f32x2 FMA per key pair, the
@@ -994,9 +1055,17 @@ __global__ void __launch_bounds__(kP1Threads, 1)
                     const float2 t = __ffma2_rn(
                         make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2v,
                         nmv);
-                    const float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
+                    float p0, p1;
+                    if (kPfPolyEvery > 0 && e % (kPfPolyEvery > 0 ? kPfPolyEvery : 1) == 0) {
+                        const float2 pp = ex2_poly2(t);
+                        p0 = pp.x;
+                        p1 = pp.y;
+                    } else {
+                        p0 = ex2_approx(t.x);
+                        p1 = ex2_approx(t.y);
+                    }
                     acc2[e & 1] = __fadd2_rn(acc2[e & 1], make_float2(p0, p1));
-                    pk[e] = pack_bf16x2(p0, p1);
+                    pk[e] = pack_bf16x2_int(p0, p1);
                 }
                 ls[0] = acc2[0].x;
                 ls[1] = acc2[0].y;
@@ -1032,8 +1101,8 @@ __global__ void __launch_bounds__(kP1Threads, 1)
             const int z0 = WIN ? max(0, min(kPfKeys, chunk_lo - key0)) : 0;
             const int z1 = min(kPfKeys, max(0, ctx - key0));
             if (z0 > 0 || z1 < kPfKeys) {
-                const int st = (u - jlo) % kPfStages;
-                if (!pf1_wait(bars, &bars->v_full[st], ((u - jlo) / kPfStages) & 1, a.timeout_ns,
+                const int st = (u - jlo) % VS;
+                if (!pf1_wait(bars, &bars->v_full[st], ((u - jlo) / VS) & 1, a.timeout_ns,
                               true)) {
                     ok = false;
                     break;

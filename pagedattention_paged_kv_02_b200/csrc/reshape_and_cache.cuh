@@ -6,10 +6,11 @@
 // rows into the slot the block manager assigned it: physical block
 // slot / block_size, offset slot % block_size.
 //
-// One thread moves one 16-byte vector of K and the matching vector of V:
-// blockIdx.y walks the tokens, blockIdx.x/threadIdx.x the vectors of a token
-// (num_kv_heads rows of head_dim*elem bytes), so reads of key/value are fully
-// coalesced and each (token, kv head) row lands contiguously in its page.
+// A thread moves one 16-byte vector of K and the matching vector of V for
+// each of a few tokens: blockIdx.y walks groups of tokens, blockIdx.x /
+// threadIdx.x the vectors of a token (num_kv_heads rows of head_dim*elem
+// bytes), so reads of key/value are fully coalesced and each (token, kv head)
+// row lands contiguously in its page.
 // Row length and block size are powers of two: positions are shifts and
 // masks, no integer division. Memory-bound: 2 * num_tokens * num_kv_heads *
 // head_dim * elem bytes read and written.
@@ -20,6 +21,7 @@
 namespace pa {
 
 constexpr int kScatterThreads = 128;
+constexpr int kScatterTokens = 4;  // tokens a thread moves per pass
 
 struct ReshapeArgs {
     const uint4 *key;
@@ -35,28 +37,45 @@ struct ReshapeArgs {
     long long num_slots;  // num_blocks * block_size
 };
 
+// Each thread moves one 16-byte vector of K and of V for kScatterTokens
+// tokens (blockIdx.y walks groups of tokens): it loads all their slots and
+// rows first, so the slot lookups and the row reads are in flight together,
+// then stores the rows whose slots are valid.
 __global__ void __launch_bounds__(kScatterThreads)
     reshape_and_cache_kernel(const __grid_constant__ ReshapeArgs a) {
     const int r = blockIdx.x * kScatterThreads + threadIdx.x;  // vector within the token
     if (r >= a.vecs_per_token) return;
     const int h = r >> a.row_shift;
     const int c = r & ((1 << a.row_shift) - 1);
-    for (long long t = blockIdx.y; t < a.num_tokens; t += gridDim.y) {
-        const long long slot = __ldg(a.slot_mapping + t);
-        if (slot < 0) continue;  // padding token
-        if (slot >= a.num_slots) {
-            flag_error(PA_ERR_BAD_TABLE);
-            continue;
+    for (long long t0 = (long long)blockIdx.y * kScatterTokens; t0 < a.num_tokens;
+         t0 += (long long)gridDim.y * kScatterTokens) {
+        long long slot[kScatterTokens];
+        uint4 kv[kScatterTokens], vv[kScatterTokens];
+#pragma unroll
+        for (int u = 0; u < kScatterTokens; ++u) {
+            const long long t = t0 + u;
+            slot[u] = -1;
+            if (t < a.num_tokens) {
+                slot[u] = __ldg(a.slot_mapping + t);
+                const long long i = t * a.vecs_per_token + r;
+                kv[u] = __ldg(a.key + i);
+                vv[u] = __ldg(a.value + i);
+            }
         }
-        const long long block = slot >> a.bs_shift;
-        const long long offset = slot & ((1LL << a.bs_shift) - 1);
-        const long long dst =
-            (((block * a.num_kv_heads + h) << a.bs_shift) + offset) * (1LL << a.row_shift) + c;
-        const long long i = t * a.vecs_per_token + r;
-        const uint4 kv = __ldg(a.key + i);
-        const uint4 vv = __ldg(a.value + i);
-        a.k_cache[dst] = kv;
-        a.v_cache[dst] = vv;
+#pragma unroll
+        for (int u = 0; u < kScatterTokens; ++u) {
+            if (slot[u] < 0) continue;  // padding token (or past the end)
+            if (slot[u] >= a.num_slots) {
+                flag_error(PA_ERR_BAD_TABLE);
+                continue;
+            }
+            const long long block = slot[u] >> a.bs_shift;
+            const long long offset = slot[u] & ((1LL << a.bs_shift) - 1);
+            const long long dst =
+                (((block * a.num_kv_heads + h) << a.bs_shift) + offset) * (1LL << a.row_shift) + c;
+            a.k_cache[dst] = kv[u];
+            a.v_cache[dst] = vv[u];
+        }
     }
 }
 

@@ -147,7 +147,7 @@ def test_prefill_host_checks(L):
     # the grid is (query head, query tile, chunk): at most 65535 tiles of 128 queries
     # and 65535 chunks; any number of query heads
     b = list(base)
-    b[8], b[9] = 65535 * 128 + 1, 65535 * 128 + 1
+    b[8], b[9] = 65536 * 256, 65536 * 256
     assert f(*b) == pa.PA_ERR_UNSUPPORTED
     b = list(base)
     b[7] = 65536

@@ -259,9 +259,10 @@ def test_model_catches_a_missing_wait():
 # ---------------------------------------------------------------------------
 # The one-query-tile form (prefill_1q_kernel): one 128-row query tile per
 # CTA, S double-buffered (S(u+2) issued behind P.V(u) into the buffer it
-# freed), K tile u freed once S(u) completes and V tile u once P.V(u) does,
-# one o_full barrier per S buffer, the softmax waiting on o_full only to
-# rescale O and in the epilogue.
+# freed), K and V streamed by two warps into rings of their own depths, K
+# tile u freed once S(u) completes and V tile u once P.V(u) does, one o_full
+# barrier per S buffer, the softmax waiting on o_full only to rescale O and
+# in the epilogue.
 
 
 def geometry_1q(C, cached, row0, W):
@@ -273,18 +274,23 @@ def geometry_1q(C, cached, row0, W):
     return (lo, hi), chunk_lo, cached + C
 
 
+K1_STAGES, V1_STAGES = 3, 2  # the one-query-tile kernel's ring depths
+
+
 def run_1q(C, cached, row0, W, seed, rescale_p=0.3, zeroing=True, o_per_buffer=True,
            free_k_early=False):
     rnd = random.Random(seed)
     (jlo, jhi), chunk_lo, ctx = geometry_1q(C, cached, row0, W)
-    stage = lambda j: (j - jlo) % STAGES
-    use = lambda j: (j - jlo) // STAGES
+    kstage = lambda j: (j - jlo) % K1_STAGES
+    kuse = lambda j: (j - jlo) // K1_STAGES
+    vstage = lambda j: (j - jlo) % V1_STAGES
+    vuse = lambda j: (j - jlo) // V1_STAGES
     buf = lambda u: (u - jlo) % 2
     nth = lambda u: (u - jlo) // 2
     zero_needed = {u for u in range(jlo, jhi)
                    if KEYS * (u + 1) > ctx or (W > 0 and KEYS * u < chunk_lo)}
-    names = ["q_full", "fin"] + [f"{k}{s}" for k in ("k_full", "k_free", "v_full", "v_free")
-                                 for s in range(STAGES)]
+    names = ["q_full", "fin"] + [f"{k}{s}" for k in ("k_full", "k_free") for s in range(K1_STAGES)]
+    names += [f"{k}{s}" for k in ("v_full", "v_free") for s in range(V1_STAGES)]
     names += [f"{k}{b}" for k in ("s_full", "p_full") for b in (0, 1)]  # p_full: 128 arrivals
     names += [f"o_full{b}" for b in (0, 1)] if o_per_buffer else ["o_full"]
     B = {n: Bar(n) for n in names}
@@ -296,21 +302,25 @@ def run_1q(C, cached, row0, W, seed, rescale_p=0.3, zeroing=True, o_per_buffer=T
     pipe, done, inflight = [], set(), []
     st = {"K": {}, "V": {}, "q": False, "S": {}, "zeroed": set()}
 
-    def tma():
+    def tma_k():  # the K warp (it also loads Q)
         inflight.append(("q_full", "Q", None))
         yield
         for j in range(jlo, jhi):
-            s, u = stage(j), use(j)
+            s, u = kstage(j), kuse(j)
             if u > 0:
                 while not B[f"k_free{s}"].ready(u - 1):
                     yield
-                assert ("S", j - STAGES) in done, "K stage reloaded under S"
+                assert ("S", j - K1_STAGES) in done, "K stage reloaded under S"
             inflight.append((f"k_full{s}", "K", j))
             yield
+
+    def tma_v():  # the V warp
+        for j in range(jlo, jhi):
+            s, u = vstage(j), vuse(j)
             if u > 0:
                 while not B[f"v_free{s}"].ready(u - 1):
                     yield
-                assert ("PV", j - STAGES) in done, "V stage reloaded under P.V"
+                assert ("PV", j - V1_STAGES) in done, "V stage reloaded under P.V"
             inflight.append((f"v_full{s}", "V", j))
             yield
 
@@ -319,26 +329,26 @@ def run_1q(C, cached, row0, W, seed, rescale_p=0.3, zeroing=True, o_per_buffer=T
             yield
 
         def issue_s(u):
-            while not B[f"k_full{stage(u)}"].ready(use(u)):
+            while not B[f"k_full{kstage(u)}"].ready(kuse(u)):
                 yield
-            assert st["K"].get(stage(u)) == u
+            assert st["K"].get(kstage(u)) == u
             if free_k_early:  # planted: the stage released before S is queued
-                pipe.append(("commit", f"k_free{stage(u)}"))
+                pipe.append(("commit", f"k_free{kstage(u)}"))
             pipe.append(("S", u))
             pipe.append(("commit", f"s_full{buf(u)}"))
             if not free_k_early:
-                pipe.append(("commit", f"k_free{stage(u)}"))
+                pipe.append(("commit", f"k_free{kstage(u)}"))
             yield
 
         def issue_pv(u):
             while not B[f"p_full{buf(u)}"].ready(nth(u)):
                 yield
-            while not B[f"v_full{stage(u)}"].ready(use(u)):
+            while not B[f"v_full{vstage(u)}"].ready(vuse(u)):
                 yield
-            assert st["V"].get(stage(u)) == u
+            assert st["V"].get(vstage(u)) == u
             pipe.append(("PV", u))
             pipe.append(("commit", o_bar(u)[0]))
-            pipe.append(("commit", f"v_free{stage(u)}"))
+            pipe.append(("commit", f"v_free{vstage(u)}"))
             yield
 
         for t in range(jlo - 2, jhi):
@@ -365,7 +375,7 @@ def run_1q(C, cached, row0, W, seed, rescale_p=0.3, zeroing=True, o_per_buffer=T
                 assert ("PV", u - 1) in done, "rescale before the previous P.V completed"
                 assert not any(op[0] == "PV" for op in pipe), "rescale under a queued P.V"
             if zeroing and u in zero_needed:
-                while not B[f"v_full{stage(u)}"].ready(use(u)):
+                while not B[f"v_full{vstage(u)}"].ready(vuse(u)):
                     yield
                 st["zeroed"].add(u)
             B[f"p_full{b}"].arrive()
@@ -385,7 +395,7 @@ def run_1q(C, cached, row0, W, seed, rescale_p=0.3, zeroing=True, o_per_buffer=T
         assert st["q"], "MMA before Q landed"
         b = buf(u)
         if kind == "S":
-            assert st["K"].get(stage(u)) == u, f"S of tile {u} reads a reloaded K stage"
+            assert st["K"].get(kstage(u)) == u, f"S of tile {u} reads a reloaded K stage"
             cur = st["S"].get(b)
             assert cur is None or cur[0] == "P" and ("PV", cur[1]) in done, \
                 f"S of tile {u} over an unread tile {cur}"
@@ -395,18 +405,19 @@ def run_1q(C, cached, row0, W, seed, rescale_p=0.3, zeroing=True, o_per_buffer=T
             assert u not in zero_needed or u in st["zeroed"], f"P.V of tile {u} reads unzeroed V rows"
         done.add((kind, u))
 
-    roles = {"tma": tma(), "mma": mma(), "sm": softmax()}
+    roles = {"tma_k": tma_k(), "tma_v": tma_v(), "mma": mma(), "sm": softmax()}
     steps = 0
     while roles or pipe or inflight:
         choice = rnd.choice(list(roles) + ["pipe"] * bool(pipe) + ["copy"] * bool(inflight))
         if choice == "pipe":
             pipe_step()
         elif choice == "copy":
-            bar, kind, j = inflight.pop(0)
+            # copies land in any order (each has its own barrier)
+            bar, kind, j = inflight.pop(rnd.randrange(len(inflight)))
             if kind == "Q":
                 st["q"] = True
             else:
-                st[kind][stage(j)] = j
+                st[kind][kstage(j) if kind == "K" else vstage(j)] = j
             B[bar].arrive()
         else:
             try:
