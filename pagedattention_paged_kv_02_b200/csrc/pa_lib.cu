@@ -132,22 +132,12 @@ pa_status launch_decode_f32(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
     return launch_status();
 }
 
-#ifndef PA_PREFILL_1Q
-#define PA_PREFILL_1Q 0
-#endif
-
 // query rows one prefill CTA covers
-constexpr int kPrefillCtaRows = PA_PREFILL_1Q ? kPfRows : kPfRows * kPfQTiles;
+constexpr int kPrefillCtaRows = kPfRows * kPfQTiles;
 
 template <int D, bool WIN>
 pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                             const CUtensorMap &mv, dim3 grid, cudaStream_t st) {
-#if PA_PREFILL_1Q
-    const size_t smem = 1024 + pf1_smem_bytes(D);
-    auto k = prefill_1q_kernel<D, WIN>;
-    if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
-    k<<<grid, kP1Threads, smem, st>>>(a, mq, mk, mv);
-#else
     const size_t smem = 1024 + pf_smem_bytes(D);
     auto k = prefill_tc_kernel<D, WIN>;
     if (set_smem(k, smem) != cudaSuccess) return PA_ERR_CUDA;
@@ -157,7 +147,6 @@ pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const C
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return PA_ERR_CUDA;
     if ((long long)fa.numRegs * kPfThreads < kPfRegsNeeded) return PA_ERR_UNSUPPORTED;
     k<<<grid, kPfThreads, smem, st>>>(a, mq, mk, mv);
-#endif
     return launch_status();
 }
 

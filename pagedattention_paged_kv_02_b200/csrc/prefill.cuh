@@ -60,12 +60,6 @@ constexpr int kPfCtlRegs = 56;
 constexpr int kPfSoftmaxRegs = 224;
 constexpr int kPfRegsNeeded = 128 * (2 * kPfSoftmaxRegs + kPfCtlRegs);
 constexpr int kPfTblMax = 4096;   // block-table entries staged in shared memory
-#ifndef PA_PREFILL_POLY_EVERY
-#define PA_PREFILL_POLY_EVERY 0
-#endif
-// every kPfPolyEvery-th pair of exponentials of an unmasked tile on the FMA
-// pipe (ex2_poly2), the rest on the special-function unit; 0: none
-constexpr int kPfPolyEvery = PA_PREFILL_POLY_EVERY;
 // A Q, K or V tile: 128 rows of head_dim bf16, as head_dim/64 halves of 128 x
 // 128 bytes (one 128-byte swizzle atom wide), each 16 KB.
 __host__ __device__ constexpr int pf_tile_bytes(int D) { return kPfRows * D * 2; }
@@ -221,45 +215,10 @@ __device__ __forceinline__ bool pf_wait(PfBars *bars, uint64_t *bar, uint32_t pa
     return ok;
 }
 
-// Two non-negative finite fp32 values -> a bf16 pair (lo in the low half),
-// rounded to nearest on the integer pipe: half a bf16 ulp added to the fp32
-// bits, the upper halves kept (a tie, low half exactly 0x8000, rounds away
-// from zero instead of to even). The softmax's conversion instruction would
-// otherwise share the special-function pipe with its exponentials.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-#if !defined(PA_PREFILL_PACK_CVT) || PA_PREFILL_PACK_CVT
-    return pack_bf16x2(lo, hi);
-#else
-    return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-#endif
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x for a pair of values on the FMA pipe (packed f32x2), so that part of
-// the softmax's exponentials leave the special-function pipe. Cody-Waite
-// style: x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low
-// mantissa bits) and |f| <= 1/2; 2^f by a cubic whose coefficients were
-// fitted for minimum maximum relative error on [-1/2, 1/2] (1.02e-4, exact at
-// f = 0: below the bf16 rounding of the weights); 2^n is added to the
-// exponent field. Inputs below -125 give 2^-125.
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 magic = make_float2(12582912.f, 12582912.f);
-    const float2 t = __fadd2_rn(x, magic);
-    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-    float2 p = __ffma2_rn(make_float2(0.05500824f, 0.05500824f), f,
-                          make_float2(0.24220951f, 0.24220951f));
-    p = __ffma2_rn(p, f, make_float2(0.69328284f, 0.69328284f));
-    p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
-    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // WIN: the sliding-window build; without it the band logic folds away at
@@ -386,12 +345,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
     if (warp >= 8) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfCtlRegs));
-#ifndef PA_PREFILL_SPLIT_KV
-#define PA_PREFILL_SPLIT_KV 0
-#endif
-      // K and V streamed by warps 8 and 10 (SPLIT_KV), or both by warp 8
-      if (warp == 8 || (PA_PREFILL_SPLIT_KV && warp == 10)) {
-        const bool do_k = warp == 8, do_v = !PA_PREFILL_SPLIT_KV || warp == 10;
+      if (warp == 8) {
         // ------------------------------------------------------------ TMA
         // One box per lane: a thread issuing tensor copies back to back is
         // slow (each issue takes a while to be accepted), so the 16 boxes
@@ -425,23 +379,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int j = jmin; j < jmax; ++j) {
             const int st = (j - jmin) % kPfStages;
             const uint32_t use = (j - jmin) / kPfStages;
-            if (do_k) {
-                if (use > 0 &&
-                    !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
-                    break;
-                issue(sK + st * TB, &tmk, &bars->k_full[st], j);
-                k_issued = j - jmin + 1;
-            }
-            if (do_v) {
-                if (use > 0 &&
-                    !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
-                    break;
-                issue(sV + st * TB, &tmv, &bars->v_full[st], j);
-                v_issued = j - jmin + 1;
-            }
+            if (use > 0 && !pf_wait(bars, &bars->k_free[st], (use - 1) & 1, a.timeout_ns, true))
+                break;
+            issue(sK + st * TB, &tmk, &bars->k_full[st], j);
+            k_issued = j - jmin + 1;
+            if (use > 0 && !pf_wait(bars, &bars->v_free[st], (use - 1) & 1, a.timeout_ns, true))
+                break;
+            issue(sV + st * TB, &tmv, &bars->v_full[st], j);
+            v_issued = j - jmin + 1;
         }
         if (bars->abort && lane == 0) {  // let copies already in flight land
-            if (do_k) mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
+            mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
             for (int j = max(0, k_issued - kPfStages); j < k_issued; ++j)
                 mbar_wait(smem_u32(&bars->k_full[j % kPfStages]), (j / kPfStages) & 1,
                           a.timeout_ns);
@@ -613,7 +561,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const float p1 = k0 + 1 <= pos && (!WIN || k0 + 1 >= lo)
                                          ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m)) : 0.f;
                     ls[e & 3] += p0 + p1;
-                    pk[e] = pack_bf16x2_int(p0, p1);
+                    pk[e] = pack_bf16x2(p0, p1);
                 }
             } else {
                 // scale and shift as one packed f32x2 FMA per key pair, the
@@ -626,17 +574,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const float2 t = __ffma2_rn(
                         make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2v,
                         nmv);
-                    float p0, p1;
-                    if (kPfPolyEvery > 0 && e % (kPfPolyEvery > 0 ? kPfPolyEvery : 1) == 0) {
-                        const float2 pp = ex2_poly2(t);
-                        p0 = pp.x;
-                        p1 = pp.y;
-                    } else {
-                        p0 = ex2_approx(t.x);
-                        p1 = ex2_approx(t.y);
-                    }
+                    const float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
                     acc2[e & 1] = __fadd2_rn(acc2[e & 1], make_float2(p0, p1));
-                    pk[e] = pack_bf16x2_int(p0, p1);
+                    pk[e] = pack_bf16x2(p0, p1);
                 }
                 ls[0] = acc2[0].x;
                 ls[1] = acc2[0].y;
@@ -700,457 +640,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 9) {
-        __syncwarp();
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// The same computation with one 128-row query tile per CTA and its S
-// double-buffered: S_b (b = 0, 1) in tensor-memory columns [128b, 128b+128)
-// (P, bf16 pairs, over the first 64 of its buffer), O in [256, 256+D). The
-// MMA thread issues, per key tile u, O += P(u) V(u) and then S(u+2) into the
-// buffer P(u) just left, so S(u+1) is already computed while the softmax of
-// tile u runs: the softmax never waits for its own P.V and the next S (the
-// chain S -> softmax -> P.V -> S that bounds the two-tile form above). The
-// price is a K/V tile per 128 query rows instead of per 256: twice the
-// L2-to-SM bytes per FLOP.
-//
-// Barriers per S buffer b: s_full (S landed), p_full (P written, 128
-// arrivals), o_full (the P.V that read buffer b completed). With o_full per
-// buffer, any completion the softmax can ask for is within one phase of the
-// barrier (S(u) landing implies P.V(u-2) completed), so the softmax waits on
-// it only when it must rescale O, and in the epilogue.
-constexpr int kP1Threads = 224;  // softmax warpgroup, K warp, MMA warp, V warp
-// ring depths: a K tile is freed when its S completes and is needed two
-// tiles ahead of the softmax, a V tile when its P.V completes; K and V are
-// streamed by warps of their own, so neither load waits behind the other
-constexpr int kP1KStages = 3;
-constexpr int kP1VStages = 2;
-
-struct Pf1Bars {
-    uint64_t q_full;
-    uint64_t k_full[kP1KStages], k_free[kP1KStages], v_full[kP1VStages], v_free[kP1VStages];
-    uint64_t s_full[2], p_full[2], o_full[2];
-    uint64_t fin;
-    uint32_t tmem_base;
-    volatile int abort;
-};
-static_assert(sizeof(Pf1Bars) <= 512, "barriers fit their slot");
-
-__host__ __device__ constexpr int pf1_smem_bytes(int D) {
-    return (1 + kP1KStages + kP1VStages) * pf_tile_bytes(D) + 512 + kPfTblMax * 4;
-}
-
-__device__ __forceinline__ bool pf1_wait(Pf1Bars *bars, uint64_t *bar, uint32_t parity,
-                                         unsigned long long timeout_ns, bool uniform) {
-    bool ok = bars->abort == 0 && mbar_wait(smem_u32(bar), parity, timeout_ns);
-    if (uniform) ok = __all_sync(0xffffffffu, ok);
-    if (!ok && bars->abort == 0) {
-        bars->abort = 1;
-        flag_error(PA_ERR_TIMEOUT);
-    }
-    return ok;
-}
-
-template <int D, bool WIN>
-__global__ void __launch_bounds__(kP1Threads, 1)
-    prefill_1q_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
-                      const __grid_constant__ CUtensorMap tmk,
-                      const __grid_constant__ CUtensorMap tmv) {
-    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-    constexpr int TB = pf_tile_bytes(D);
-    constexpr int HALVES = D / 64;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
-    constexpr int KS = kP1KStages, VS = kP1VStages;
-    const uint32_t sQ = smem_u32(smem);            // the Q tile
-    const uint32_t sK = sQ + TB;                   // K stage st at sK + st*TB
-    const uint32_t sV = sK + KS * TB;              // V stage st at sV + st*TB
-    Pf1Bars *bars = reinterpret_cast<Pf1Bars *>(smem + (1 + KS + VS) * TB);
-    int32_t *tbl = reinterpret_cast<int32_t *>(smem + (1 + KS + VS) * TB + 512);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // CTAs start in order of decreasing work: the last chunk first, within it
-    // the last query tile first, every query head of a tile together
-    const int h = blockIdx.x;
-    const int tq = (int)gridDim.y - 1 - (int)blockIdx.y;
-    const int c = a.n_chunks - 1 - (int)blockIdx.z;
-    const int q0 = a.qsl[c];
-    const int C = a.qsl[c + 1] - q0;
-    const int ctx = a.context_lens[c];
-    // the chunk is checked before any CTA leaves for lack of rows, so that a
-    // malformed chunk is recorded even when it has no rows at all
-    if (q0 < 0 || C < 0 || q0 + C > a.total_q || ctx < C || (long long)ctx > (long long)a.MB * a.bs) {
-        if (threadIdx.x == 0) flag_error(PA_ERR_BAD_TABLE);
-        return;
-    }
-    // rows past the grid's reach (a chunk longer than max_query_len rounded
-    // up to the CTA's rows) would be left unwritten: recorded once per chunk
-    if (C > (int)gridDim.y * kPfRows && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
-        flag_error(PA_ERR_BAD_TABLE);
-    const int row0 = tq * kPfRows;  // first query of this CTA within the chunk
-    if (row0 >= C) return;
-    const int cached = ctx - C;
-    // The key tiles [jlo, jhi) the query tile needs: up to its last row's
-    // position, from its first row's band start. Key positions below the
-    // chunk's smallest band start (chunk_lo) are never needed: their blocks
-    // may have been freed.
-    const int rows = min(kPfRows, C - row0);
-    const int W = WIN ? a.window : 0;
-    const int chunk_lo = W > 0 ? max(0, cached - W + 1) : 0;
-    const int pos_first = cached + row0;
-    const int jlo = (W > 0 ? max(0, pos_first - W + 1) : 0) / kPfKeys;
-    const int jhi = (pos_first + rows - 1) / kPfKeys + 1;
-    const int kvh = h / a.group;
-
-    if (warp == 4) {
-      if (lane == 0) {
-        mbar_init(smem_u32(&bars->q_full), 1);
-        for (int st = 0; st < KS; ++st) {
-            mbar_init(smem_u32(&bars->k_full[st]), 1);
-            mbar_init(smem_u32(&bars->k_free[st]), 1);
-        }
-        for (int st = 0; st < VS; ++st) {
-            mbar_init(smem_u32(&bars->v_full[st]), 1);
-            mbar_init(smem_u32(&bars->v_free[st]), 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&bars->s_full[b]), 1);
-            mbar_init(smem_u32(&bars->p_full[b]), 128);
-            mbar_init(smem_u32(&bars->o_full[b]), 1);
-        }
-        mbar_init(smem_u32(&bars->fin), 1);
-        bars->abort = 0;
-        fence_mbar_init();
-      }
-      __syncwarp();
-      // the Q tile needs no table: its copy overlaps the table staging below
-      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars->q_full), TB);
-      __syncwarp();
-      if (lane < HALVES)
-          tma_load_3d(sQ + lane * 16384, &tmq, smem_u32(&bars->q_full), lane * 64, h, q0 + row0);
-    }
-    if (warp == 5) {
-        tmem_alloc(smem_u32(&bars->tmem_base), 512);
-        tmem_relinquish();
-    }
-    // the block-table slice this CTA streams, from its first key tile's
-    // block, checked once, into shared memory (kPfTblMax entries; a longer
-    // span reads the rest from global). Blocks wholly before chunk_lo are
-    // neither read nor checked.
-    const int n_blk = (ctx + a.bs - 1) / a.bs;
-    const int blk0 = jlo * kPfKeys / a.bs, blk_lo = chunk_lo / a.bs;
-    const int32_t *trow = a.block_tables + (size_t)c * a.MB;
-    for (int e = threadIdx.x; e < min(n_blk - blk0, kPfTblMax); e += kP1Threads) {
-        int id = -1;
-        if (blk0 + e >= blk_lo) {
-            id = __ldg(trow + blk0 + e);
-            if (id < 0 || id >= a.NB) {
-                flag_error(PA_ERR_BAD_TABLE);
-                id = -1;
-            }
-        }
-        tbl[e] = id;
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = bars->tmem_base;
-
-    if (warp == 4 || warp == 6) {
-        // ----------------------------------------------------- TMA (K, V)
-        // warp 4 streams K, warp 6 V, each into its own ring; one 16-token
-        // x 64-dim box per lane (16 lanes per tile); lane 0 arms the
-        // barrier with the bytes of the pieces that exist
-        const bool is_k = warp == 4;
-        const int NSt = is_k ? KS : VS;
-        const CUtensorMap *map = is_k ? &tmk : &tmv;
-        uint64_t *full = is_k ? bars->k_full : bars->v_full;
-        uint64_t *freeb = is_k ? bars->k_free : bars->v_free;
-        const uint32_t ring = is_k ? sK : sV;
-        const int s16 = lane / HALVES, half = lane % HALVES;
-        int issued = 0;  // tiles issued, counted from jlo
-        for (int j = jlo; j < jhi; ++j) {
-            const int st = (j - jlo) % NSt;
-            const uint32_t use = (j - jlo) / NSt;
-            if (use > 0 && !pf1_wait(bars, &freeb[st], (use - 1) & 1, a.timeout_ns, true)) break;
-            const int key = j * kPfKeys + s16 * 16;
-            int id = -1;
-            if (lane < 8 * HALVES && key < ctx && (!WIN || key + 15 >= chunk_lo)) {
-                const int lb = key >> a.bs_shift;
-                if (lb - blk0 < kPfTblMax) {
-                    id = tbl[lb - blk0];
-                } else {
-                    id = __ldg(trow + lb);
-                    if (id < 0 || id >= a.NB) {
-                        flag_error(PA_ERR_BAD_TABLE);
-                        id = -1;
-                    }
-                }
-            }
-            const int n = __popc(__ballot_sync(0xffffffffu, id >= 0));
-            if (lane == 0) mbar_arrive_expect_tx(smem_u32(&full[st]), n * 2048);
-            __syncwarp();
-            if (id >= 0)
-                tma_load_4d(ring + st * TB + half * 16384 + s16 * 2048, map, smem_u32(&full[st]),
-                            half * 64, key & (a.bs - 1), kvh, id);
-            issued = j - jlo + 1;
-        }
-        if (bars->abort && lane == 0) {  // let copies already in flight land
-            if (is_k) mbar_wait(smem_u32(&bars->q_full), 0, a.timeout_ns);
-            for (int j = max(0, issued - NSt); j < issued; ++j)
-                mbar_wait(smem_u32(&full[j % NSt]), (j / NSt) & 1, a.timeout_ns);
-        }
-    } else if (warp == 5) {
-        // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            constexpr uint32_t kIdQK = f16_idesc(128, kPfKeys, false);
-            constexpr uint32_t kIdPV = f16_idesc(128, D, true);
-            auto issue_s = [&](int u) -> bool {  // S(u) = Q K(u)^T into buffer (u - jlo) & 1
-                const int st = (u - jlo) % KS;
-                if (!pf1_wait(bars, &bars->k_full[st], ((u - jlo) / KS) & 1, a.timeout_ns, false))
-                    return false;
-                tc_fence_after();
-                const uint32_t k = sK + st * TB;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_ss(tmem + 128 * ((u - jlo) & 1), sw128_desc(sQ + koff, 16, 1024),
-                           sw128_desc(k + koff, 16, 1024), kIdQK, ks > 0);
-                }
-                tc_commit(smem_u32(&bars->s_full[(u - jlo) & 1]));
-                // S(u) is K tile u's only reader: free its stage on completion
-                tc_commit(smem_u32(&bars->k_free[st]));
-                return true;
-            };
-            auto issue_pv = [&](int u) -> bool {  // O += P(u) V(u)
-                const int st = (u - jlo) % VS, b = (u - jlo) & 1;
-                if (!pf1_wait(bars, &bars->p_full[b], ((u - jlo) >> 1) & 1, a.timeout_ns, false))
-                    return false;
-                if (!pf1_wait(bars, &bars->v_full[st], ((u - jlo) / VS) & 1, a.timeout_ns, false))
-                    return false;
-                tc_fence_after();
-                const uint32_t v = sV + st * TB;
-#pragma unroll
-                for (int ks = 0; ks < kPfKeys / 16; ++ks)
-                    mma_ts(tmem + 256, tmem + 128 * b + ks * 8,
-                           sw128_desc(v + ks * 2048, 16384, 1024), kIdPV,
-                           (u > jlo || ks > 0) ? 1u : 0u);
-                tc_commit(smem_u32(&bars->o_full[b]));
-                tc_commit(smem_u32(&bars->v_free[st]));  // P.V(u) is V tile u's only reader
-                return true;
-            };
-            bool ok = pf1_wait(bars, &bars->q_full, 0, a.timeout_ns, false);
-            // step t: P.V of tile t, then S of tile t+2 into the buffer it
-            // freed; the first two S go out at steps jlo-2 and jlo-1
-            for (int t = jlo - 2; ok && t < jhi; ++t) {
-                if (t >= jlo) ok = issue_pv(t);
-                if (ok && t + 2 < jhi) ok = issue_s(t + 2);
-            }
-            // every tensor-core operation issued above completes before teardown
-            tc_commit(smem_u32(&bars->fin));
-            mbar_wait(smem_u32(&bars->fin), 0, a.timeout_ns);
-        }
-    } else {
-        // -------------------------------------------------------- softmax
-        const int r = threadIdx.x;                    // row of the tile == lane
-        const int i = row0 + r;                       // query index in the chunk
-        const bool row_valid = i < C;
-        const int pos = cached + min(i, C - 1);       // keys <= pos are visible
-        const int lo = W > 0 ? pos - W + 1 : 0;       // ... and keys >= lo
-        const int lo_last = W > 0 ? pos_first + rows - W : 0;  // largest lo of the tile
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t tO = tmem + 256 + lane_off;
-        const float sl2 = a.scale_log2;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int u = jlo; u < jhi; ++u) {
-            const int b = (u - jlo) & 1;
-            if (!pf1_wait(bars, &bars->s_full[b], ((u - jlo) >> 1) & 1, a.timeout_ns, true)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t tS = tmem + 128 * b + lane_off;
-            uint32_t sv[128];
-            tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
-            tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
-            tmem_ld_wait();
-            const int key0 = u * kPfKeys;
-            // some key masked for some row: past the first row's position,
-            // or before the last row's band start
-            const bool diag = key0 + kPfKeys - 1 > pos_first || (WIN && key0 < lo_last);
-            if (diag) {
-#pragma unroll
-                for (int e = 0; e < 128; ++e)
-                    if (key0 + e > pos || (WIN && key0 + e < lo))
-                        sv[e] = __float_as_uint(sl2 >= 0.f ? -INFINITY : INFINITY);
-            }
-            // the row's largest scaled score (raw max, or raw min for a
-            // negative scale): eight independent running extrema, then a tree
-            float ext;
-            {
-                float t8[8];
-#pragma unroll
-                for (int w = 0; w < 8; ++w) t8[w] = __uint_as_float(sv[w]);
-                if (sl2 >= 0.f) {
-#pragma unroll
-                    for (int e = 8; e < 128; ++e) t8[e & 7] = fmaxf(t8[e & 7], __uint_as_float(sv[e]));
-#pragma unroll
-                    for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                        for (int v = 0; v < w; ++v) t8[v] = fmaxf(t8[v], t8[v + w]);
-                } else {
-#pragma unroll
-                    for (int e = 8; e < 128; ++e) t8[e & 7] = fminf(t8[e & 7], __uint_as_float(sv[e]));
-#pragma unroll
-                    for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                        for (int v = 0; v < w; ++v) t8[v] = fminf(t8[v], t8[v + w]);
-                }
-                ext = t8[0];
-            }
-            const float m_tile = isinf(ext) ? -INFINITY : ext * sl2;
-            const float m_new = fmaxf(m, m_tile);
-            // O and the sum are re-referenced to a new max only when it grew
-            // by more than 2^8 for some row of the warp (exact for any
-            // reference as long as O and the sum share it); O itself is
-            // rescaled after P is stored, when the scores are dead
-            bool rescale = false;
-            float corr = 1.f;
-            if (u == jlo) {
-                m = m_new;
-            } else if (__any_sync(0xffffffffu, m_new > m + 8.f)) {
-                // a row that has seen no visible key yet has nothing to rescale
-                rescale = true;
-                corr = m == -INFINITY ? 0.f : ex2_approx(m - m_new);
-                m = m_new;
-            }
-            const float neg_m = -m;
-            uint32_t pk[64];
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
-            if (diag) {
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const int k0 = key0 + 2 * e;
-                    const float p0 = k0 <= pos && (!WIN || k0 >= lo)
-                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m)) : 0.f;
-                    const float p1 = k0 + 1 <= pos && (!WIN || k0 + 1 >= lo)
-                                         ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m)) : 0.f;
-                    ls[e & 3] += p0 + p1;
-                    pk[e] = pack_bf16x2_int(p0, p1);
-                }
-            } else {
-                // scale and shift as one packed f32x2 FMA per key pair, the
-                // row sum as packed adds
-                const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(neg_m, neg_m);
-                float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const float2 t = __ffma2_rn(
-                        make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sl2v,
-                        nmv);
-                    float p0, p1;
-                    if (kPfPolyEvery > 0 && e % (kPfPolyEvery > 0 ? kPfPolyEvery : 1) == 0) {
-                        const float2 pp = ex2_poly2(t);
-                        p0 = pp.x;
-                        p1 = pp.y;
-                    } else {
-                        p0 = ex2_approx(t.x);
-                        p1 = ex2_approx(t.y);
-                    }
-                    acc2[e & 1] = __fadd2_rn(acc2[e & 1], make_float2(p0, p1));
-                    pk[e] = pack_bf16x2_int(p0, p1);
-                }
-                ls[0] = acc2[0].x;
-                ls[1] = acc2[0].y;
-                ls[2] = acc2[1].x;
-                ls[3] = acc2[1].y;
-            }
-            l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-            tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-            tmem_st_wait();
-            if (rescale) {
-                // once the P.V of the previous tile (the last one on O) has
-                // completed; this tile's P.V follows the arrival below
-                if (!pf1_wait(bars, &bars->o_full[(u - 1 - jlo) & 1],
-                              ((uint32_t)(u - 1 - jlo) >> 1) & 1, a.timeout_ns, true)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-#pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + cc * 32, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * corr);
-                    tmem_st32(tO + cc * 32, v);
-                }
-                tmem_st_wait();
-            }
-            // V rows past the context, or before chunk_lo, hold stale or
-            // unloaded data: zero them so that P = 0 cannot meet a NaN there
-            const int z0 = WIN ? max(0, min(kPfKeys, chunk_lo - key0)) : 0;
-            const int z1 = min(kPfKeys, max(0, ctx - key0));
-            if (z0 > 0 || z1 < kPfKeys) {
-                const int st = (u - jlo) % VS;
-                if (!pf1_wait(bars, &bars->v_full[st], ((u - jlo) / VS) & 1, a.timeout_ns,
-                              true)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t vb = sV + st * TB;
-                const int nz = z0 + (kPfKeys - z1);  // rows [0, z0) and [z1, 128)
-                for (int e = r; e < nz * (D / 8); e += 128) {  // 16-byte units of a row
-                    const int zr = e / (D / 8), un = e % (D / 8);
-                    const int row = zr < z0 ? zr : z1 + (zr - z0);
-                    const uint32_t addr = vb + (un / 8) * 16384 + row * 128 + (un % 8) * 16;
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0)
-                                 : "memory");
-                }
-                fence_proxy_async_smem();
-            }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bars->p_full[b]));
-        }
-        if (ok && jhi > jlo) {
-            if (pf1_wait(bars, &bars->o_full[(jhi - 1 - jlo) & 1],
-                         ((uint32_t)(jhi - 1 - jlo) >> 1) & 1, a.timeout_ns, true)) {
-                tc_fence_after();
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-                __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + h) * D;
-#pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + cc * 32, v);
-                    tmem_ld_wait();
-                    uint32_t o[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
-                                           __uint_as_float(v[2 * e + 1]) * inv);
-                    if (row_valid) {
-                        uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-                    }
-                }
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 5) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);

@@ -43,27 +43,37 @@ def test_reference_arm_with_window(capsys, monkeypatch):
     assert line["value"] > 0
 
 
-def test_profiled_traffic_follows_the_source_digest(tmp_path, monkeypatch):
+def test_profiled_traffic_follows_the_source_digest_and_workload(tmp_path, monkeypatch):
     """The DRAM bytes of a committed ncu summary are reported only while the
-    kernel source still hashes to the digest recorded beside them."""
+    kernel source still hashes to the digest recorded beside them and the run
+    is on the workload the summary was taken on (the same batch name: head
+    dim, block size and cache type are part of it)."""
     (tmp_path / "profiles").mkdir()
     src = tmp_path / "k.cuh"
     src.write_text("kernel v1\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     digest = bench.source_digest(["k.cuh"])
     (tmp_path / "profiles" / "p.md").write_text(
-        f"# summary\n\n- source-sha256: `{digest}`\n- dram-bytes-per-launch: `123456`\n")
-    assert bench.profiled_traffic("p.md", ["k.cuh"]) == 123456.0
-    assert bench.profiled_traffic("missing.md", ["k.cuh"]) is None
+        f"# summary\n\n- workload: `wl_d128_bs16`\n- source-sha256: `{digest}`\n"
+        "- dram-bytes-per-launch: `123456`\n")
+    assert bench.profiled_traffic("p.md", ["k.cuh"], "wl_d128_bs16") == 123456.0
+    assert bench.profiled_traffic("p.md", ["k.cuh"], "wl_d64_bs16") is None
+    assert bench.profiled_traffic("p.md", ["k.cuh"], None) is None
+    assert bench.profiled_traffic("missing.md", ["k.cuh"], "wl_d128_bs16") is None
     src.write_text("kernel v2\n")
-    assert bench.profiled_traffic("p.md", ["k.cuh"]) is None
+    assert bench.profiled_traffic("p.md", ["k.cuh"], "wl_d128_bs16") is None
+    # a summary without a workload field is never used
+    (tmp_path / "profiles" / "q.md").write_text(
+        f"- source-sha256: `{bench.source_digest(['k.cuh'])}`\n- dram-bytes-per-launch: `7`\n")
+    assert bench.profiled_traffic("q.md", ["k.cuh"], "wl_d128_bs16") is None
 
 
 def test_committed_profiles_carry_a_source_digest():
-    """Every committed kernel summary names the digest of the kernel sources it
-    was taken on and its DRAM bytes per launch; bench reports that traffic
-    only while the digest matches the current sources (a summary taken
-    before a kernel change yields traffic = null, never a stale number)."""
+    """Every committed kernel summary names the workload and the digest of the
+    kernel sources it was taken on and its DRAM bytes per launch; bench
+    reports that traffic only while both match (a summary taken before a
+    kernel change, or on another workload, yields traffic = null, never a
+    stale number)."""
     import glob
     import os
     import re
@@ -72,22 +82,9 @@ def test_committed_profiles_carry_a_source_digest():
         name = os.path.basename(path)
         assert re.search(r"source-sha256: `[0-9a-f]{16}`", text), f"{name}: no digest"
         assert re.search(r"dram-bytes-per-launch: `[0-9]+`", text), f"{name}: no DRAM bytes"
-
-
-def test_stale_profile_reports_no_traffic(tmp_path, monkeypatch):
-    """A summary whose digest does not match the sources gives None."""
-    import os
-    prof = tmp_path / "profiles"
-    prof.mkdir()
-    src = tmp_path / "k.cuh"
-    src.write_text("kernel v1")
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    digest = bench.source_digest(["k.cuh"])
-    (prof / "x.md").write_text(f"- source-sha256: `{digest}`\n- dram-bytes-per-launch: `123`\n")
-    assert bench.profiled_traffic("x.md", ["k.cuh"]) == 123.0
-    src.write_text("kernel v2")
-    assert bench.profiled_traffic("x.md", ["k.cuh"]) is None
-    assert bench.profiled_traffic("missing.md", ["k.cuh"]) is None
+        # a batch name: the workload with its heads, head dim and block size
+        assert re.search(r"workload: `\w+_d(64|128)_bs(16|32|64)\w*`", text), \
+            f"{name}: no workload"
 
 
 def test_unique_bytes_count_shared_prefix_blocks_once():

@@ -67,6 +67,7 @@ class Bar:
 
 
 def run(C, cached, row0, W, seed):
+    """One seeded interleaving of the four roles for one CTA's geometry."""
     rnd = random.Random(seed)
     (r0, r1), chunk_lo, ctx = geometry(C, cached, row0, W)
     ranges = [r0, r1]
@@ -74,10 +75,13 @@ def run(C, cached, row0, W, seed):
     jmin, jmax = r0[0], max(r0[1], r1[1])
     stage = lambda j: (j - jmin) % STAGES
     use = lambda j: (j - jmin) // STAGES
+    # the query tile whose band reaches the last key tile zeroes its tail
+    # rows (the first one in issue order when both do)
     zeroes_tail = [r0[1] == jmax, r1[1] == jmax and not r0[1] == jmax]
 
-    B = {n: Bar(n) for n in ["q_full", "fin"] + [f"{k}{s}" for k in ("k_full", "k_free", "v_full",
-                                                                       "v_free") for s in range(STAGES)]
+    B = {n: Bar(n) for n in ["q_full", "fin"] + [f"{k}{s}" for k in ("k_full", "k_free",
+                                                                    "v_full", "v_free")
+                                                for s in range(STAGES)]
          + [f"{k}{x}" for k in ("s_full", "o_full") for x in (0, 1)]}
     for x in (0, 1):
         B[f"p_full{x}"] = Bar(f"p_full{x}", 1)  # 128 arrivals, modelled as one
@@ -109,6 +113,7 @@ def run(C, cached, row0, W, seed):
             yield
 
     def mma():
+        """The MMA thread: its operations and commits run in issue order."""
         while not B["q_full"].ready(0):
             yield
 
@@ -159,7 +164,10 @@ def run(C, cached, row0, W, seed):
                 assert not any(op[0] == "PV" and op[1] == x for op in pipe), \
                     "rescale under a queued P.V"
             st["S"][x] = ("P", j)
-            if j in st["zero_needed"] and ((j == jmin and x == 0) or (j == j1 - 1 and zeroes_tail[x])):
+            # the first consumer of a tile in issue order zeroes its rows
+            # past the context or before the band
+            if j in st["zero_needed"] and ((j == jmin and x == 0) or
+                                           (j == j1 - 1 and zeroes_tail[x])):
                 while not B[f"v_full{stage(j)}"].ready(use(j)):
                     yield
                 st["zeroed"].add(j)
@@ -184,7 +192,8 @@ def run(C, cached, row0, W, seed):
             st["S"][x] = ("S", j)
         else:
             assert st["S"].get(x) == ("P", j), f"P.V of tile {j} without its P"
-            assert j not in st["zero_needed"] or j in st["zeroed"], f"P.V of tile {j} reads unzeroed V rows"
+            assert j not in st["zero_needed"] or j in st["zeroed"], \
+                f"P.V of tile {j} reads unzeroed V rows"
         done.add((kind, x, j))
 
     roles = {"tma": tma(), "mma": mma(), "sm0": softmax(0), "sm1": softmax(1)}
@@ -206,7 +215,7 @@ def run(C, cached, row0, W, seed):
             except StopIteration:
                 del roles[choice]
         steps += 1
-        assert steps < 200000, f"deadlock: roles {list(roles)} waiting, queue {pipe[:2]}"
+        assert steps < 200000, f"deadlock: roles {list(roles)} waiting, queue {pipe}"
     assert B["fin"].done == 1
 
 
@@ -254,215 +263,3 @@ def test_model_catches_a_missing_wait():
                 run(512, 300, 0, 0, seed)
     finally:
         Bar.ready = old
-
-
-# ---------------------------------------------------------------------------
-# The one-query-tile form (prefill_1q_kernel): one 128-row query tile per
-# CTA, S double-buffered (S(u+2) issued behind P.V(u) into the buffer it
-# freed), K and V streamed by two warps into rings of their own depths, K
-# tile u freed once S(u) completes and V tile u once P.V(u) does, one o_full
-# barrier per S buffer, the softmax waiting on o_full only to rescale O and
-# in the epilogue.
-
-
-def geometry_1q(C, cached, row0, W):
-    rows = min(ROWS, C - row0)
-    first = cached + row0
-    lo = (max(0, first - W + 1) if W > 0 else 0) // KEYS
-    hi = (first + rows - 1) // KEYS + 1
-    chunk_lo = max(0, cached - W + 1) if W > 0 else 0
-    return (lo, hi), chunk_lo, cached + C
-
-
-K1_STAGES, V1_STAGES = 3, 2  # the one-query-tile kernel's ring depths
-
-
-def run_1q(C, cached, row0, W, seed, rescale_p=0.3, zeroing=True, o_per_buffer=True,
-           free_k_early=False):
-    rnd = random.Random(seed)
-    (jlo, jhi), chunk_lo, ctx = geometry_1q(C, cached, row0, W)
-    kstage = lambda j: (j - jlo) % K1_STAGES
-    kuse = lambda j: (j - jlo) // K1_STAGES
-    vstage = lambda j: (j - jlo) % V1_STAGES
-    vuse = lambda j: (j - jlo) // V1_STAGES
-    buf = lambda u: (u - jlo) % 2
-    nth = lambda u: (u - jlo) // 2
-    zero_needed = {u for u in range(jlo, jhi)
-                   if KEYS * (u + 1) > ctx or (W > 0 and KEYS * u < chunk_lo)}
-    names = ["q_full", "fin"] + [f"{k}{s}" for k in ("k_full", "k_free") for s in range(K1_STAGES)]
-    names += [f"{k}{s}" for k in ("v_full", "v_free") for s in range(V1_STAGES)]
-    names += [f"{k}{b}" for k in ("s_full", "p_full") for b in (0, 1)]  # p_full: 128 arrivals
-    names += [f"o_full{b}" for b in (0, 1)] if o_per_buffer else ["o_full"]
-    B = {n: Bar(n) for n in names}
-
-    def o_bar(u):
-        """The barrier and completion number that P.V(u) completes."""
-        return (f"o_full{buf(u)}", nth(u)) if o_per_buffer else ("o_full", u - jlo)
-
-    pipe, done, inflight = [], set(), []
-    st = {"K": {}, "V": {}, "q": False, "S": {}, "zeroed": set()}
-
-    def tma_k():  # the K warp (it also loads Q)
-        inflight.append(("q_full", "Q", None))
-        yield
-        for j in range(jlo, jhi):
-            s, u = kstage(j), kuse(j)
-            if u > 0:
-                while not B[f"k_free{s}"].ready(u - 1):
-                    yield
-                assert ("S", j - K1_STAGES) in done, "K stage reloaded under S"
-            inflight.append((f"k_full{s}", "K", j))
-            yield
-
-    def tma_v():  # the V warp
-        for j in range(jlo, jhi):
-            s, u = vstage(j), vuse(j)
-            if u > 0:
-                while not B[f"v_free{s}"].ready(u - 1):
-                    yield
-                assert ("PV", j - V1_STAGES) in done, "V stage reloaded under P.V"
-            inflight.append((f"v_full{s}", "V", j))
-            yield
-
-    def mma():
-        while not B["q_full"].ready(0):
-            yield
-
-        def issue_s(u):
-            while not B[f"k_full{kstage(u)}"].ready(kuse(u)):
-                yield
-            assert st["K"].get(kstage(u)) == u
-            if free_k_early:  # planted: the stage released before S is queued
-                pipe.append(("commit", f"k_free{kstage(u)}"))
-            pipe.append(("S", u))
-            pipe.append(("commit", f"s_full{buf(u)}"))
-            if not free_k_early:
-                pipe.append(("commit", f"k_free{kstage(u)}"))
-            yield
-
-        def issue_pv(u):
-            while not B[f"p_full{buf(u)}"].ready(nth(u)):
-                yield
-            while not B[f"v_full{vstage(u)}"].ready(vuse(u)):
-                yield
-            assert st["V"].get(vstage(u)) == u
-            pipe.append(("PV", u))
-            pipe.append(("commit", o_bar(u)[0]))
-            pipe.append(("commit", f"v_free{vstage(u)}"))
-            yield
-
-        for t in range(jlo - 2, jhi):
-            if t >= jlo:
-                yield from issue_pv(t)
-            if t + 2 < jhi:
-                yield from issue_s(t + 2)
-        pipe.append(("commit", "fin"))
-        while not B["fin"].ready(0):
-            yield
-
-    def softmax():
-        for u in range(jlo, jhi):
-            b = buf(u)
-            while not B[f"s_full{b}"].ready(nth(u)):
-                yield
-            assert st["S"].get(b) == ("S", u), f"tile {u}: S not there"
-            yield
-            st["S"][b] = ("P", u)
-            if u > jlo and rnd.random() < rescale_p:  # the row max grew: O rescaled in place
-                name, n = o_bar(u - 1)
-                while not B[name].ready(n):
-                    yield
-                assert ("PV", u - 1) in done, "rescale before the previous P.V completed"
-                assert not any(op[0] == "PV" for op in pipe), "rescale under a queued P.V"
-            if zeroing and u in zero_needed:
-                while not B[f"v_full{vstage(u)}"].ready(vuse(u)):
-                    yield
-                st["zeroed"].add(u)
-            B[f"p_full{b}"].arrive()
-            yield
-        if jhi > jlo:
-            name, n = o_bar(jhi - 1)
-            while not B[name].ready(n):
-                yield
-            assert all(("PV", u) in done for u in range(jlo, jhi)), "epilogue before the last P.V"
-
-    def pipe_step():
-        op = pipe.pop(0)
-        if op[0] == "commit":
-            B[op[1]].arrive()
-            return
-        kind, u = op
-        assert st["q"], "MMA before Q landed"
-        b = buf(u)
-        if kind == "S":
-            assert st["K"].get(kstage(u)) == u, f"S of tile {u} reads a reloaded K stage"
-            cur = st["S"].get(b)
-            assert cur is None or cur[0] == "P" and ("PV", cur[1]) in done, \
-                f"S of tile {u} over an unread tile {cur}"
-            st["S"][b] = ("S", u)
-        else:
-            assert st["S"].get(b) == ("P", u), f"P.V of tile {u} without its P"
-            assert u not in zero_needed or u in st["zeroed"], f"P.V of tile {u} reads unzeroed V rows"
-        done.add((kind, u))
-
-    roles = {"tma_k": tma_k(), "tma_v": tma_v(), "mma": mma(), "sm": softmax()}
-    steps = 0
-    while roles or pipe or inflight:
-        choice = rnd.choice(list(roles) + ["pipe"] * bool(pipe) + ["copy"] * bool(inflight))
-        if choice == "pipe":
-            pipe_step()
-        elif choice == "copy":
-            # copies land in any order (each has its own barrier)
-            bar, kind, j = inflight.pop(rnd.randrange(len(inflight)))
-            if kind == "Q":
-                st["q"] = True
-            else:
-                st[kind][kstage(j) if kind == "K" else vstage(j)] = j
-            B[bar].arrive()
-        else:
-            try:
-                next(roles[choice])
-            except StopIteration:
-                del roles[choice]
-        steps += 1
-        assert steps < 400000, f"deadlock: roles {list(roles)} waiting, queue {pipe[:2]}"
-    assert B["fin"].done == 1
-    assert all(("PV", u) in done for u in range(jlo, jhi))
-
-
-Q1_SHAPES = [(C, cached, row0, W)
-             for C in (1, 100, 127, 128, 129, 255, 256, 300, 512)
-             for cached in (0, 5, 127, 128, 300, 1000)
-             for row0 in (0, 128, 384) if row0 < C
-             for W in (0, 1, 64, 128, 200, 1024)]
-
-
-def test_1q_geometry_matches_the_bounds():
-    # the tile range covers exactly the rows' visible keys
-    for C, cached, row0, W in Q1_SHAPES:
-        (jlo, jhi), chunk_lo, ctx = geometry_1q(C, cached, row0, W)
-        rows = min(ROWS, C - row0)
-        first, last = cached + row0, cached + row0 + rows - 1
-        lo = max(0, first - W + 1) if W > 0 else 0
-        assert jlo * KEYS <= lo < (jlo + 1) * KEYS
-        assert (jhi - 1) * KEYS <= last < jhi * KEYS <= -(-ctx // KEYS) * KEYS
-
-
-@pytest.mark.parametrize("shape", Q1_SHAPES[::3])
-def test_1q_protocol_has_no_deadlock_alias_or_hazard(shape):
-    for seed in range(4):
-        for p in (0.0, 0.3, 1.0):  # how often a row max grows past the rescale bound
-            run_1q(*shape, seed, rescale_p=p)
-
-
-@pytest.mark.parametrize("plant", ["shared_o_barrier", "no_zeroing", "k_freed_early"])
-def test_1q_model_catches_planted_mistakes(plant):
-    # one o_full for both S buffers lets a parity wait see a phase two
-    # behind; a V tile left unzeroed is read by its P.V; a K stage released
-    # before its S is queued is reloaded under it: the model must say so
-    kw = {"shared_o_barrier": dict(o_per_buffer=False), "no_zeroing": dict(zeroing=False),
-          "k_freed_early": dict(free_k_early=True)}[plant]
-    with pytest.raises(AssertionError):
-        for seed in range(20):
-            run_1q(1024 if plant != "no_zeroing" else 100, 300 if plant != "no_zeroing" else 5,
-                   0, 0, seed, rescale_p=0.3, **kw)
