@@ -600,14 +600,16 @@ def run_ours(args, rank, world):
         comp.wait_stream(down_s)
 
     # the steps, uploads and downloads included, captured as CUDA graphs of
-    # up to 8 steps (the host issue cost of a step's dozen stream operations
+    # up to 32 steps (the host issue cost of a step's dozen stream operations
     # would otherwise exceed a short step's device time); replays of one
-    # graph serialise on the stream, so consecutive graphs do not overlap
+    # graph serialise on the stream, so the upload/download pipeline drains
+    # once per graph: the longer the graph, the less that costs per step
     comp = torch.cuda.current_stream()
     e2e_graphs = {}
     if args.graph:
         side = torch.cuda.Stream()
-        for n in sorted({min(8, K), K % min(8, K)} - {0}):
+        G = min(32, K)
+        for n in sorted({G, K % G} - {0}):
             g = torch.cuda.CUDAGraph()
             side.wait_stream(comp)
             with torch.cuda.stream(side):
