@@ -343,6 +343,7 @@ class Runner:
             qsl = d.query_start_loc.cpu()
             self.max_q = int((qsl[1:] - qsl[:-1]).max())
         self._calls = self.calls()
+        self.side = None  # second stream of a mixed step
 
     def launches_per_step(self) -> int:
         n = 1  # reshape_and_cache
@@ -390,8 +391,23 @@ class Runner:
 
     def step(self, ev=None, calls=None, stream=None):
         """One pass; ``ev`` maps a call's name ("reshape", "prefill",
-        "decode") to (start, end) events recorded around it."""
+        "decode") to (start, end) events recorded around it. Untimed per
+        call, a mixed step's prefill and decode go on two streams: both read
+        the cache the scatter just wrote and nothing of each other, so the
+        GPU may run them side by side (each grid's last wave leaves SMs the
+        other can use)."""
+        import torch
         c = calls or self._calls
+        if ev is None and "prefill" in c and "decode" in c:
+            main = stream if stream is not None else torch.cuda.current_stream()
+            if self.side is None:
+                self.side = torch.cuda.Stream()
+            c["reshape"](main)
+            self.side.wait_stream(main)
+            c["prefill"](self.side)
+            c["decode"](main)
+            main.wait_stream(self.side)
+            return
         for name in ("reshape", "prefill", "decode"):
             if name in c:
                 if ev is not None and name in ev:
