@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         for (int x = 0; x < kPfQTiles; ++x) {
             mbar_init(smem_u32(&bars->s_full[x]), 1);
-            mbar_init(smem_u32(&bars->p_full[x]), 128);
+            mbar_init(smem_u32(&bars->p_full[x]), 4);  // one arrive per softmax warp
             mbar_init(smem_u32(&bars->o_full[x]), 1);
         }
         mbar_init(smem_u32(&bars->fin), 1);
@@ -402,11 +402,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (lane == 0) {
             constexpr uint32_t kIdQK = f16_idesc(128, 128, false);
             constexpr uint32_t kIdPV = f16_idesc(128, D, true);
-            auto issue_s = [&](int x, int j) -> bool {  // S_x = Q_x K_j^T
+            auto wait_k = [&](int j) -> bool {  // K_j landed
                 const int st = (j - jmin) % kPfStages;
-                if (!pf_wait(bars, &bars->k_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
-                             false))
-                    return false;
+                return pf_wait(bars, &bars->k_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
+                               false);
+            };
+            auto wait_v = [&](int j) -> bool {  // V_j landed
+                const int st = (j - jmin) % kPfStages;
+                return pf_wait(bars, &bars->v_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
+                               false);
+            };
+            // S_x = Q_x K_j^T; K_j has landed
+            auto issue_s = [&](int x, int j) {
+                const int st = (j - jmin) % kPfStages;
                 tc_fence_after();
                 const uint32_t q = sQ + x * TB, k = sK + st * TB;
 #pragma unroll
@@ -416,14 +424,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                            sw128_desc(k + koff, 16, 1024), kIdQK, ks > 0);
                 }
                 tc_commit(smem_u32(&bars->s_full[x]));
-                return true;
             };
-            auto issue_pv = [&](int x, int j) -> bool {  // O_x += P_x V_j
+            // O_x += P_x V_j; V_j has landed, P_x is waited for here
+            auto issue_pv = [&](int x, int j) -> bool {
                 const int st = (j - jmin) % kPfStages;
                 if (!pf_wait(bars, &bars->p_full[x], (j - jlo(x)) & 1, a.timeout_ns, false))
-                    return false;
-                if (!pf_wait(bars, &bars->v_full[st], ((j - jmin) / kPfStages) & 1, a.timeout_ns,
-                             false))
                     return false;
                 tc_fence_after();
                 const uint32_t v = sV + st * TB;
@@ -441,15 +446,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             // order (the tensor core runs one thread's operations in order,
             // so S may reuse the P columns), S of each Q tile that uses tile
             // j+1 (a Q tile whose band starts one tile later starts there)
+            if (ok) ok = wait_k(jmin);
 #pragma unroll
             for (int x = 0; x < kPfQTiles; ++x)
-                if (ok && active(x, jmin)) ok = issue_s(x, jmin);
+                if (ok && active(x, jmin)) issue_s(x, jmin);
             if (ok) tc_commit(smem_u32(&bars->k_free[0]));
             for (int j = jmin; ok && j < jmax; ++j) {
+                // the K and V tiles land long before a softmax hands over its
+                // P: waiting for them first keeps their waits off the path
+                // from P to its multiplication
+                const bool s_next = active(0, j + 1) || active(1, j + 1);
+                ok = wait_v(j) && (!s_next || wait_k(j + 1));
 #pragma unroll
                 for (int x = 0; x < kPfQTiles; ++x) {
                     if (ok && active(x, j)) ok = issue_pv(x, j);
-                    if (ok && active(x, j + 1)) ok = issue_s(x, j + 1);
+                    if (ok && active(x, j + 1)) issue_s(x, j + 1);
                 }
                 if (!ok) break;
                 if (j + 1 < jmax)
@@ -609,8 +620,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
                 fence_proxy_async_smem();
             }
+            // the warp's P stores (and V zeroing) are complete and fenced:
+            // one arrive per warp (128 arrivals on one barrier serialise)
             tc_fence_before();
-            mbar_arrive(smem_u32(&bars->p_full[x]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[x]));
         }
         if (ok && j1 > j0 &&
             pf_wait(bars, &bars->o_full[x], (j1 - j0 - 1) & 1, a.timeout_ns, true)) {

@@ -84,7 +84,7 @@ def run(C, cached, row0, W, seed):
                                                 for s in range(STAGES)]
          + [f"{k}{x}" for k in ("s_full", "o_full") for x in (0, 1)]}
     for x in (0, 1):
-        B[f"p_full{x}"] = Bar(f"p_full{x}", 1)  # 128 arrivals, modelled as one
+        B[f"p_full{x}"] = Bar(f"p_full{x}", 1)  # one arrival per softmax warp, modelled as one
     pipe, done, inflight = [], set(), []
     st = {"K": {}, "V": {}, "q": False, "S": {}, "O": {}, "zero_needed": set(), "zeroed": set()}
     for j in range(jmin, jmax):
@@ -117,29 +117,38 @@ def run(C, cached, row0, W, seed):
         while not B["q_full"].ready(0):
             yield
 
-        def issue_s(x, j):
+        def wait_k(j):
             while not B[f"k_full{stage(j)}"].ready(use(j)):
                 yield
-            assert st["K"].get(stage(j)) == j
+
+        def wait_v(j):
+            while not B[f"v_full{stage(j)}"].ready(use(j)):
+                yield
+
+        def issue_s(x, j):  # K_j was waited for
+            assert st["K"].get(stage(j)) == j, f"S of tile {j} over K stage {st['K']}"
             pipe.append(("S", x, j))
             pipe.append(("commit", f"s_full{x}"))
             yield
 
-        def issue_pv(x, j):
+        def issue_pv(x, j):  # V_j was waited for; P is waited for here
             while not B[f"p_full{x}"].ready(j - ranges[x][0]):
                 yield
-            while not B[f"v_full{stage(j)}"].ready(use(j)):
-                yield
-            assert st["V"].get(stage(j)) == j
+            assert st["V"].get(stage(j)) == j, f"P.V of tile {j} over V stage {st['V']}"
             pipe.append(("PV", x, j))
             pipe.append(("commit", f"o_full{x}"))
             yield
 
+        yield from wait_k(jmin)
         for x in (0, 1):
             if act(x, jmin):
                 yield from issue_s(x, jmin)
         pipe.append(("commit", f"k_free{stage(jmin)}"))
         for j in range(jmin, jmax):
+            # V_j and K_{j+1} first, then each query tile's P
+            yield from wait_v(j)
+            if act(0, j + 1) or act(1, j + 1):
+                yield from wait_k(j + 1)
             for x in (0, 1):
                 if act(x, j):
                     yield from issue_pv(x, j)
