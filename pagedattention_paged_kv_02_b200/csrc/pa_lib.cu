@@ -132,9 +132,6 @@ pa_status launch_decode_f32(const DecodeArgs &a, dim3 grid, cudaStream_t st) {
     return launch_status();
 }
 
-// query rows one prefill CTA covers
-constexpr int kPrefillCtaRows = kPfRows * kPfQTiles;
-
 template <int D, bool WIN>
 pa_status launch_prefill_tc(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                             const CUtensorMap &mv, dim3 grid, cudaStream_t st) {
@@ -661,7 +658,11 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
         return PA_ERR_INVALID_ARG;
-    const long long qtiles = (max_query_len + kPrefillCtaRows - 1) / kPrefillCtaRows;
+    // a CTA's two query tiles: the same 128 rows of two query heads of one KV
+    // head when the group size is even, else 256 consecutive rows of one head
+    const bool pair_heads = (num_q_heads / num_kv_heads) % 2 == 0;
+    const int cta_rows = pair_heads ? kPfRows : kPfRows * kPfQTiles;
+    const long long qtiles = (max_query_len + cta_rows - 1) / cta_rows;
     if (qtiles > 65535 || num_chunks > 65535) return PA_ERR_UNSUPPORTED;
 
     EncodeTiledFn fn = encode_fn();
@@ -697,10 +698,12 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     a.NB = num_blocks;
     a.MB = max_blocks_per_seq;
     a.window = window;
+    a.pair_heads = pair_heads ? 1 : 0;
     a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
-    const dim3 grid((unsigned)num_q_heads, (unsigned)qtiles, (unsigned)num_chunks);
+    const dim3 grid((unsigned)(pair_heads ? num_q_heads / 2 : num_q_heads), (unsigned)qtiles,
+                    (unsigned)num_chunks);
     if (head_dim == 64)
         return window > 0 ? launch_prefill_tc<64, true>(a, mq, mk, mv, grid, stream)
                           : launch_prefill_tc<64, false>(a, mq, mk, mv, grid, stream);

@@ -15,9 +15,12 @@
 // cached+i only; key tiles wholly before a query tile's band are neither
 // loaded nor multiplied.
 //
-// One CTA = two 128-row query tiles (the tcgen05 M) of one query head of one
-// chunk, sharing every K/V tile; keys are processed in tiles of 128. Twelve
-// warps:
+// One CTA = two 128-row query tiles (the tcgen05 M) of one chunk sharing
+// every K/V tile: when the query heads of a KV head come in pairs, the same
+// 128 rows of two query heads of that KV head (both tiles then need the same
+// key tiles and stay interleaved to the end); otherwise 256 consecutive rows
+// of one query head (the second tile needs one key tile more, its diagonal).
+// Keys are processed in tiles of 128. Twelve warps:
 //   warp 8   TMA: both Q tiles once, then each key tile's K and V as
 //            16-token page pieces (128-byte swizzle) gathered through the
 //            block table, one piece per lane, into two-stage K and V rings
@@ -74,6 +77,7 @@ struct PrefillArgs {
     const int32_t *qsl;
     int n_chunks, total_q, H_q, H_kv, group, bs, NB, MB;
     int window;  // > 0: query at position p sees keys p-window+1 .. p only
+    int pair_heads;  // 1: the two query tiles are the same rows of query heads 2x, 2x+1
     int bs_shift;  // log2(bs)
     float scale_log2;
     unsigned long long timeout_ns;
@@ -244,10 +248,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // CTAs start in order of decreasing work (the scheduler hands them out
-    // in launch order): the last chunk first, within it the last query-tile
-    // pair first, every query head of one pair before the next pair
-    const int h = blockIdx.x;
+    // in launch order): the last chunk first, within it the last row tile
+    // first, every query head (pair) of one row tile before the next
     const int tp = (int)gridDim.y - 1 - (int)blockIdx.y;
+    // query head of each tile
+    const int hq0 = a.pair_heads ? 2 * (int)blockIdx.x : (int)blockIdx.x;
+    const int hq1 = a.pair_heads ? hq0 + 1 : hq0;
     const int c = a.n_chunks - 1 - (int)blockIdx.z;
     const int q0 = a.qsl[c];
     const int C = a.qsl[c + 1] - q0;
@@ -260,21 +266,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     // rows past the grid's reach (a chunk longer than max_query_len rounded
     // up to the CTA's rows) would be left unwritten: recorded once per chunk
-    if (C > (int)gridDim.y * kPfRows * kPfQTiles && blockIdx.x == 0 && blockIdx.y == 0 &&
-        threadIdx.x == 0)
+    const int cta_rows = a.pair_heads ? kPfRows : kPfRows * kPfQTiles;
+    if (C > (int)gridDim.y * cta_rows && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         flag_error(PA_ERR_BAD_TABLE);
-    const int row0 = tp * kPfRows * kPfQTiles;  // first query of this CTA within the chunk
+    const int row0 = tp * cta_rows;  // first query of query tile 0 within the chunk
     if (row0 >= C) return;
+    const int row1 = a.pair_heads ? row0 : row0 + kPfRows;  // ... of query tile 1
     const int cached = ctx - C;
     // Rows of each Q tile (a Q tile past the chunk has none) and the K/V
     // tiles [jlo_x, jhi_x) it needs: up to its last row's position, from its
     // first row's band start. Key positions below the chunk's smallest band
     // start (chunk_lo) are never needed: their blocks may have been freed.
     const int rows0 = min(kPfRows, C - row0);
-    const int rows1 = max(0, min(kPfRows, C - row0 - kPfRows));
+    const int rows1 = max(0, min(kPfRows, C - row1));
     const int W = WIN ? a.window : 0;
     const int chunk_lo = W > 0 ? max(0, cached - W + 1) : 0;
-    const int pf0 = cached + row0, pf1 = pf0 + kPfRows;  // first positions
+    const int pf0 = cached + row0, pf1 = cached + row1;  // first positions
     const int jlo0 = (W > 0 ? max(0, pf0 - W + 1) : 0) / kPfKeys;
     const int jlo1 = (W > 0 ? max(0, pf1 - W + 1) : 0) / kPfKeys;
     const int jhi0 = (pf0 + rows0 - 1) / kPfKeys + 1;
@@ -283,7 +290,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     auto jhi = [&](int x) { return x == 0 ? jhi0 : jhi1; };
     auto active = [&](int x, int j) { return j >= jlo(x) && j < jhi(x); };
     const int jmin = jlo0, jmax = max(jhi0, jhi1);  // K/V tiles this CTA streams
-    const int kvh = h / a.group;
+    const int kvh = hq0 / a.group;
 
     const int nq = rows1 > 0 ? 2 : 1;  // Q tiles with rows
     if (warp == 8) {
@@ -310,8 +317,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       __syncwarp();
       if (lane < HALVES * nq) {
           const int x = lane / HALVES, hf = lane % HALVES;
-          tma_load_3d(sQ + x * TB + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64, h,
-                      q0 + row0 + x * kPfRows);
+          tma_load_3d(sQ + x * TB + hf * 16384, &tmq, smem_u32(&bars->q_full), hf * 64,
+                      x == 0 ? hq0 : hq1, q0 + (x == 0 ? row0 : row1));
       }
     }
     if (warp == 9) {
@@ -477,11 +484,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // -------------------------------------------------------- softmax
         const int x = warp >> 2;                      // Q tile of this warpgroup
         const int r = threadIdx.x & 127;              // row of the tile == lane
-        const int i = row0 + x * kPfRows + r;         // query index in the chunk
+        const int xrow0 = x == 0 ? row0 : row1;       // first row of the tile
+        const int i = xrow0 + r;                      // query index in the chunk
         const bool row_valid = i < C;
         const int pos = cached + min(i, C - 1);       // keys <= pos are visible
         const int lo = W > 0 ? pos - W + 1 : 0;       // ... and keys >= lo
-        const int pos_first = cached + row0 + x * kPfRows;  // smallest pos of the tile
+        const int pos_first = cached + xrow0;         // smallest pos of the tile
         const int lo_last = W > 0 ? pos_first + (x == 0 ? rows0 : rows1) - W : 0;  // largest lo
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + x * 128 + lane_off;
@@ -630,7 +638,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             pf_wait(bars, &bars->o_full[x], (j1 - j0 - 1) & 1, a.timeout_ns, true)) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + h) * D;
+            __nv_bfloat16 *dst = a.out + ((size_t)(q0 + i) * a.H_q + (x == 0 ? hq0 : hq1)) * D;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t v[32];

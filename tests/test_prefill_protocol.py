@@ -30,13 +30,15 @@ ROWS = KEYS = 128
 STAGES = 2
 
 
-def geometry(C, cached, row0, W):
+def geometry(C, cached, row0, W, pair=False):
     """Tile ranges [jlo_x, jhi_x) of the two query tiles of a CTA (the
-    kernel's formulas), the chunk's lowest needed key, and the context."""
+    kernel's formulas), the chunk's lowest needed key, and the context.
+    pair: the two tiles are the same rows of two query heads."""
+    row1 = row0 if pair else row0 + ROWS
     rows0 = min(ROWS, C - row0)
-    rows1 = max(0, min(ROWS, C - row0 - ROWS))
+    rows1 = max(0, min(ROWS, C - row1))
     pf0 = cached + row0
-    pf1 = pf0 + ROWS
+    pf1 = cached + row1
     jlo0 = (max(0, pf0 - W + 1) if W > 0 else 0) // KEYS
     jlo1 = (max(0, pf1 - W + 1) if W > 0 else 0) // KEYS
     jhi0 = (pf0 + rows0 - 1) // KEYS + 1
@@ -66,10 +68,10 @@ class Bar:
         return hw
 
 
-def run(C, cached, row0, W, seed):
+def run(C, cached, row0, W, seed, pair=False):
     """One seeded interleaving of the four roles for one CTA's geometry."""
     rnd = random.Random(seed)
-    (r0, r1), chunk_lo, ctx = geometry(C, cached, row0, W)
+    (r0, r1), chunk_lo, ctx = geometry(C, cached, row0, W, pair)
     ranges = [r0, r1]
     act = lambda x, j: ranges[x][0] <= j < ranges[x][1]
     jmin, jmax = r0[0], max(r0[1], r1[1])
@@ -233,6 +235,12 @@ SHAPES = [(C, cached, row0, W)
           for cached in (0, 5, 127, 128, 300, 1000)
           for row0 in (0, 256) if row0 < C
           for W in (0, 1, 64, 128, 200, 1024)]
+# head-paired CTAs: both tiles cover the same 128 rows
+PAIR_SHAPES = [(C, cached, row0, W)
+               for C in (1, 100, 128, 129, 300, 512)
+               for cached in (0, 5, 128, 1000)
+               for row0 in (0, 128, 384) if row0 < C
+               for W in (0, 1, 64, 200, 1024)]
 
 
 def test_geometry_matches_the_causal_bound():
@@ -253,6 +261,19 @@ def test_geometry_matches_the_causal_bound():
 def test_protocol_has_no_deadlock_alias_or_hazard(shape):
     for seed in range(6):
         run(*shape, seed)
+
+
+@pytest.mark.parametrize("shape", PAIR_SHAPES[::3])
+def test_head_paired_protocol_has_no_deadlock_alias_or_hazard(shape):
+    for seed in range(6):
+        run(*shape, seed, pair=True)
+
+
+def test_head_pairs_share_one_key_range():
+    # same rows: both query tiles stream exactly the same key tiles
+    for C, cached, row0, W in PAIR_SHAPES:
+        (r0, r1), _, _ = geometry(C, cached, row0, W, pair=True)
+        assert r0 == r1
 
 
 def test_model_catches_a_missing_wait():
