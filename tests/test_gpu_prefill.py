@@ -51,10 +51,14 @@ def oracle_prefill(batch, k, v, select=None):
 
 CASES = [
     # (cached per chunk, chunk lengths), H_q, H_kv, bs
+    # groups of even size put two query heads' same rows in one CTA, odd ones
+    # (1, 3) two consecutive 128-row tiles of one head
     (([0, 0, 100, 37], [5, 128, 129, 300]), 8, 2, 16),
     (([1000, 300, 0], [64, 1, 257]), 4, 4, 32),
     (([250, 700], [200, 77]), 8, 1, 64),
     (([16, 127, 128], [16, 1, 129]), 32, 8, 16),
+    (([0, 333], [384, 130]), 4, 2, 16),   # group 2: each head pair is a whole group
+    (([40, 0], [300, 129]), 6, 2, 32),    # group 3: row pairs
 ]
 
 
