@@ -702,8 +702,17 @@ static pa_status prefill_impl(void *out, const void *q, const void *k_cache, con
     a.bs_shift = __builtin_ctz((unsigned)block_size);
     a.scale_log2 = scale * 1.4426950408889634f;
     a.timeout_ns = kWaitTimeoutNs;
-    const dim3 grid((unsigned)(pair_heads ? num_q_heads / 2 : num_q_heads), (unsigned)qtiles,
-                    (unsigned)num_chunks);
+    // persistent: one CTA per SM (its 512 TMEM columns) deals the items out
+    a.gx = pair_heads ? num_q_heads / 2 : num_q_heads;
+    a.gy = (int)qtiles;
+    const long long n_items = (long long)a.gx * a.gy * num_chunks;
+    if (n_items > (1LL << 30)) return PA_ERR_UNSUPPORTED;
+    a.n_items = (int)n_items;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return PA_ERR_CUDA;
+    const dim3 grid((unsigned)std::min<long long>(n_items, sms));
     if (head_dim == 64)
         return window > 0 ? launch_prefill_tc<64, true>(a, mq, mk, mv, grid, stream)
                           : launch_prefill_tc<64, false>(a, mq, mk, mv, grid, stream);
