@@ -400,17 +400,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             PfItem w;
             if (!pf_item<WIN>(a, it, lane == 0, w)) continue;
             const int32_t *trow = a.block_tables + (size_t)w.c * a.MB;
-            auto piece_id = [&](int j) {
+            // the table entry of this lane's piece of key tile j (-1: no
+            // piece); read ahead of its use and checked only there, so that
+            // waiting for the read never holds up the copies before it
+            auto piece_raw = [&](int j) {
                 const int key = j * kPfKeys + s16 * 16;
-                int id = -1;
-                if (lane < 8 * HALVES && key < w.ctx && (!WIN || key + 15 >= w.chunk_lo)) {
-                    id = __ldg(trow + (key >> a.bs_shift));
-                    if (id < 0 || id >= a.NB) {
-                        flag_error(PA_ERR_BAD_TABLE);
-                        id = -1;
-                    }
+                return lane < 8 * HALVES && key < w.ctx && (!WIN || key + 15 >= w.chunk_lo)
+                           ? __ldg(trow + (key >> a.bs_shift))
+                           : -1;
+            };
+            auto checked = [&](int raw, int j) {  // -1 for no piece or a bad id (recorded)
+                const int key = j * kPfKeys + s16 * 16;
+                const bool piece =
+                    lane < 8 * HALVES && key < w.ctx && (!WIN || key + 15 >= w.chunk_lo);
+                if (piece && (raw < 0 || raw >= a.NB)) {
+                    flag_error(PA_ERR_BAD_TABLE);
+                    return -1;
                 }
-                return id;
+                return piece ? raw : -1;
             };
             auto issue = [&](uint32_t dst, const CUtensorMap *map, uint64_t *bar, int j, int id) {
                 const int n = __popc(__ballot_sync(0xffffffffu, id >= 0));
@@ -420,7 +427,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     tma_load_4d(dst + half * 16384 + s16 * 2048, map, smem_u32(bar), half * 64,
                                 (j * kPfKeys + s16 * 16) & (a.bs - 1), w.kvh, id);
             };
-            int id = piece_id(w.jmin);
+            int raw = piece_raw(w.jmin);
             // the Q tiles, once the previous item's last S has read them
             if (qn > 0 && !pf_wait(bars, &bars->q_free, (qn - 1) & 1, a.timeout_ns, true)) {
                 ok = false;
@@ -435,8 +442,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             x == 0 ? w.hq0 : w.hq1, w.q0 + (x == 0 ? w.row0 : w.row1));
             }
             ++qn;
+            int id = checked(raw, w.jmin);
             for (int j = w.jmin; j < w.jmax; ++j, ++g) {
-                const int nid = j + 1 < w.jmax ? piece_id(j + 1) : -1;
+                const int nraw = j + 1 < w.jmax ? piece_raw(j + 1) : -1;
                 const int st = g % kPfStages;
                 const uint32_t use = g / kPfStages;
                 if (use > 0 &&
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
                 issue(sV + st * TB, &tmv, &bars->v_full[st], j, id);
                 v_issued = g + 1;
-                id = nid;
+                if (j + 1 < w.jmax) id = checked(nraw, j + 1);
             }
         }
         if (bars->abort && lane == 0) {  // let copies already in flight land
