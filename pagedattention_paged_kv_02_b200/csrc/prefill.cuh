@@ -751,10 +751,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv,
                                        __uint_as_float(v[2 * e + 1]) * inv);
                 if (row_valid) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 32);
+                    // whole 32-byte sectors: a thread's row is 8 KB away from
+                    // its neighbours', so 16-byte stores would each write half
+                    // a sector, twice as many store instructions
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                    for (int e = 0; e < 2; ++e)
+                        asm volatile(
+                            "st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                                dst + cc * 32 + e * 16),
+                            "r"(o[8 * e]), "r"(o[8 * e + 1]), "r"(o[8 * e + 2]), "r"(o[8 * e + 3]),
+                            "r"(o[8 * e + 4]), "r"(o[8 * e + 5]), "r"(o[8 * e + 6]),
+                            "r"(o[8 * e + 7])
+                            : "memory");
                 }
             }
         }
