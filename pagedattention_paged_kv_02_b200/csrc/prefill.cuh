@@ -15,16 +15,19 @@
 // cached+i only; key tiles wholly before a query tile's band are neither
 // loaded nor multiplied.
 //
-// One CTA = two 128-row query tiles (the tcgen05 M) of one chunk sharing
+// Work item = two 128-row query tiles (the tcgen05 M) of one chunk sharing
 // every K/V tile: when the query heads of a KV head come in pairs, the same
 // 128 rows of two query heads of that KV head (both tiles then need the same
 // key tiles and stay interleaved to the end); otherwise 256 consecutive rows
 // of one query head (the second tile needs one key tile more, its diagonal).
-// Keys are processed in tiles of 128. Twelve warps:
-//   warp 8   TMA: both Q tiles once, then each key tile's K and V as
-//            16-token page pieces (128-byte swizzle) gathered through the
-//            block table, one piece per lane, into two-stage K and V rings
-//            with full/free barriers.
+// Keys are processed in tiles of 128. The kernel is persistent: one CTA per
+// SM works through its share of the items (see prefill_tc_kernel), and
+// across items the K/V rings and barrier phases carry on. Twelve warps:
+//   warp 8   TMA: an item's Q tiles once the previous item's last S has read
+//            the Q buffers, then each key tile's K and V as 16-token page
+//            pieces (128-byte swizzle) gathered through the block table, one
+//            piece per lane (block ids read one key tile ahead), into
+//            two-stage K and V rings with full/free barriers.
 //   warp 9   MMA (one lane) and the tensor-memory allocation: S_x = Q_x K^T
 //            (8 x 128x128x16, both operands K-major in shared memory) into
 //            tensor-memory columns [128x, 128x+128); O_x += P_x V with P_x
@@ -32,7 +35,8 @@
 //            V MN-major in shared memory, into columns [256+128x, ...).
 //            After P_x.V_j it issues S_x for tile j+1 (the tensor core runs
 //            one thread's operations in order), so one query tile's softmax
-//            overlaps the other tile's multiplications.
+//            overlaps the other tile's multiplications; the next item's
+//            first S follows the current item's last P.V.
 //   warps 0-3 / 4-7   softmax of query tile 0 / 1: thread r owns row r
 //            (tensor-memory lane r): row max, exp2, the running sum, bf16 P
 //            written back over the consumed S columns; O is rescaled in
@@ -50,7 +54,7 @@
 namespace pa {
 
 constexpr int kPfRows = 128;      // query rows per Q tile (the tcgen05 M)
-constexpr int kPfQTiles = 2;      // Q tiles per CTA, sharing every K/V tile
+constexpr int kPfQTiles = 2;      // Q tiles per item, sharing every K/V tile
 constexpr int kPfKeys = 128;      // keys per K/V tile
 constexpr int kPfStages = 2;      // K and V ring depth
 constexpr int kPfThreads = 384;   // 2 softmax warpgroups + a control warpgroup
