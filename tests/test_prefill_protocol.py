@@ -398,3 +398,49 @@ def test_model_catches_an_early_q_reload():
                 run([(512, 1000, 0, 0, True), (512, 1000, 128, 0, True)], seed)
     finally:
         Bar.ready = old
+
+
+def item_of(r, b, G):
+    """CTA b's r-th item in the persistent kernel's dealing: rounds of one item
+    per CTA, every other round reversed."""
+    return r * G + ((G - 1 - b) if r & 1 else b)
+
+
+@pytest.mark.parametrize("n_items,G", [(1, 148), (147, 148), (148, 148), (149, 148), (512, 148),
+                                       (1152, 148), (5, 3), (7, 1), (4096, 132)])
+def test_dealing_gives_every_item_to_one_cta(n_items, G):
+    G = min(G, n_items)  # the host launches min(items, SMs) CTAs
+    seen = []
+    for b in range(G):
+        r = 0
+        while item_of(r, b, G) < n_items:
+            seen.append(item_of(r, b, G))
+            r += 1
+    assert sorted(seen) == list(range(n_items))
+
+
+def test_dealing_balances_the_mixed_launch():
+    """The mixed launch's 512 items dealt over 148 CTAs (cost of an item: its
+    key tiles plus 0.3 of a tile for its start and epilogue): the busiest CTA
+    within 4 % of the mean, no worse than a greedy longest-first assignment."""
+    import heapq
+    cached = [round(i * 4096 / 7) for i in range(8)]
+    work = []  # in item order: chunks from the last, row tiles from the last, heads fastest
+    for c in reversed(cached):
+        for rt in reversed(range(4)):
+            pf = c + rt * ROWS
+            work += [(pf + ROWS - 1) // KEYS + 1 + 0.3] * 16
+    G = 148
+    load = [0.0] * G
+    for b in range(G):
+        r = 0
+        while item_of(r, b, G) < len(work):
+            load[b] += work[item_of(r, b, G)]
+            r += 1
+    heap = [(0.0, b) for b in range(G)]
+    for w in sorted(work, reverse=True):
+        l, b = heapq.heappop(heap)
+        heapq.heappush(heap, (l + w, b))
+    greedy = max(l for l, _ in heap)
+    assert max(load) <= 1.04 * sum(load) / G
+    assert max(load) <= greedy * 1.001
