@@ -300,9 +300,10 @@ PA_API pa_status pa_decode_sliding_window(void *out, const void *q, const void *
  *                     query_start_loc), with context_lens[c] < C_c or above
  *                     max_blocks_per_seq*block_size is skipped and recorded
  *                     as PA_ERR_BAD_TABLE.
- *   max_query_len     host-side upper bound of every C_c. The launch covers
- *                     max_query_len rounded up to a multiple of 128 rows per
- *                     chunk; the rows of a longer chunk past that are left
+ *   max_query_len     host-side upper bound of every C_c. The work covers
+ *                     max_query_len rounded up to whole row tiles per chunk
+ *                     (128 rows when num_q_heads / num_kv_heads is even, else
+ *                     256); the rows of a longer chunk past that are left
  *                     unwritten and the chunk is recorded as PA_ERR_BAD_TABLE.
  * bf16 with head_dim 64 or 128 (the tcgen05 tensor-core path), at most
  * 65535 chunks and max_query_len at most 65535 * 128; anything else returns

@@ -144,8 +144,8 @@ def test_prefill_host_checks(L):
     b = list(base)
     b[7] = 0
     assert f(*b) == pa.PA_OK
-    # the grid is (query head, query tile, chunk): at most 65535 tiles of 128 queries
-    # and 65535 chunks; any number of query heads
+    # work items are (query head or head pair, row tile, chunk): at most 65535 row
+    # tiles and 65535 chunks; any number of query heads
     b = list(base)
     b[8], b[9] = 65536 * 256, 65536 * 256
     assert f(*b) == pa.PA_ERR_UNSUPPORTED
